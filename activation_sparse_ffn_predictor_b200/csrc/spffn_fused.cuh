@@ -1,0 +1,9 @@
+// Persistent whole-stack decode kernel (spffn_fused.cu).
+#pragma once
+#include "spffn_internal.cuh"
+
+namespace spffn {
+bool fused_decode_supported(spffn_ctx* const* layers, int L, int B);
+cudaError_t launch_fused_decode(spffn_ctx* const* layers, int L, const void* x_in, int B, void* x_out, float* y,
+                                int32_t* counts, cudaStream_t st);
+}  // namespace spffn

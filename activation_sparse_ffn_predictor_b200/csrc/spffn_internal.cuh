@@ -1,0 +1,121 @@
+// Internal definitions shared by the spffn kernels and the C-ABI glue.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include "../../include/spffn.h"
+
+namespace spffn {
+
+// Device error word bits (latched with atomicOr, read by spffn_last_device_error).
+enum : uint32_t {
+    ERR_COUNT_CLAMPED = 1u << 0,   // caller-supplied count > n (clamped to n) or < 0 (clamped to 0)
+    ERR_IDX_RANGE = 1u << 1,       // a neuron table entry outside [0, n) (skipped)
+    ERR_BARRIER_TIMEOUT = 1u << 2, // a grid barrier wait hit its iteration limit
+    ERR_PIPE_TIMEOUT = 1u << 3,    // a copy-completion wait hit its iteration limit
+};
+
+constexpr int kMaxBatch = 32;
+constexpr int kCtlBytes = 1024;    // control block at the head of the workspace
+
+// Control block (u32 words) at the start of every workspace.
+struct Ctl {
+    uint32_t err;          // latched error bits
+    uint32_t ticket;       // reserved
+    uint32_t pad0[14];
+    uint32_t barrier[64];  // grid-barrier counters (persistent kernels)
+};
+
+struct Layout {
+    size_t ctl, h, mask, wcount, partial, xbuf, ybuf, idx, count, total;
+    int S;  // number of FFN partial sums
+};
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline Layout make_layout(const spffn_config& c, int S) {
+    Layout L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
+    L.S = S;
+    L.ctl = take(kCtlBytes);
+    L.h = take((size_t)c.max_batch * c.H * sizeof(float));
+    L.mask = take((size_t)(c.n / 32) * sizeof(uint32_t));
+    L.wcount = take((size_t)(c.n / 32) * sizeof(uint32_t));
+    L.partial = take((size_t)S * c.max_batch * c.d * sizeof(float));
+    L.xbuf = take((size_t)2 * c.max_batch * c.d * 2);
+    L.ybuf = take((size_t)c.max_batch * c.d * sizeof(float));
+    L.idx = take((size_t)c.n * sizeof(int32_t));
+    L.count = take(256);
+    L.total = off;
+    return L;
+}
+
+}  // namespace spffn
+
+struct spffn_ctx {
+    spffn_config cfg;
+    spffn_weights w;
+    char* ws;
+    size_t ws_bytes;
+    spffn::Layout lay;
+    int num_sms;
+    int device;
+
+    spffn::Ctl* ctl() const { return reinterpret_cast<spffn::Ctl*>(ws + lay.ctl); }
+    float* h() const { return reinterpret_cast<float*>(ws + lay.h); }
+    uint32_t* mask() const { return reinterpret_cast<uint32_t*>(ws + lay.mask); }
+    uint32_t* wcount() const { return reinterpret_cast<uint32_t*>(ws + lay.wcount); }
+    float* partial() const { return reinterpret_cast<float*>(ws + lay.partial); }
+    void* xbuf(int i) const { return ws + lay.xbuf + (size_t)i * cfg.max_batch * cfg.d * 2; }
+    float* ybuf() const { return reinterpret_cast<float*>(ws + lay.ybuf); }
+    int32_t* idx() const { return reinterpret_cast<int32_t*>(ws + lay.idx); }
+    int32_t* count() const { return reinterpret_cast<int32_t*>(ws + lay.count); }
+};
+
+namespace spffn {
+
+// ---------------------------------------------------------------------------
+// storage-dtype helpers
+template <typename T> struct DT;
+template <> struct DT<__half> {
+    static __device__ __forceinline__ float f(__half v) { return __half2float(v); }
+    static __device__ __forceinline__ __half r(float v) { return __float2half_rn(v); }
+    static __device__ __forceinline__ float2 f2(uint32_t u) {
+        __half2 h = *reinterpret_cast<__half2*>(&u);
+        return __half22float2(h);
+    }
+};
+template <> struct DT<__nv_bfloat16> {
+    static __device__ __forceinline__ float f(__nv_bfloat16 v) { return __bfloat162float(v); }
+    static __device__ __forceinline__ __nv_bfloat16 r(float v) { return __float2bfloat16_rn(v); }
+    static __device__ __forceinline__ float2 f2(uint32_t u) {
+        __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&u);
+        return __bfloat1622float2(h);
+    }
+};
+
+// 8 storage elements (one 16-byte vector) -> 8 floats
+template <typename T>
+__device__ __forceinline__ void unpack8(const uint4& v, float* f) {
+    float2 a = DT<T>::f2(v.x), b = DT<T>::f2(v.y), c = DT<T>::f2(v.z), d = DT<T>::f2(v.w);
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y; f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
+}
+
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+    uint4 r;
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ void latch(uint32_t* err, uint32_t bits) { atomicOr(err, bits); }
+
+}  // namespace spffn

@@ -1,0 +1,16 @@
+// Launchers for the per-phase kernels (spffn_kernels.cu).
+#pragma once
+#include "spffn_internal.cuh"
+
+namespace spffn {
+cudaError_t launch_predict(const spffn_ctx& c, const void* x, int B, int32_t* idx, int32_t* count,
+                           int32_t* count2, cudaStream_t st);
+cudaError_t launch_forward(const spffn_ctx& c, const void* x, int B, const int32_t* idx, const int32_t* count,
+                           float* y, cudaStream_t st);
+cudaError_t launch_chain(const spffn_ctx& c, const void* x, const float* y, int B, void* xn, cudaStream_t st);
+cudaError_t launch_profile(const spffn_ctx& c, const void* X, int T, uint32_t* counts, cudaStream_t st);
+cudaError_t launch_permute_rows(const void* src, void* dst, int rows, int row_bytes, const int32_t* perm,
+                                cudaStream_t st);
+cudaError_t launch_permute_vec(const void* src, void* dst, int count, const int32_t* perm, cudaStream_t st);
+int ffn_token_group(const spffn_ctx& c);
+}  // namespace spffn

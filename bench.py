@@ -1,0 +1,404 @@
+#!/usr/bin/env python
+"""Sparse-FFN decode benchmark: tokens/s per layer stack and achieved HBM GB/s
+over the bytes the path touches, on seeded synthetic power-law-sparse inputs.
+
+Default workload: the OPT-6.7B-shaped stack (32 layers, d=4096, n=16384,
+predictor H=1024, fp16 weights, batch 1, mean activation rate 5%, alpha=1.2),
+weights generated in HBM, hot-first reordered offline (untimed), then K decode
+steps timed with CUDA events.  One step = spffn_decode over all layers:
+predictor (two GEMVs + threshold + compaction), sparse FC1/FC2 with the
+deterministic split reduction, and the chaining into the next layer.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1] [--impl ours|reference]
+
+Under torchrun each rank runs its own replica on its own decode stream
+(independent requests: weak scaling, no data-path collective); the reported time
+is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workload as wl  # noqa: E402
+
+METRIC = "sparse-FFN decode tokens/s per layer-stack"
+UNIT = "tokens/s"
+PROFILE_TOKENS = 256
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (host-side only: barrier and max-over-ranks timing)
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def dist_init(world, backend):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return world > 1
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def rank_seed(rank: int) -> int:
+    """Each replica decodes its own request stream."""
+    return 1 + rank
+
+
+# ---------------------------------------------------------------------------
+# bytes the path touches (algorithmic; x, y and L2-resident partials excluded)
+def predictor_bytes(cfg) -> int:
+    return 2 * (cfg.H * cfg.d + cfg.n * cfg.H) + 2 * cfg.n + 2 * cfg.H
+
+
+def ffn_bytes_per_neuron(cfg) -> int:
+    return 4 * cfg.d + 2 + 4          # W1 row + W2T row + b1 + table entry
+
+
+def step_bytes(cfg, counts_sum: int, layers: int) -> int:
+    return layers * predictor_bytes(cfg) + counts_sum * ffn_bytes_per_neuron(cfg)
+
+
+# ---------------------------------------------------------------------------
+class Clocks:
+    """Samples SM clocks and throttle reasons (NVML, read-only) during the timed region."""
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.index = index
+        self.period = period_s
+        self.rows = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByIndex(self.index)
+            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            while not self._stop.is_set():
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.rows.append((sm, mx, rs))
+                self._stop.wait(self.period)
+        except Exception as e:  # NVML missing: leave the record empty and say why
+            self.error = repr(e)
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join(timeout=10)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "error": getattr(self, "error", "no samples")}
+        bits = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+                "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+        reasons = sorted({k for _, _, r in self.rows for k, b in bits.items() if r & b})
+        return {"sm_mhz": statistics.median(r[0] for r in self.rows), "sm_max_mhz": max(r[1] for r in self.rows),
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+def build_stack(cfg, layers, device, rate=None, reorder=True, log=print):
+    """All layers in HBM; hot-first reordered from an offline profile (untimed)."""
+    import torch
+    import activation_sparse_ffn_predictor_b200 as sp
+    out = []
+    for l in range(layers):
+        dl = wl.device_layer(cfg, l, device=device, rate=rate)
+        L = sp.Layer.from_device_layer(dl, max_batch=cfg.batch)
+        if reorder:
+            Xp = wl.to_torch(wl.tokens(cfg, PROFILE_TOKENS, aux=l, tensor=wl.T_XPROF), cfg, device)
+            counts = torch.zeros(cfg.n, dtype=torch.int32, device=device)
+            L.profile_counts(Xp, counts)
+            perm = sp.reorder(counts.cpu().numpy().astype(np.uint32))
+            pt = torch.from_numpy(perm).to(device)
+            for name in ("W1", "W2T", "Wp2"):
+                src = getattr(dl, name)
+                dst = torch.empty_like(src)
+                sp.permute_rows(src, dst, pt)
+                setattr(dl, name, dst)
+                del src
+            for name in ("b1", "bp2"):
+                src = getattr(dl, name)
+                dst = torch.empty_like(src)
+                sp.permute_vector(src, dst, pt)
+                setattr(dl, name, dst)
+            L.close()
+            L = sp.Layer.from_device_layer(dl, max_batch=cfg.batch)
+        out.append((dl, L))
+    torch.cuda.synchronize()
+    return out
+
+
+def run_ours(args, cfg, world, rank, local):
+    import torch
+    import activation_sparse_ffn_predictor_b200 as sp
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist_init(world, "nccl")
+    L = cfg.layers
+    stack = build_stack(cfg, L, device, rate=args.rate)
+    layers = [s[1] for s in stack]
+    B, K, W = cfg.batch, args.steps, args.warmup
+    seed = rank_seed(rank)
+    dt = torch.bfloat16 if cfg.bf16 else torch.float16
+    xs = torch.stack([wl.to_torch(wl.tokens(cfg, B, aux=s, seed=seed), cfg, device) for s in range(K + W)])
+    x_in = torch.empty(B, cfg.d, dtype=dt, device=device)
+    x_out = torch.empty(B, cfg.d, dtype=dt, device=device)
+    y = torch.empty(B, cfg.d, dtype=torch.float32, device=device)
+    counts = torch.zeros(L, dtype=torch.int32, device=device)
+    hist = torch.zeros(K + W, L, dtype=torch.int32, device=device)
+    stream = torch.cuda.Stream(device)
+
+    def one_step():
+        sp.decode(layers, x_in, x_out, y, counts, stream=stream)
+
+    # CUDA graph of one decode step (removes host launch cost from the timed region)
+    with torch.cuda.stream(stream):
+        one_step()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        one_step()
+    launches_per_step = args.launches_per_step or _count_launches_per_step(L)
+
+    with torch.cuda.stream(stream):
+        for s in range(W):
+            x_in.copy_(xs[s])
+            g.replay()
+            hist[s].copy_(counts)
+    stream.synchronize()
+    barrier(world, device)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(local) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for s in range(K):
+                x_in.copy_(xs[W + s])
+                ev[s][0].record(stream)
+                g.replay()
+                ev[s][1].record(stream)
+                hist[W + s].copy_(counts)
+            e1.record(stream)
+        stream.synchronize()
+    torch.cuda.synchronize()
+    barrier(world, device)
+    total_ms = e0.elapsed_time(e1)
+    kernel_ms = [a.elapsed_time(b) for a, b in ev]
+    t_max = max_over_ranks(total_ms, world, device)
+    ks = hist[W:].cpu().numpy()
+    bytes_per_step = [step_bytes(cfg, int(ks[s].sum()), L) for s in range(K)]
+    peak, peak_kind = measured_peaks()
+    mean_launch_ms = sum(kernel_ms) / K
+    achieved = (sum(bytes_per_step) / K) / (mean_launch_ms * 1e-3) / 1e9
+
+    # end to end through the public API: pinned host x in, y back, each step
+    xh = torch.empty(K, B, cfg.d, dtype=dt).pin_memory()
+    xh.copy_(xs[W:].cpu())
+    yh = torch.empty(K, B, cfg.d, dtype=torch.float32).pin_memory()
+    barrier(world, device)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for s in range(K):
+            x_in.copy_(xh[s], non_blocking=True)
+            g.replay()
+            yh[s].copy_(y, non_blocking=True)
+        f1.record(stream)
+    stream.synchronize()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world, device)
+    del g
+
+    value = world * B * K / (t_max * 1e-3)
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": t_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": cfg.dtype, "data": "synthetic",
+        "config": {"workload": cfg.name, "layers": L, "d": cfg.d, "n": cfg.n, "H": cfg.H, "batch": B,
+                   "activation_rate": args.rate or cfg.rate, "alpha": cfg.alpha, "global_batch": B * world,
+                   "mean_active_neurons": float(ks.mean()), "parallelism": "replicas%d" % world,
+                   "reordered": True, "l2": "inputs larger than L2 (%.2f GB touched per step)"
+                   % (sum(bytes_per_step) / K / 1e9)},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "spffn decode step (one replay per step)", "peak_kind": peak_kind},
+        "e2e": {"value": world * B * K / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": B * cfg.d * 2, "d2h_bytes_per_step": B * cfg.d * 4},
+        "gpu_launches": launches_per_step * K,
+        "clocks": clk.summary(),
+    }
+    return res, (rank == 0)
+
+
+def _count_launches_per_step(L):
+    import activation_sparse_ffn_predictor_b200 as sp
+    return sp.launches_per_decode(L) if hasattr(sp, "launches_per_decode") else 6 * L
+
+
+# ---------------------------------------------------------------------------
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_sample(cfg, budget_s: float, rate=None, seed=1):
+    """Time the CPU oracle on (layer, step) samples of the same workload until
+    `budget_s` of oracle compute is spent; returns tokens/s per layer stack."""
+    import oracle as O
+    prepared = []
+    for l in range(min(2, cfg.layers)):
+        p, Wp1, bp1, Wp2, bp2 = wl.host_predictor(cfg, l, rate=rate)
+        prepared.append((l, p, wl.widen(Wp1, cfg.bf16), wl.widen(bp1, cfg.bf16), wl.widen(Wp2, cfg.bf16),
+                         wl.widen(bp2, cfg.bf16), wl.widen(wl.fc1_bias(p, cfg.bf16), cfg.bf16)))
+    spent, samples, s = 0.0, 0, 0
+    while spent < budget_s and samples < 10000:
+        l, p, Wp1, bp1, Wp2, bp2, b1 = prepared[samples % len(prepared)]
+        x64 = wl.widen(wl.tokens(cfg, cfg.batch, aux=s, seed=seed), cfg.bf16)
+        idx, k, _ = O.predict(Wp1, Wp2, bp2, x64, bp1)
+        sc = 1.0 / math.sqrt(cfg.d)
+        W1 = wl.widen(wl.fill_rows(wl.stream_id(wl.T_W1, l), cfg.d, idx, sc, cfg.bf16), cfg.bf16)
+        W2T = wl.widen(wl.fill_rows(wl.stream_id(wl.T_W2T, l), cfg.d, idx, sc, cfg.bf16), cfg.bf16)
+        t0 = time.perf_counter()
+        idx, k, _ = O.predict(Wp1, Wp2, bp2, x64, bp1)
+        O.sparse_ffn(W1, b1, W2T, None, x64, idx, row_ids=idx)
+        spent += time.perf_counter() - t0
+        samples += 1
+        s += 1
+    per_layer = spent / samples
+    tok_s = cfg.batch / (per_layer * cfg.layers)
+    return tok_s, samples, spent
+
+
+def run_reference(args, cfg, world, rank, local):
+    """The oracle as it stands on the host cores, same workload, bounded samples per step."""
+    if rank != 0:
+        return None, False
+    K, W = args.steps, args.warmup
+    per_step_budget = max(0.5, min(10.0, args.ref_budget / max(1, K + W)))
+    for _ in range(W):
+        oracle_sample(cfg, per_step_budget * 0.2, rate=args.rate)
+    vals, spent, samples = [], 0.0, 0
+    for _ in range(K):
+        v, n_s, sp_ = oracle_sample(cfg, per_step_budget, rate=args.rate)
+        vals.append(v)
+        spent += sp_
+        samples += n_s
+    value = statistics.mean(vals)
+    cores = cpu_threads()
+    ms = cfg.batch / value * 1e3
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": cfg.name, "layers": cfg.layers, "d": cfg.d, "n": cfg.n, "H": cfg.H,
+                   "batch": cfg.batch, "activation_rate": args.rate or cfg.rate, "alpha": cfg.alpha},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": "%d (layer, step) samples of the first 2 layers, %.1f s of oracle compute, "
+                                   "extrapolated to %d layers" % (samples, spent, cfg.layers)},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    return res, True
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--rate", type=float, default=None)
+    ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--layers", type=int, default=None)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle compute for cpu_baseline")
+    ap.add_argument("--ref-budget", type=float, default=60.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--launches-per-step", type=int, default=0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = wl.CONFIGS[args.config]
+    if args.batch:
+        cfg = cfg.with_(batch=args.batch)
+    if args.layers:
+        cfg = cfg.with_(layers=args.layers)
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        res, show = run_reference(args, cfg, world, rank, local)
+    else:
+        res, show = run_ours(args, cfg, world, rank, local)
+        if show and world == 1 and not args.no_cpu_baseline:
+            v, n_s, spent = oracle_sample(cfg, args.cpu_budget, rate=args.rate)
+            res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                                   "sample": "%d (layer, step) samples of the first 2 layers, %.1f s of oracle "
+                                             "compute, extrapolated to %d layers" % (n_s, spent, cfg.layers)}
+    if show and res is not None:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

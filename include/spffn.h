@@ -1,0 +1,187 @@
+/*
+ * spffn.h — activation-sparse FFN decoding on one NVIDIA B200 (sm_100a).
+ *
+ * A ReLU FFN block  y = W2 ReLU(W1 x + b1) + b2  is decoded activation-sparsely:
+ * a two-layer X-H-O MLP predictor scores every FFN neuron, the neurons whose
+ * sigmoid output exceeds 0.5 (logit > 0) are compacted into an ascending
+ * neuron table, and only those rows of W1 and of the neuron-major W2T = W2^T
+ * are read and computed.
+ *
+ * Passages that define the operations (page title, section):
+ *   [PI1] "LLM模型之PowerInfer1.0" — §2.1 (FFN: FC1, ReLU gate, FC2), §3.2
+ *         (single-layer example, Figure 3), §4.1 (adaptive sparse predictor,
+ *         X-H-O MLP), §4.2 (neuron tables), §4.4 (neuron-aware operators),
+ *         §5.1 (offline profiler counting activations), §5.2 equation (1)
+ *         (impact = activation frequency), DejaVu appendix equation (-1)
+ *         (predict S_M, then MLP restricted to S_M), closing question 3 (AXPY
+ *         over contiguous neuron columns for the down projection).
+ *   [SPX] "Técnicas dispersas para una aceleración 100X en la inferencia de
+ *         modelos de lenguaje grandes" — batch size erodes the sparsity
+ *         (union of per-token sets), 128-byte memory blocks.
+ *
+ * Conventions (all entry points):
+ *   - Every pointer argument named as "device" is a device pointer into memory
+ *     owned by the caller (e.g. allocated with the PyTorch caching allocator)
+ *     and must be 16-byte aligned.  The library never allocates device memory:
+ *     scratch lives in a caller-provided workspace.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every device call is asynchronous on `stream`; none syncs the
+ *     host, none copies device->host.
+ *   - Argument errors are detected on the host and returned before anything is
+ *     enqueued.  CUDA launch errors return SPFFN_ERR_CUDA.  Data-dependent
+ *     problems found on the device (e.g. a caller-supplied count > n) are
+ *     clamped, latched in the workspace's error word, and reported by
+ *     spffn_last_device_error.  No device code traps or spins without bound.
+ *   - One context is used by one stream at a time.  Contexts that share a
+ *     workspace must not run concurrently.
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef SPFFN_H
+#define SPFFN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SPFFN_OK = 0,
+    SPFFN_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or shape */
+    SPFFN_ERR_UNSUPPORTED = 2,   /* valid request this build does not serve (no sm_100 device) */
+    SPFFN_ERR_WORKSPACE = 3,     /* workspace missing or smaller than spffn_workspace_bytes() */
+    SPFFN_ERR_CUDA = 4,          /* a CUDA runtime call failed */
+    SPFFN_ERR_DEVICE_CHECK = 5,  /* a device-side check latched an error (see spffn_last_device_error) */
+    SPFFN_ERR_TIMEOUT = 6        /* a bounded device wait gave up */
+} spffn_status;
+
+typedef enum { SPFFN_F16 = 0, SPFFN_BF16 = 1 } spffn_dtype;
+
+/* Shape of one FFN layer and its predictor.
+ *   d          model width; d % 64 == 0, 64 <= d <= 16384
+ *   n          FFN neurons;  n % 32 == 0, 32 <= n <= 131072
+ *   H          predictor hidden width; H % 64 == 0, 64 <= H <= 8192
+ *   max_batch  largest batch B the context will see; 1 <= max_batch <= 32
+ *   dtype      storage type of weights and of x (accumulation is always fp32)
+ *   flags      0 (reserved) */
+typedef struct {
+    int32_t d, n, H, max_batch;
+    int32_t dtype;
+    uint32_t flags;
+} spffn_config;
+
+/* One layer's weights: device pointers, row-major, storage dtype, borrowed
+ * until spffn_destroy.
+ *   W1  [n][d]   FC1 rows (row j = neuron j)
+ *   b1  [n]      FC1 bias
+ *   W2T [n][d]   FC2 stored neuron-major: row j = column j of W2 ([PI1]
+ *                closing question 3), so each neuron is one contiguous row
+ *   b2  [d]      FC2 bias, may be NULL (= 0)
+ *   Wp1 [H][d]   predictor layer 1;  bp1 [H] may be NULL (= 0)
+ *   Wp2 [n][H]   predictor layer 2;  bp2 [n] may be NULL (= 0) */
+typedef struct {
+    const void *W1, *b1, *W2T, *b2, *Wp1, *bp1, *Wp2, *bp2;
+} spffn_weights;
+
+typedef struct spffn_ctx spffn_ctx;
+
+/* Bytes of device workspace a context with this config needs (0 on a bad
+ * config).  Pure host function. */
+size_t spffn_workspace_bytes(const spffn_config* cfg);
+
+/* Validate `cfg` and `w`, bind the caller's workspace (device, >=
+ * spffn_workspace_bytes(cfg) bytes, 256-byte aligned, zero-filled by the
+ * caller before first use, borrowed until spffn_destroy), and return a new
+ * host-side context in *out.  Enqueues nothing.  Kernels initialise every
+ * scratch word they read except the latched error word, which starts from the
+ * caller's zero fill and is cleared by spffn_last_device_error. */
+spffn_status spffn_create(const spffn_config* cfg, const spffn_weights* w, void* workspace,
+                          size_t workspace_bytes, spffn_ctx** out);
+
+/* Free the host-side context.  Safe on NULL.  Does not touch device memory. */
+spffn_status spffn_destroy(spffn_ctx* ctx);
+
+/* Predictor + threshold + compaction ([PI1] §4.1, DejaVu appendix (-1);
+ * [PI1] §4.2 neuron table; batch union per [SPX]):
+ *   h_t   = ReLU(Wp1 x_t + bp1)                  (fp32)
+ *   l_t,i = Wp2[i] . h_t + bp2_i                 (fp32)
+ *   neuron i selected  <=>  l_t,i > 0 for some token t  (sigmoid > 0.5)
+ *   idx[0..count) = selected neurons, ascending; *count written on device.
+ * x: device [B][d] storage dtype; 1 <= B <= max_batch.
+ * idx: device int32, capacity n.  count: device int32 scalar. */
+spffn_status spffn_predict(spffn_ctx* ctx, const void* x, int32_t B,
+                           int32_t* idx, int32_t* count, void* stream);
+
+/* Neuron-aware FFN over a neuron table ([PI1] §4.4 vec_dot for FC1, AXPY
+ * over neuron-major rows for FC2):
+ *   y_t = b2 + sum over j in idx[0..count), ascending, of ReLU(W1[j].x_t + b1_j) W2T[j]
+ * computed as fixed per-chunk fp32 partial sums reduced in a fixed order
+ * (deterministic: same inputs give the same bits).  Every token is computed
+ * on every neuron of the table.
+ * idx/count: device, e.g. from spffn_predict or any caller mask; entries must
+ * be in [0,n) (out-of-range entries are skipped and latched as a device
+ * error) and *count is clamped to n (latched).  count == 0 gives y = b2.
+ * y: device fp32 [B][d]. */
+spffn_status spffn_forward(spffn_ctx* ctx, const void* x, int32_t B, const int32_t* idx,
+                           const int32_t* count, float* y, void* stream);
+
+/* spffn_predict followed by spffn_forward on the same x (one layer's decode). */
+spffn_status spffn_step(spffn_ctx* ctx, const void* x, int32_t B, int32_t* idx, int32_t* count,
+                        float* y, void* stream);
+
+/* Layer chaining used between stacked layers (the pages give no attention or
+ * norm; this is the library's stated choice):
+ *   x_next_t = round_dtype( (x_t + y_t) / sqrt(mean_c (x_t + y_t)_c^2 + 1e-6) )
+ * x, x_next: device [B][d] storage dtype (may not alias); y: device fp32 [B][d]. */
+spffn_status spffn_chain(spffn_ctx* ctx, const void* x, const float* y, int32_t B, void* x_next,
+                         void* stream);
+
+/* One decode step through a stack of L layers: for l = 0..L-1
+ *   (idx_l, count_l) = predict_l(x_l);  y_l = forward_l(x_l);  x_{l+1} = chain(x_l, y_l)
+ * layers: host array of L contexts with equal d, dtype and max_batch.
+ * x_in: device [B][d]; x_out: device [B][d] = x_L; y: device fp32 [B][d] = y_{L-1};
+ * counts: device int32 [L] (count_l), may be NULL.  Intermediate x_l live in
+ * the layers' workspaces. */
+spffn_status spffn_decode(spffn_ctx* const* layers, int32_t L, const void* x_in, int32_t B,
+                          void* x_out, float* y, int32_t* counts, void* stream);
+
+/* Offline profiler ([PI1] §5.1): for T profiling tokens X [T][d] (device,
+ * storage dtype), counts[j] += #{t : W1[j].X_t + b1_j > 0}.  counts: device
+ * uint32 [n], accumulated (caller zeroes it before the first batch). */
+spffn_status spffn_profile_counts(spffn_ctx* ctx, const void* X, int32_t T, uint32_t* counts,
+                                  void* stream);
+
+/* Hot-first placement ([PI1] §5.2 equation (1), impact = frequency): host
+ * arrays; perm[s] = original neuron placed in slot s, ordering by count
+ * descending, ties by original index ascending.  Pure host function. */
+spffn_status spffn_reorder(const uint32_t* counts_host, int32_t n, int32_t* perm_host);
+
+/* Row gather applying a neuron table: dst row s = src row perm[s], for `rows`
+ * rows of `row_bytes` bytes (row_bytes % 16 == 0).  src, dst, perm: device;
+ * dst must not alias src; perm entries must lie in [0, rows) (out-of-range
+ * rows are left unwritten).  Permutes W1, W2T and Wp2 into hot-first order;
+ * 2-byte bias vectors use spffn_permute_vector. */
+spffn_status spffn_permute_rows(const void* src, void* dst, int32_t rows, int32_t row_bytes,
+                                const int32_t* perm, void* stream);
+
+/* Element gather dst[s] = src[perm[s]] for a vector of 2-byte elements. */
+spffn_status spffn_permute_vector(const void* src, void* dst, int32_t count, const int32_t* perm,
+                                  void* stream);
+
+/* Read and clear the context's device error word (synchronises `stream`).
+ * Returns SPFFN_OK if clean, SPFFN_ERR_DEVICE_CHECK or SPFFN_ERR_TIMEOUT;
+ * *code (may be NULL) receives the raw word. */
+spffn_status spffn_last_device_error(spffn_ctx* ctx, uint32_t* code, void* stream);
+
+/* Static description of a status code. */
+const char* spffn_status_string(spffn_status s);
+
+/* Number of fp32 partial sums the forward reduction uses (its fixed split). */
+int32_t spffn_num_partials(const spffn_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPFFN_H */

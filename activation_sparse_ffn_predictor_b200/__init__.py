@@ -26,7 +26,8 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_CHECK,
 EXPORTS = ("spffn_workspace_bytes", "spffn_create", "spffn_destroy", "spffn_predict", "spffn_forward",
            "spffn_step", "spffn_chain", "spffn_decode", "spffn_profile_counts", "spffn_reorder",
            "spffn_permute_rows", "spffn_permute_vector", "spffn_last_device_error", "spffn_status_string",
-           "spffn_num_partials")
+           "spffn_num_partials", "spffn_decode_kernel_launches", "spffn_set_trace", "spffn_trace_marks",
+           "spffn_last_cuda_error_string", "spffn_reorder_dealt")
 
 
 class SpffnError(RuntimeError):
@@ -73,11 +74,16 @@ def library(path: Optional[str] = None):
         "spffn_decode": (st, [ctypes.POINTER(vp), i32, vp, i32, vp, vp, vp, vp]),
         "spffn_profile_counts": (st, [vp, vp, i32, vp, vp]),
         "spffn_reorder": (st, [vp, i32, vp]),
+        "spffn_reorder_dealt": (st, [vp, i32, i32, vp]),
         "spffn_permute_rows": (st, [vp, vp, i32, i32, vp, vp]),
         "spffn_permute_vector": (st, [vp, vp, i32, vp, vp]),
         "spffn_last_device_error": (st, [vp, ctypes.POINTER(ctypes.c_uint32), vp]),
         "spffn_status_string": (ctypes.c_char_p, [st]),
         "spffn_num_partials": (i32, [vp]),
+        "spffn_decode_kernel_launches": (i32, [ctypes.POINTER(vp), i32, i32]),
+        "spffn_set_trace": (st, [vp, sz]),
+        "spffn_trace_marks": (i32, []),
+        "spffn_last_cuda_error_string": (ctypes.c_char_p, []),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -96,6 +102,8 @@ def _status_string(s: int) -> str:
 
 def _check(status: int, what: str):
     if status != OK:
+        if status == ERR_CUDA:
+            what = "%s [%s]" % (what, library().spffn_last_cuda_error_string().decode())
         raise SpffnError(status, what)
 
 
@@ -211,11 +219,37 @@ def decode(layers: Sequence[Layer], x_in, x_out, y, counts=None, stream=None):
                                   _stream(stream)), "spffn_decode")
 
 
+def decode_kernel_launches(layers: Sequence[Layer], B: int) -> int:
+    arr = (ctypes.c_void_p * len(layers))(*[l.ctx.value for l in layers])
+    return int(library().spffn_decode_kernel_launches(arr, len(layers), B))
+
+
+def set_trace(buf=None):
+    """Bind (or unbind with None) a uint64 CUDA tensor that whole-stack decode
+    launches fill with per-(CTA, layer, mark) %globaltimer stamps."""
+    if buf is None:
+        _check(library().spffn_set_trace(None, 0), "spffn_set_trace")
+    else:
+        _check(library().spffn_set_trace(_p(buf), buf.numel() * buf.element_size()), "spffn_set_trace")
+
+
+def trace_marks() -> int:
+    return int(library().spffn_trace_marks())
+
+
 def reorder(counts: np.ndarray) -> np.ndarray:
     c = np.ascontiguousarray(counts, dtype=np.uint32)
     perm = np.empty(c.size, dtype=np.int32)
     _check(library().spffn_reorder(c.ctypes.data_as(ctypes.c_void_p), c.size,
                                    perm.ctypes.data_as(ctypes.c_void_p)), "spffn_reorder")
+    return perm
+
+
+def reorder_dealt(counts: np.ndarray, parts: int) -> np.ndarray:
+    c = np.ascontiguousarray(counts, dtype=np.uint32)
+    perm = np.empty(c.size, dtype=np.int32)
+    _check(library().spffn_reorder_dealt(c.ctypes.data_as(ctypes.c_void_p), c.size, parts,
+                                         perm.ctypes.data_as(ctypes.c_void_p)), "spffn_reorder_dealt")
     return perm
 
 

@@ -34,11 +34,21 @@ int device_sms() {
     return sms;
 }
 
-spffn_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SPFFN_OK : SPFFN_ERR_CUDA; }
+thread_local cudaError_t t_last_cuda = cudaSuccess;
+
+spffn_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return SPFFN_OK;
+    t_last_cuda = e;
+    return SPFFN_ERR_CUDA;
+}
 
 }  // namespace
 
 extern "C" {
+
+const char* spffn_last_cuda_error_string(void) {
+    return t_last_cuda == cudaSuccess ? "no CUDA error recorded" : cudaGetErrorString(t_last_cuda);
+}
 
 const char* spffn_status_string(spffn_status s) {
     switch (s) {
@@ -139,17 +149,31 @@ spffn_status spffn_decode(spffn_ctx* const* layers, int32_t L, const void* x_in,
     for (int l = 0; l < L; ++l) {
         const spffn_ctx& c = *layers[l];
         cudaError_t e = launch_predict(c, xcur, B, c.idx(), c.count(), counts ? counts + l : nullptr, st);
-        if (e != cudaSuccess) return SPFFN_ERR_CUDA;
+        if (e != cudaSuccess) return cuda_status(e);
         float* yl = (l == L - 1) ? y : c.ybuf();
         e = launch_forward(c, xcur, B, c.idx(), c.count(), yl, st);
-        if (e != cudaSuccess) return SPFFN_ERR_CUDA;
+        if (e != cudaSuccess) return cuda_status(e);
         void* xn = (l == L - 1) ? x_out : c.xbuf(l & 1);
         e = launch_chain(c, xcur, yl, B, xn, st);
-        if (e != cudaSuccess) return SPFFN_ERR_CUDA;
+        if (e != cudaSuccess) return cuda_status(e);
         xcur = xn;
     }
     return SPFFN_OK;
 }
+
+int32_t spffn_decode_kernel_launches(spffn_ctx* const* layers, int32_t L, int32_t B) {
+    if (!layers || L < 1 || !layers[0] || B < 1 || B > layers[0]->cfg.max_batch) return 0;
+    for (int l = 0; l < L; ++l)
+        if (!layers[l]) return 0;
+    return fused_decode_supported(layers, L, B) ? 1 : 6 * L;
+}
+
+spffn_status spffn_set_trace(void* buf, size_t bytes) {
+    set_trace(buf, bytes);
+    return SPFFN_OK;
+}
+
+int32_t spffn_trace_marks(void) { return trace_marks(); }
 
 spffn_status spffn_profile_counts(spffn_ctx* ctx, const void* X, int32_t T, uint32_t* counts, void* stream) {
     if (!ctx || !X || !counts || T < 1 || !aligned16(X)) return SPFFN_ERR_INVALID_ARG;
@@ -163,6 +187,23 @@ spffn_status spffn_reorder(const uint32_t* counts_host, int32_t n, int32_t* perm
     std::stable_sort(p.begin(), p.end(),
                      [&](int32_t a, int32_t b) { return counts_host[a] > counts_host[b]; });
     std::copy(p.begin(), p.end(), perm_host);
+    return SPFFN_OK;
+}
+
+spffn_status spffn_reorder_dealt(const uint32_t* counts_host, int32_t n, int32_t parts, int32_t* perm_host) {
+    if (!counts_host || !perm_host || n < 1 || parts < 1) return SPFFN_ERR_INVALID_ARG;
+    std::vector<int32_t> hot(n);
+    std::iota(hot.begin(), hot.end(), 0);
+    std::stable_sort(hot.begin(), hot.end(),
+                     [&](int32_t a, int32_t b) { return counts_host[a] > counts_host[b]; });
+    std::vector<int64_t> lo(parts + 1);
+    int64_t widest = 0;
+    for (int c = 0; c <= parts; ++c) lo[c] = (int64_t)n * c / parts;
+    for (int c = 0; c < parts; ++c) widest = std::max(widest, lo[c + 1] - lo[c]);
+    int64_t next = 0;
+    for (int64_t r = 0; r < widest; ++r)
+        for (int c = 0; c < parts; ++c)
+            if (lo[c] + r < lo[c + 1]) perm_host[lo[c] + r] = hot[next++];
     return SPFFN_OK;
 }
 

@@ -1,9 +1,1046 @@
-// Persistent whole-stack decode kernel.
+// Persistent whole-stack decode kernel for small batches (B <= 2).
+//
+// One CTA per SM runs every layer of the stack in a single launch.  Per layer,
+// four phases separated by grid barriers:
+//   A  h = ReLU(Wp1 x + bp1)          Wp1 rows split across CTAs
+//   B  logits, threshold, mask bits    Wp2 rows split across CTAs (atomicOr into
+//                                      the mask words, per-CTA counts)
+//   C  neuron table + FFN              every CTA takes an equal slice of the
+//                                      ascending table, gathers W1/W2T rows,
+//                                      FC1 (vec_dot) + ReLU, FC2 (AXPY) into a
+//                                      fixed per-CTA fp32 partial
+//   D  y = b2 + sum of partials (fixed order), u = x + y, per-CTA sum of squares
+// and the next layer's input x = round(u / rms(u)) is formed at the start of
+// its phase A.
+//
+// Weight bytes move with cp.async.bulk (TMA bulk copies) into shared-memory
+// rings guarded by mbarriers.  The predictor weights do not depend on the
+// data, so a dedicated producer warp streams them ahead across the grid
+// barriers (the ring keeps HBM busy while the consumers wait); a second
+// producer warp gathers the FFN rows as soon as the neuron table is known.
+//
+// Every wait is bounded (globaltimer): on expiry the CTA latches an error,
+// raises a grid-wide abort flag, stops issuing copies, waits (bounded) for the
+// copies it already issued and returns.
 #include "spffn_fused.cuh"
 
 namespace spffn {
-bool fused_decode_supported(spffn_ctx* const*, int, int) { return false; }
-cudaError_t launch_fused_decode(spffn_ctx* const*, int, const void*, int, void*, float*, int32_t*, cudaStream_t) {
-    return cudaErrorNotSupported;
+
+namespace {
+
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kThreads = kConsumers + 64;      // + predictor producer warp + FFN producer warp
+constexpr int kMaxFusedLayers = 128;
+constexpr int kMaxVPT = 5;                      // 16-byte column vectors per consumer thread (d <= 10240)
+constexpr int kMaxG = 256;
+constexpr unsigned long long kWaitNs = 2000000000ull;   // 2 s per wait
+constexpr int kTraceMarks = 16;                 // stamps per (CTA, layer), see TRACE() below
+constexpr int kMaxMaskWords = 2048;             // n <= 65536 on this path
+
+struct LayerW {
+    const void *W1, *b1, *W2T, *b2, *Wp1, *bp1, *Wp2, *bp2;
+    int32_t* idx;
+};
+
+struct Params {
+    int L, B, d, n, H, G;
+    const void* x_in;
+    void* x_out;
+    float* y;
+    int32_t* counts;
+    uint32_t* bar;        // grid-barrier counter
+    uint32_t* err;
+    uint32_t* abort;
+    uint32_t* mask;       // [2][n/32]
+    int32_t* cta_count;   // [G]
+    float* h;             // [B][H]
+    float* partial;       // [G][B][d]
+    float* u;             // [B][d]
+    float* ss;            // [G][B]
+    int pred_slots, pred_slot_bytes, ffn_slots, R1, R2, max_rows;
+    unsigned long long* trace;   // optional [G][L][kTraceMarks] globaltimer stamps
+    LayerW layer[kMaxFusedLayers];
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+__device__ __forceinline__ uint32_t sptr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ unsigned long long gtime() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
 }
+
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(sptr(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(sptr(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(sptr(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(sptr(b)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(sptr(dst)),
+        "l"(src), "r"(bytes), "r"(sptr(bar))
+        : "memory");
+}
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory"); }
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+struct Shared {
+    uint64_t* pfull;
+    uint64_t* pempty;
+    uint64_t* ffull;
+    uint64_t* fempty;
+    uint64_t* fready;
+    volatile int* flags;     // [0] local abort, [1] ffn_m, [2] pred issued, [3] ffn issued, [4] pred done, [5] ffn done
+    char* pring;
+    char* fring;
+    void* xs;
+    float* hs;
+    unsigned char* sel;
+    int32_t* nl;
+    uint32_t* maskw;         // [n/32] copy of the layer's mask words
+    float* bias1;            // [max_rows_h] bp1 for the CTA's Wp1 rows
+    float* bias2;            // [max_rows]   bp2 for the CTA's Wp2 rows
+    float* biasy;            // [max_cols]   b2 for the CTA's output columns
+    float* red;              // [2][8][NB]
+    float* red2;             // [8][NB]
+    int32_t* scan;           // [kMaxG + 1]
+    float* misc;             // [16]
+};
+
+__device__ __forceinline__ bool aborted(const Shared& S, const Params& p) {
+    return S.flags[0] != 0 || *(volatile uint32_t*)p.abort != 0;
+}
+
+__device__ __forceinline__ void raise_abort(const Shared& S, const Params& p, uint32_t bits) {
+    S.flags[0] = 1;
+    atomicOr(p.err, bits);
+    atomicExch(p.abort, 1u);
+}
+
+// Bounded wait on an mbarrier phase; false on timeout (or abort, for a producer).
+// Consumer threads ignore the abort flag here: a phase either completes for all
+// of them or for none, so every consumer leaves a wait the same way and no
+// named barrier is left short of arrivals.
+__device__ __forceinline__ bool wait_bounded(const Shared& S, const Params& p, uint64_t* b, uint32_t parity,
+                             bool producer = false) {
+    if (mbar_try(b, parity)) return true;
+    const unsigned long long t0 = gtime();
+    while (!mbar_try(b, parity)) {
+        if (producer && aborted(S, p)) return false;
+        if (gtime() - t0 > kWaitNs) {
+            raise_abort(S, p, ERR_PIPE_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// Grid barrier among the consumer groups of all CTAs (monotonic counter).
+__device__ __forceinline__ bool grid_barrier(const Shared& S, const Params& p, uint32_t& epoch) {
+    consumer_sync();
+    epoch += 1;
+    if (threadIdx.x == 0) {
+        // the CTA barrier above orders every consumer's writes before this release
+        red_release_add(p.bar, 1u);
+        const uint32_t target = epoch * (uint32_t)p.G;
+        if (ld_acquire(p.bar) < target) {
+            const unsigned long long t0 = gtime();
+            while (ld_acquire(p.bar) < target) {
+                if (*(volatile uint32_t*)p.abort) { S.flags[0] = 1; break; }
+                if (gtime() - t0 > kWaitNs) { raise_abort(S, p, ERR_BARRIER_TIMEOUT); break; }
+            }
+        }
+    }
+    consumer_sync();
+    return S.flags[0] == 0;
+}
+
+__device__ __forceinline__ int split_lo(int total, int parts, int i) {
+    return (int)((long long)total * i / parts);
+}
+
+// ---------------------------------------------------------------------------
+// arithmetic helpers
+//
+// Weight x activation products where both are in the storage dtype (GEMV1 and
+// FC1) use the mixed-precision FMA of sm_100 (fp16/bf16 operands, fp32
+// accumulator: the product is exact, one rounding).  Products with fp32
+// activations (GEMV2 with h, FC2 with a) convert the weight pair and use the
+// packed two-lane fp32 FMA.
+typedef unsigned long long u64;
+
+#ifndef SPFFN_WAIT_HINT_NS
+#define SPFFN_WAIT_HINT_NS 1000000
+#endif
+
+__device__ __forceinline__ u64 pk(float a, float b) {
+    u64 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ float2 upk(u64 r) {
+    float2 f;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(r));
+    return f;
+}
+__device__ __forceinline__ void ffma2(u64& acc, u64 a, u64 b) {
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
+}
+
+template <typename T> struct Arith;
+template <> struct Arith<__half> {
+    // a0 += w.lo * x.lo ; a1 += w.hi * x.hi  (w, x: packed pairs of fp16)
+    static __device__ __forceinline__ void mix2(float& a0, float& a1, uint32_t w, uint32_t x) {
+        unsigned short wl, wh, xl, xh;
+        asm("mov.b32 {%0, %1}, %2;" : "=h"(wl), "=h"(wh) : "r"(w));
+        asm("mov.b32 {%0, %1}, %2;" : "=h"(xl), "=h"(xh) : "r"(x));
+        asm("fma.rn.f32.f16 %0, %1, %2, %0;" : "+f"(a0) : "h"(wl), "h"(xl));
+        asm("fma.rn.f32.f16 %0, %1, %2, %0;" : "+f"(a1) : "h"(wh), "h"(xh));
+    }
+    static __device__ __forceinline__ u64 widen2(uint32_t w) {
+        const float2 f = DT<__half>::f2(w);
+        return pk(f.x, f.y);
+    }
+};
+template <> struct Arith<__nv_bfloat16> {
+    static __device__ __forceinline__ void mix2(float& a0, float& a1, uint32_t w, uint32_t x) {
+        unsigned short wl, wh, xl, xh;
+        asm("mov.b32 {%0, %1}, %2;" : "=h"(wl), "=h"(wh) : "r"(w));
+        asm("mov.b32 {%0, %1}, %2;" : "=h"(xl), "=h"(xh) : "r"(x));
+        asm("fma.rn.f32.bf16 %0, %1, %2, %0;" : "+f"(a0) : "h"(wl), "h"(xl));
+        asm("fma.rn.f32.bf16 %0, %1, %2, %0;" : "+f"(a1) : "h"(wh), "h"(xh));
+    }
+    static __device__ __forceinline__ u64 widen2(uint32_t w) {
+        return pk(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    }
+};
+
+// 16-byte weight vector . 16-byte storage-dtype vector into four partial sums
+template <typename T>
+__device__ __forceinline__ void dot_mix(float* a, const uint4& w, const uint4& x) {
+    Arith<T>::mix2(a[0], a[1], w.x, x.x);
+    Arith<T>::mix2(a[2], a[3], w.y, x.y);
+    Arith<T>::mix2(a[0], a[1], w.z, x.z);
+    Arith<T>::mix2(a[2], a[3], w.w, x.w);
+}
+
+__device__ __forceinline__ float sum4(const float* a) { return (a[0] + a[1]) + (a[2] + a[3]); }
+
+__device__ __forceinline__ bool mbar_try_hint(uint64_t* b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(sptr(b)), "r"(parity), "r"((uint32_t)SPFFN_WAIT_HINT_NS)
+        : "memory");
+    return ok != 0;
+}
+
+// Consumer-side bounded wait: suspends in hardware between checks.
+__device__ __forceinline__ bool cwait(const Shared& S, const Params& p, uint64_t* b, uint32_t parity) {
+    if (mbar_try(b, parity)) return true;
+    const unsigned long long t0 = gtime();
+    while (!mbar_try_hint(b, parity)) {
+        if (gtime() - t0 > kWaitNs) {
+            raise_abort(S, p, ERR_PIPE_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// Phase stamps (only when a trace buffer is bound): consumer thread 0 records
+// %globaltimer at fixed points of each layer.
+#define TRACE(mark)                                                                                  \
+    do {                                                                                             \
+        if (p.trace && tid == 0 && l < p.L)                                                          \
+            p.trace[((size_t)c * p.L + l) * kTraceMarks + (mark)] = gtime();                         \
+    } while (0)
+
+// ---------------------------------------------------------------------------
+template <typename T, int NB, int HV>
+__global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ Params p)
+{
+    extern __shared__ __align__(128) char smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int c = blockIdx.x, G = p.G, d = p.d, n = p.n, H = p.H, B = p.B;
+    const int nvec = d >> 3;                   // 16-byte vectors per d-row
+    const int hv = H >> 3;                     // 16-byte vectors per H-row
+    const int fslot_bytes = 4 * d + 128;       // W1 row, W2T row, 16-byte block holding b1[j]
+
+    // ---- carve shared memory
+    Shared S;
+    {
+        char* q = smem;
+        S.pring = q; q += (size_t)p.pred_slots * p.pred_slot_bytes;
+        S.fring = q; q += (size_t)p.ffn_slots * fslot_bytes;
+        S.xs = q; q += ((size_t)NB * d * sizeof(T) + 127) / 128 * 128;
+        S.hs = reinterpret_cast<float*>(q); q += ((size_t)NB * H * 4 + 127) / 128 * 128;
+        S.sel = reinterpret_cast<unsigned char*>(q); q += (p.max_rows + 127) / 128 * 128;
+        S.nl = reinterpret_cast<int32_t*>(q); q += ((size_t)p.max_rows * 4 + 127) / 128 * 128;
+        S.maskw = reinterpret_cast<uint32_t*>(q); q += ((size_t)(n >> 5) * 4 + 127) / 128 * 128;
+        S.bias1 = reinterpret_cast<float*>(q); q += ((size_t)(H / G + 2) * 4 + 127) / 128 * 128;
+        S.bias2 = reinterpret_cast<float*>(q); q += ((size_t)p.max_rows * 4 + 127) / 128 * 128;
+        S.biasy = reinterpret_cast<float*>(q); q += ((size_t)(d / G + 8) * 4 + 127) / 128 * 128;
+        S.red = reinterpret_cast<float*>(q); q += 2 * 8 * 2 * NB * 4;
+        S.red2 = reinterpret_cast<float*>(q); q += 8 * NB * 4;
+        S.scan = reinterpret_cast<int32_t*>(q); q += (kMaxG + 1) * 4;
+        S.misc = reinterpret_cast<float*>(q); q += 16 * 4;
+        q = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(q) + 15) & ~uintptr_t(15));
+        uint64_t* bars = reinterpret_cast<uint64_t*>(q);
+        S.pfull = bars; S.pempty = bars + p.pred_slots;
+        S.ffull = S.pempty + p.pred_slots; S.fempty = S.ffull + p.ffn_slots;
+        S.fready = S.fempty + p.ffn_slots;
+        S.flags = reinterpret_cast<volatile int*>(S.fready + 1);
+    }
+    if (tid == 0) {
+        for (int i = 0; i < p.pred_slots; ++i) { mbar_init(&S.pfull[i], 1); mbar_init(&S.pempty[i], kConsumerWarps); }
+        for (int i = 0; i < p.ffn_slots; ++i) { mbar_init(&S.ffull[i], 1); mbar_init(&S.fempty[i], kConsumerWarps); }
+        mbar_init(S.fready, 1);
+        for (int i = 0; i < 8; ++i) S.flags[i] = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    // CTA c's rows of Wp1 and Wp2 (contiguous spans)
+    const int a0 = split_lo(H, G, c), a1 = split_lo(H, G, c + 1);
+    const int b0 = split_lo(n, G, c), b1 = split_lo(n, G, c + 1);
+
+    // =======================================================================
+    // predictor producer: streams [Wp1 rows a0..a1) then [Wp2 rows b0..b1) per layer, and
+    // once a layer's copies are all issued, asks L2 to prefetch the next layer's spans so
+    // HBM keeps streaming while the consumers sit in latency-bound phases.
+    if (warp == kConsumerWarps) {
+        if (lane == 0) {
+            int k = 0;
+            for (int l = 0; l < p.L && !aborted(S, p); ++l) {
+                for (int part = 0; part < 2; ++part) {
+                    const int r0 = part ? b0 : a0, r1 = part ? b1 : a1, R = part ? p.R2 : p.R1;
+                    const size_t rb = part ? (size_t)H * 2 : (size_t)d * 2;
+                    const char* base = reinterpret_cast<const char*>(part ? p.layer[l].Wp2 : p.layer[l].Wp1);
+                    for (int r = r0; r < r1; r += R, ++k) {
+                        const int s = k % p.pred_slots;
+                        if (!wait_bounded(S, p, &S.pempty[s], ((k / p.pred_slots) & 1) ^ 1, true)) goto pred_done;
+                        const uint32_t bytes = (uint32_t)(min(R, r1 - r) * rb);
+                        mbar_expect_tx(&S.pfull[s], bytes);
+                        bulk_g2s(S.pring + (size_t)s * p.pred_slot_bytes, base + (size_t)r * rb, bytes, &S.pfull[s]);
+                        S.flags[2] = k + 1;
+                    }
+                }
+#ifndef SPFFN_NO_L2_PREFETCH
+                if (l + 1 < p.L) {
+                    for (int part = 0; part < 2; ++part) {
+                        const int r0 = part ? b0 : a0, r1 = part ? b1 : a1;
+                        const size_t rb = part ? (size_t)H * 2 : (size_t)d * 2;
+                        const char* base = reinterpret_cast<const char*>(part ? p.layer[l + 1].Wp2 : p.layer[l + 1].Wp1);
+                        const size_t total = (size_t)(r1 - r0) * rb;
+                        for (size_t off = 0; off < total; off += 32768)
+                            bulk_prefetch_l2(base + (size_t)r0 * rb + off, (uint32_t)min((size_t)32768, total - off));
+                    }
+                }
+#endif
+            }
+        pred_done:
+            __threadfence_block();
+            S.flags[4] = 1;
+        }
+        return;
+    }
+    // =======================================================================
+    // FFN producer: gathers W1[j], W2T[j] and b1[j]'s 16-byte block for every neuron the
+    // consumers append to this CTA's list, as soon as it appears.
+    if (warp == kConsumerWarps + 1) {
+        if (lane == 0) {
+            int k = 0;
+            bool stop = false;
+            for (int l = 0; l < p.L && !stop; ++l) {
+                const char* w1 = reinterpret_cast<const char*>(p.layer[l].W1);
+                const char* w2 = reinterpret_cast<const char*>(p.layer[l].W2T);
+                const char* bb0 = reinterpret_cast<const char*>(p.layer[l].b1);
+                int issued = 0;
+                unsigned long long t0 = gtime();
+                while (true) {
+                    const int f = S.flags[1];
+                    const int avail = ((f >> 16) & 0x7fff) == (l & 0x7fff) ? (f & 0xffff) : 0;
+                    if (issued < avail) {
+                        __threadfence_block();
+                        const int s = k % p.ffn_slots;
+                        if (!wait_bounded(S, p, &S.fempty[s], ((k / p.ffn_slots) & 1) ^ 1, true)) { stop = true; break; }
+                        const int j = S.nl[issued];
+                        char* dst = S.fring + (size_t)s * fslot_bytes;
+                        mbar_expect_tx(&S.ffull[s], (uint32_t)(4 * d + 16));
+                        bulk_g2s(dst, w1 + (size_t)j * 2 * d, (uint32_t)(2 * d), &S.ffull[s]);
+                        bulk_g2s(dst + 2 * d, w2 + (size_t)j * 2 * d, (uint32_t)(2 * d), &S.ffull[s]);
+                        bulk_g2s(dst + 4 * d, bb0 + (size_t)(j & ~7) * 2, 16u, &S.ffull[s]);
+                        S.flags[3] = ++k;
+                        ++issued;
+                        t0 = gtime();
+                        continue;
+                    }
+                    if (S.flags[7] == l + 1) {
+                        const int f2 = S.flags[1];
+                        const int fin = ((f2 >> 16) & 0x7fff) == (l & 0x7fff) ? (f2 & 0xffff) : 0;
+                        if (issued >= fin) break;
+                        continue;
+                    }
+                    if (aborted(S, p)) { stop = true; break; }
+                    if (gtime() - t0 > kWaitNs) { raise_abort(S, p, ERR_PIPE_TIMEOUT); stop = true; break; }
+                    __nanosleep(64);
+                }
+            }
+            __threadfence_block();
+            S.flags[5] = 1;
+        }
+        return;
+    }
+    // =======================================================================
+    // consumers (warps 0..7)
+    uint32_t epoch = 0;
+    int pk_ = 0, fk = 0;       // chunks consumed from each ring
+    int rpar = 0;
+    T* xs = reinterpret_cast<T*>(S.xs);
+    const int R1 = p.R1, R2 = p.R2;
+    const int words = n >> 5;
+    bool ok = true;
+
+    for (int l = 0; l <= p.L && ok; ++l) {
+        const LayerW& W = p.layer[l < p.L ? l : 0];
+        // -------------------------------------------------------------- phase A: form x_l
+        // this layer's bias slices, in the same round trip as the input
+        if (l < p.L) {
+            const T* bp1 = reinterpret_cast<const T*>(W.bp1);
+            const T* bp2 = reinterpret_cast<const T*>(W.bp2);
+            const T* b2p = reinterpret_cast<const T*>(W.b2);
+            const int ng = d >> 2;
+            const int c0 = split_lo(ng, G, c) * 4, c1 = split_lo(ng, G, c + 1) * 4;
+            for (int i = tid; i < b1 - b0; i += kConsumers) S.bias2[i] = bp2 ? DT<T>::f(bp2[b0 + i]) : 0.f;
+            if (tid < a1 - a0) S.bias1[tid] = bp1 ? DT<T>::f(bp1[a0 + tid]) : 0.f;
+            if (tid < c1 - c0) S.biasy[tid] = b2p ? DT<T>::f(b2p[c0 + tid]) : 0.f;
+        }
+        // Thread tid owns the 16-byte column vectors v = tid + m*256 of x.
+        if (l == 0) {
+            const T* xin = reinterpret_cast<const T*>(p.x_in);
+#pragma unroll
+            for (int m = 0; m < kMaxVPT; ++m) {
+                const int v = tid + m * kConsumers;
+#pragma unroll
+                for (int t = 0; t < NB; ++t)
+                    if (v < nvec)
+                        reinterpret_cast<uint4*>(xs + (size_t)t * d)[v] =
+                            __ldcg(reinterpret_cast<const uint4*>(xin + (size_t)t * d) + v);
+            }
+        } else {
+            float4 uv[kMaxVPT][2][NB];
+#pragma unroll
+            for (int m = 0; m < kMaxVPT; ++m) {
+                const int v = tid + m * kConsumers;
+#pragma unroll
+                for (int t = 0; t < NB; ++t) {
+                    if (v < nvec) {
+                        const float4* up = reinterpret_cast<const float4*>(p.u + (size_t)t * d + v * 8);
+                        uv[m][0][t] = __ldcg(up);
+                        uv[m][1][t] = __ldcg(up + 1);
+                    }
+                }
+            }
+            // rms of u = x + y from the loaded values themselves (same tree in every CTA)
+            {
+                float sq[NB];
+#pragma unroll
+                for (int t = 0; t < NB; ++t) {
+                    sq[t] = 0.f;
+#pragma unroll
+                    for (int m = 0; m < kMaxVPT; ++m) {
+                        const int v = tid + m * kConsumers;
+                        if (v < nvec) {
+                            const float4 a = uv[m][0][t], b = uv[m][1][t];
+                            sq[t] = fmaf(a.x, a.x, sq[t]); sq[t] = fmaf(a.y, a.y, sq[t]);
+                            sq[t] = fmaf(a.z, a.z, sq[t]); sq[t] = fmaf(a.w, a.w, sq[t]);
+                            sq[t] = fmaf(b.x, b.x, sq[t]); sq[t] = fmaf(b.y, b.y, sq[t]);
+                            sq[t] = fmaf(b.z, b.z, sq[t]); sq[t] = fmaf(b.w, b.w, sq[t]);
+                        }
+                    }
+                    sq[t] = warp_sum(sq[t]);
+                    if (lane == 0) S.red2[warp * NB + t] = sq[t];
+                }
+                consumer_sync();
+                if (tid < NB) {
+                    float z = 0.f;
+                    for (int q = 0; q < kConsumerWarps; ++q) z += S.red2[q * NB + tid];
+                    S.misc[tid] = 1.0f / sqrtf(z / (float)d + 1e-6f);
+                }
+            }
+            consumer_sync();
+#pragma unroll
+            for (int t = 0; t < NB; ++t) {
+                const float rs = S.misc[t];
+#pragma unroll
+                for (int m = 0; m < kMaxVPT; ++m) {
+                    const int v = tid + m * kConsumers;
+                    if (v < nvec) {
+                        const float f[8] = {uv[m][0][t].x, uv[m][0][t].y, uv[m][0][t].z, uv[m][0][t].w,
+                                            uv[m][1][t].x, uv[m][1][t].y, uv[m][1][t].z, uv[m][1][t].w};
+                        T r8[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) r8[q] = DT<T>::r(f[q] * rs);
+                        reinterpret_cast<uint4*>(xs + (size_t)t * d)[v] = *reinterpret_cast<const uint4*>(r8);
+                    }
+                }
+            }
+            if (l == p.L) {
+                if (c == 0) {
+                    T* xo = reinterpret_cast<T*>(p.x_out);
+#pragma unroll
+                    for (int m = 0; m < kMaxVPT; ++m) {
+                        const int v = tid + m * kConsumers;
+                        for (int t = 0; t < B; ++t)
+                            if (v < nvec)
+                                reinterpret_cast<uint4*>(xo + (size_t)t * d)[v] =
+                                    reinterpret_cast<const uint4*>(xs + (size_t)t * d)[v];
+                    }
+                }
+                break;
+            }
+        }
+        consumer_sync();
+        TRACE(0);
+        // GEMV1 over Wp1 rows [a0, a1): mixed-precision dot of each row with x
+        for (int r = a0; r < a1 && ok; r += R1, ++pk_) {
+            const int s = pk_ % p.pred_slots;
+            if (!cwait(S, p, &S.pfull[s], (pk_ / p.pred_slots) & 1)) { ok = false; break; }
+            if (r == a0) TRACE(1); else TRACE(13);
+            const uint4* slot = reinterpret_cast<const uint4*>(S.pring + (size_t)s * p.pred_slot_bytes);
+            const int rows = min(R1, a1 - r);
+            const int Q = R1 >= kConsumerWarps ? 1 : kConsumerWarps / R1;
+            const int rw = warp / Q, seg = warp % Q;
+            const int vlo = split_lo(nvec, Q, seg), vhi = split_lo(nvec, Q, seg + 1);
+            for (int rr = rw; rr < rows; rr += kConsumerWarps / Q) {
+                const uint4* wrow = slot + (size_t)rr * nvec;
+                float acc[NB][4];
+#pragma unroll
+                for (int t = 0; t < NB; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+#pragma unroll 4
+                for (int v = vlo + lane; v < vhi; v += 32) {
+                    const uint4 w = wrow[v];
+#pragma unroll
+                    for (int t = 0; t < NB; ++t)
+                        dot_mix<T>(acc[t], w, reinterpret_cast<const uint4*>(xs + (size_t)t * d)[v]);
+                }
+                float z[NB];
+#pragma unroll
+                for (int t = 0; t < NB; ++t) z[t] = warp_sum(sum4(acc[t]));
+                if (Q == 1) {
+                    if (lane == 0) {
+                        const float bias = S.bias1[r + rr - a0];
+                        for (int t = 0; t < B; ++t) p.h[(size_t)t * H + r + rr] = fmaxf(z[t] + bias, 0.f);
+                    }
+                } else if (lane == 0) {
+#pragma unroll
+                    for (int t = 0; t < NB; ++t) S.red2[warp * NB + t] = z[t];
+                }
+            }
+            if (r == a0) TRACE(12); else TRACE(14);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.pempty[s]);
+            if (Q > 1) {
+                consumer_sync();
+                if (tid < rows * NB) {
+                    const int rr = tid / NB, t = tid % NB;
+                    float zz = 0.f;
+                    for (int q = 0; q < Q; ++q) zz += S.red2[(rr * Q + q) * NB + t];
+                    if (t < B) p.h[(size_t)t * H + r + rr] = fmaxf(zz + S.bias1[r + rr - a0], 0.f);
+                }
+                consumer_sync();
+            }
+        }
+        TRACE(2);
+        if (!ok || !grid_barrier(S, p, epoch)) { ok = false; break; }
+        TRACE(3);
+
+        // -------------------------------------------------------------- phase B: logits, own FFN
+        // Lane l keeps h's 16-byte column groups v = l + 32 i in registers as fp32 pairs.
+        // Every selected neuron of this CTA's rows is appended (ascending) to the CTA's
+        // list as soon as its chunk is done, so the FFN producer starts gathering its
+        // W1/W2T rows while the rest of Wp2 still streams.
+        int m = 0;                                  // selected neurons of this CTA in this layer
+        {
+            constexpr int kHV = HV;                // H <= 256 * HV
+            // one L2 read of h per CTA (every CTA reads the same few lines: keep that traffic small)
+            for (int i = tid; i < (NB * H) >> 2; i += kConsumers)
+                reinterpret_cast<float4*>(S.hs)[i] = __ldcg(reinterpret_cast<const float4*>(p.h) + i);
+            consumer_sync();
+            u64 hr[kHV][4][NB];
+#pragma unroll
+            for (int i = 0; i < kHV; ++i) {
+                const int v = lane + 32 * i;
+#pragma unroll
+                for (int t = 0; t < NB; ++t) {
+                    if (v < hv) {
+                        const float4* hp = reinterpret_cast<const float4*>(S.hs + (size_t)t * H + v * 8);
+                        const float4 a = hp[0], b = hp[1];
+                        hr[i][0][t] = pk(a.x, a.y); hr[i][1][t] = pk(a.z, a.w);
+                        hr[i][2][t] = pk(b.x, b.y); hr[i][3][t] = pk(b.z, b.w);
+                    } else {
+                        hr[i][0][t] = hr[i][1][t] = hr[i][2][t] = hr[i][3][t] = 0ull;
+                    }
+                }
+            }
+            TRACE(4);
+            for (int r = b0; r < b1 && ok; r += R2, ++pk_) {
+                const int s = pk_ % p.pred_slots;
+                if (!cwait(S, p, &S.pfull[s], (pk_ / p.pred_slots) & 1)) { ok = false; break; }
+                if (r == b0) TRACE(5);
+                const uint4* slot = reinterpret_cast<const uint4*>(S.pring + (size_t)s * p.pred_slot_bytes);
+                const int rows = min(R2, b1 - r);
+                // two rows per warp per step for independent FMA chains
+                for (int rr = warp; rr < rows; rr += 2 * kConsumerWarps) {
+                    const int rr2 = rr + kConsumerWarps;
+                    const bool two = rr2 < rows;
+                    const uint4* w0p = slot + (size_t)rr * hv;
+                    const uint4* w1p = slot + (size_t)(two ? rr2 : rr) * hv;
+                    u64 a0[2][NB], a1[2][NB];
+#pragma unroll
+                    for (int t = 0; t < NB; ++t) a0[0][t] = a0[1][t] = a1[0][t] = a1[1][t] = 0ull;
+#pragma unroll
+                    for (int i = 0; i < kHV; ++i) {
+                        const int v = lane + 32 * i;
+                        if (v < hv) {
+                            const uint4 w0 = w0p[v], w1 = w1p[v];
+                            const u64 p00 = Arith<T>::widen2(w0.x), p01 = Arith<T>::widen2(w0.y);
+                            const u64 p02 = Arith<T>::widen2(w0.z), p03 = Arith<T>::widen2(w0.w);
+                            const u64 p10 = Arith<T>::widen2(w1.x), p11 = Arith<T>::widen2(w1.y);
+                            const u64 p12 = Arith<T>::widen2(w1.z), p13 = Arith<T>::widen2(w1.w);
+#pragma unroll
+                            for (int t = 0; t < NB; ++t) {
+                                ffma2(a0[0][t], p00, hr[i][0][t]); ffma2(a0[1][t], p01, hr[i][1][t]);
+                                ffma2(a0[0][t], p02, hr[i][2][t]); ffma2(a0[1][t], p03, hr[i][3][t]);
+                                ffma2(a1[0][t], p10, hr[i][0][t]); ffma2(a1[1][t], p11, hr[i][1][t]);
+                                ffma2(a1[0][t], p12, hr[i][2][t]); ffma2(a1[1][t], p13, hr[i][3][t]);
+                            }
+                        }
+                    }
+                    bool any0 = false, any1 = false;
+#pragma unroll
+                    for (int t = 0; t < NB; ++t) {
+                        const float2 x0 = upk(a0[0][t]), x1 = upk(a0[1][t]);
+                        const float2 y0 = upk(a1[0][t]), y1 = upk(a1[1][t]);
+                        const float z0 = warp_sum((x0.x + x0.y) + (x1.x + x1.y));
+                        const float z1 = warp_sum((y0.x + y0.y) + (y1.x + y1.y));
+                        if (t < B) {
+                            any0 |= (z0 + S.bias2[r + rr - b0]) > 0.f;
+                            if (two) any1 |= (z1 + S.bias2[r + rr2 - b0]) > 0.f;
+                        }
+                    }
+                    if (lane == 0) {
+                        S.sel[rr] = any0;
+                        if (two) S.sel[rr2] = any1;
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.pempty[s]);
+                consumer_sync();
+                // append this chunk's selected rows in ascending order and publish the count
+                if (warp == 0) {
+                    for (int q0 = 0; q0 < rows; q0 += 32) {
+                        const bool on = q0 + lane < rows && S.sel[q0 + lane];
+                        const uint32_t bal = __ballot_sync(0xffffffffu, on);
+                        if (on) S.nl[m + __popc(bal & ((1u << lane) - 1u))] = r + q0 + lane;
+                        m += __popc(bal);
+                    }
+                    __syncwarp();
+                    if (lane == 0) {
+                        __threadfence_block();
+                        S.flags[1] = (l << 16) | m;
+                    }
+                }
+            }
+        }
+        if (!ok) break;
+        consumer_sync();
+        {
+            const int f = S.flags[1];
+            m = ((f >> 16) & 0x7fff) == (l & 0x7fff) ? (f & 0xffff) : 0;   // no rows (b0 == b1): empty list
+        }
+        consumer_sync();
+        if (tid == 0) {
+            __threadfence_block();
+            S.flags[7] = l + 1;                       // the list of layer l is final
+            p.cta_count[c] = m;
+        }
+        TRACE(6);
+        {
+            // FC1 operand: this thread's x column vectors, packed storage pairs
+            uint4 xr[kMaxVPT][NB];
+#pragma unroll
+            for (int a = 0; a < kMaxVPT; ++a) {
+                const int v = tid + a * kConsumers;
+#pragma unroll
+                for (int t = 0; t < NB; ++t)
+                    xr[a][t] = v < nvec ? reinterpret_cast<const uint4*>(xs + (size_t)t * d)[v] : make_uint4(0, 0, 0, 0);
+            }
+            u64 acc[kMaxVPT][4][NB];
+#pragma unroll
+            for (int a = 0; a < kMaxVPT; ++a)
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int t = 0; t < NB; ++t) acc[a][q][t] = 0ull;
+            // neurons two at a time: one shared-memory reduction per pair
+            for (int i = 0; i < m; i += 2, fk += 2) {
+                const bool two = i + 1 < m;
+                const int s0 = fk % p.ffn_slots, s1 = (fk + 1) % p.ffn_slots;
+                if (!cwait(S, p, &S.ffull[s0], (fk / p.ffn_slots) & 1)) { ok = false; break; }
+                if (two && !cwait(S, p, &S.ffull[s1], ((fk + 1) / p.ffn_slots) & 1)) { ok = false; break; }
+                if (i == 0) TRACE(7);
+                const char* sl0 = S.fring + (size_t)s0 * fslot_bytes;
+                const char* sl1 = S.fring + (size_t)(two ? s1 : s0) * fslot_bytes;
+                float part[2][NB][4];
+#pragma unroll
+                for (int u = 0; u < 2; ++u)
+#pragma unroll
+                    for (int t = 0; t < NB; ++t) part[u][t][0] = part[u][t][1] = part[u][t][2] = part[u][t][3] = 0.f;
+#pragma unroll
+                for (int a = 0; a < kMaxVPT; ++a) {
+                    const int v = tid + a * kConsumers;
+                    if (v < nvec) {
+                        const uint4 w0 = reinterpret_cast<const uint4*>(sl0)[v];
+                        const uint4 w1 = reinterpret_cast<const uint4*>(sl1)[v];
+#pragma unroll
+                        for (int t = 0; t < NB; ++t) {
+                            dot_mix<T>(part[0][t], w0, xr[a][t]);
+                            dot_mix<T>(part[1][t], w1, xr[a][t]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 2; ++u)
+#pragma unroll
+                    for (int t = 0; t < NB; ++t) {
+                        const float v = warp_sum(sum4(part[u][t]));
+                        if (lane == 0) S.red[((rpar * 8 + warp) * 2 + u) * NB + t] = v;
+                    }
+                consumer_sync();
+                u64 av[2][NB];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const char* sl = u ? sl1 : sl0;
+                    const int j = S.nl[u ? (two ? i + 1 : i) : i];
+                    const float bias = DT<T>::f(reinterpret_cast<const T*>(sl + 4 * d)[j & 7]);
+#pragma unroll
+                    for (int t = 0; t < NB; ++t) {
+                        float z = 0.f;
+#pragma unroll
+                        for (int q = 0; q < kConsumerWarps; ++q) z += S.red[((rpar * 8 + q) * 2 + u) * NB + t];
+                        float a = fmaxf(z + bias, 0.f);
+                        if (u == 1 && !two) a = 0.f;
+                        av[u][t] = pk(a, a);
+                    }
+                }
+                rpar ^= 1;
+#pragma unroll
+                for (int a = 0; a < kMaxVPT; ++a) {
+                    const int v = tid + a * kConsumers;
+                    if (v < nvec) {
+                        const uint4 w0 = reinterpret_cast<const uint4*>(sl0 + 2 * d)[v];
+                        const uint4 w1 = reinterpret_cast<const uint4*>(sl1 + 2 * d)[v];
+                        const u64 q00 = Arith<T>::widen2(w0.x), q01 = Arith<T>::widen2(w0.y);
+                        const u64 q02 = Arith<T>::widen2(w0.z), q03 = Arith<T>::widen2(w0.w);
+#pragma unroll
+                        for (int t = 0; t < NB; ++t) {
+                            ffma2(acc[a][0][t], av[0][t], q00); ffma2(acc[a][1][t], av[0][t], q01);
+                            ffma2(acc[a][2][t], av[0][t], q02); ffma2(acc[a][3][t], av[0][t], q03);
+                        }
+                        if (two) {
+                            const u64 q10 = Arith<T>::widen2(w1.x), q11 = Arith<T>::widen2(w1.y);
+                            const u64 q12 = Arith<T>::widen2(w1.z), q13 = Arith<T>::widen2(w1.w);
+#pragma unroll
+                            for (int t = 0; t < NB; ++t) {
+                                ffma2(acc[a][0][t], av[1][t], q10); ffma2(acc[a][1][t], av[1][t], q11);
+                                ffma2(acc[a][2][t], av[1][t], q12); ffma2(acc[a][3][t], av[1][t], q13);
+                            }
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&S.fempty[s0]);
+                    if (two) mbar_arrive(&S.fempty[s1]);
+                }
+                if (!two) fk -= 1;               // only one slot consumed
+            }
+            if (!ok) break;
+#pragma unroll
+            for (int a = 0; a < kMaxVPT; ++a) {
+                const int v = tid + a * kConsumers;
+                if (v < nvec) {
+#pragma unroll
+                    for (int t = 0; t < NB; ++t) {
+                        float4* dst = reinterpret_cast<float4*>(p.partial + ((size_t)c * NB + t) * d + v * 8);
+                        const float2 e0 = upk(acc[a][0][t]), e1 = upk(acc[a][1][t]);
+                        const float2 e2 = upk(acc[a][2][t]), e3 = upk(acc[a][3][t]);
+                        __stcg(dst, make_float4(e0.x, e0.y, e1.x, e1.y));
+                        __stcg(dst + 1, make_float4(e2.x, e2.y, e3.x, e3.y));
+                    }
+                }
+            }
+        }
+        TRACE(8);
+        if (!grid_barrier(S, p, epoch)) { ok = false; break; }
+        TRACE(9);
+
+        // -------------------------------------------------------------- phase D: reduce, u = x + y
+        {
+            // neuron table of layer l: this CTA's ascending entries at their global positions
+            {
+                const int v = tid < G ? __ldcg(p.cta_count + tid) : 0;
+                if (tid < G) S.scan[tid] = v;
+            }
+        }
+        {
+            const int NG = d >> 2;                         // float4 column groups
+            const int g0 = split_lo(NG, G, c), g1 = split_lo(NG, G, c + 1);
+            const int tasks = (g1 - g0) * NB;
+            for (int task = warp; task < tasks; task += kConsumerWarps) {
+                const int g = g0 + task / NB, t = task % NB;
+                float4 v[kMaxG / 32];
+#pragma unroll
+                for (int i = 0; i < kMaxG / 32; ++i) {
+                    const int s = lane + 32 * i;
+                    v[i] = s < G ? __ldcg(reinterpret_cast<const float4*>(p.partial + ((size_t)s * NB + t) * d + g * 4))
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+                float4 a = v[0];
+#pragma unroll
+                for (int i = 1; i < kMaxG / 32; ++i) { a.x += v[i].x; a.y += v[i].y; a.z += v[i].z; a.w += v[i].w; }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    a.x += __shfl_xor_sync(0xffffffffu, a.x, o);
+                    a.y += __shfl_xor_sync(0xffffffffu, a.y, o);
+                    a.z += __shfl_xor_sync(0xffffffffu, a.z, o);
+                    a.w += __shfl_xor_sync(0xffffffffu, a.w, o);
+                }
+                if (lane == 0 && t < B) {
+                    float yv[4] = {a.x, a.y, a.z, a.w};
+                    float uv[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int col = g * 4 + q;
+                        yv[q] += S.biasy[col - g0 * 4];
+                        uv[q] = DT<T>::f(xs[(size_t)t * d + col]) + yv[q];
+                    }
+                    if (l == p.L - 1)
+                        *reinterpret_cast<float4*>(p.y + (size_t)t * d + g * 4) = make_float4(yv[0], yv[1], yv[2], yv[3]);
+                    __stcg(reinterpret_cast<float4*>(p.u + (size_t)t * d + g * 4), make_float4(uv[0], uv[1], uv[2], uv[3]));
+                }
+            }
+        }
+        consumer_sync();
+        if (warp == 0) {
+            int off = 0, tot = 0;
+            for (int g = lane; g < G; g += 32) {
+                const int v = S.scan[g];
+                off += g < c ? v : 0;
+                tot += v;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                off += __shfl_xor_sync(0xffffffffu, off, o);
+                tot += __shfl_xor_sync(0xffffffffu, tot, o);
+            }
+            for (int i = lane; i < m; i += 32) W.idx[off + i] = S.nl[i];
+            if (c == 0 && lane == 0 && p.counts) p.counts[l] = tot;
+        }
+        TRACE(10);
+        if (!grid_barrier(S, p, epoch)) { ok = false; break; }
+        TRACE(11);
+    }
+
+    // ---- drain: never leave a bulk copy in flight
+    if (!ok) {
+        if (tid == 0) {
+            const unsigned long long t0 = gtime();
+            while (!(S.flags[4] && S.flags[5]) && gtime() - t0 < kWaitNs) {}
+            const int pi = S.flags[2], fi = S.flags[3];
+            for (int k = pk_; k < pi; ++k) {
+                const unsigned long long t1 = gtime();
+                while (!mbar_try(&S.pfull[k % p.pred_slots], (k / p.pred_slots) & 1) && gtime() - t1 < kWaitNs) {}
+            }
+            for (int k = fk; k < fi; ++k) {
+                const unsigned long long t1 = gtime();
+                while (!mbar_try(&S.ffull[k % p.ffn_slots], (k / p.ffn_slots) & 1) && gtime() - t1 < kWaitNs) {}
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+unsigned long long* g_trace = nullptr;
+size_t g_trace_bytes = 0;
+
+int pow2_floor(int v) {
+    int r = 1;
+    while (r * 2 <= v) r *= 2;
+    return r;
+}
+
+struct Geometry {
+    int pred_slots, pred_slot_bytes, ffn_slots, R1, R2, max_rows;
+    size_t smem;
+};
+
+template <typename T, int NB>
+Geometry geometry(const spffn_config& c, int G) {
+    Geometry g;
+    const int budget = 227 * 1024;
+    g.pred_slot_bytes = 32 * 1024;
+    g.R1 = max(1, pow2_floor(g.pred_slot_bytes / (2 * c.d)));
+    g.R2 = max(1, pow2_floor(g.pred_slot_bytes / (2 * c.H)));
+    if (g.R2 > 32) g.R2 = 32;
+    if (g.R1 > 32) g.R1 = 32;
+    g.max_rows = (c.n + G - 1) / G + 1;
+    size_t fixed = 0;
+    fixed += ((size_t)NB * c.d * sizeof(T) + 127) / 128 * 128;      // xs
+    fixed += ((size_t)NB * c.H * 4 + 127) / 128 * 128;              // hs
+    fixed += (g.max_rows + 127) / 128 * 128;                         // sel
+    fixed += ((size_t)g.max_rows * 4 + 127) / 128 * 128;             // nl
+    fixed += ((size_t)(c.n / 32) * 4 + 127) / 128 * 128;             // maskw
+    fixed += ((size_t)(c.H / G + 2) * 4 + 127) / 128 * 128;          // bias1
+    fixed += ((size_t)g.max_rows * 4 + 127) / 128 * 128;             // bias2
+    fixed += ((size_t)(c.d / G + 8) * 4 + 127) / 128 * 128;          // biasy
+    fixed += 2 * 8 * 2 * NB * 4 + 8 * NB * 4 + (kMaxG + 1) * 4 + 16 * 4 + 16;
+    fixed += 8 * (2 * 8 + 2 * 8 + 1) + 8 * 8 + 128;                  // barriers + flags + slack
+    const size_t fslot = 4 * (size_t)c.d + 128;
+    g.pred_slots = 4;
+    g.ffn_slots = 8;
+    auto total = [&]() { return fixed + (size_t)g.pred_slots * g.pred_slot_bytes + g.ffn_slots * fslot; };
+    while (total() > (size_t)budget && g.ffn_slots > 3) --g.ffn_slots;
+    while (total() > (size_t)budget && g.pred_slots > 3) --g.pred_slots;
+    while (total() > (size_t)budget && g.ffn_slots > 2) --g.ffn_slots;
+    while (total() > (size_t)budget && g.pred_slots > 2) --g.pred_slots;
+    g.smem = total();
+    return g;
+}
+
+template <typename T, int NB, int HV>
+cudaError_t launch_t(spffn_ctx* const* layers, int L, const void* x_in, int B, void* x_out, float* y,
+                     int32_t* counts, cudaStream_t st)
+{
+    const spffn_ctx& c0 = *layers[0];
+    const int G = c0.lay.S;
+    Geometry g = geometry<T, NB>(c0.cfg, G);
+    if (g.smem > 227 * 1024) return cudaErrorInvalidConfiguration;
+    static Params p;   // host staging copy; the launch copies it into the kernel's parameter space
+    p.L = L; p.B = B; p.d = c0.cfg.d; p.n = c0.cfg.n; p.H = c0.cfg.H; p.G = G;
+    p.x_in = x_in; p.x_out = x_out; p.y = y; p.counts = counts;
+    Ctl* ctl = c0.ctl();
+    p.bar = &ctl->barrier[0];
+    p.err = &ctl->err;
+    p.abort = &ctl->barrier[1];
+    p.mask = c0.mask2();
+    p.cta_count = c0.ctacnt();
+    p.h = c0.h();
+    p.partial = c0.partial();
+    p.u = c0.ybuf();
+    p.ss = c0.ssbuf();
+    p.pred_slots = g.pred_slots; p.pred_slot_bytes = g.pred_slot_bytes; p.ffn_slots = g.ffn_slots;
+    p.R1 = g.R1; p.R2 = g.R2; p.max_rows = g.max_rows;
+    p.trace = (g_trace && g_trace_bytes >= (size_t)G * L * kTraceMarks * 8) ? g_trace : nullptr;
+    for (int l = 0; l < L; ++l) {
+        const spffn_ctx& c = *layers[l];
+        p.layer[l] = LayerW{c.w.W1, c.w.b1, c.w.W2T, c.w.b2, c.w.Wp1, c.w.bp1, c.w.Wp2, c.w.bp2, c.idx()};
+    }
+    cudaError_t e = cudaFuncSetAttribute(k_decode<T, NB, HV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem);
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(&ctl->barrier[0], 0, 2 * sizeof(uint32_t), st);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(G);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = g.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_decode<T, NB, HV>, p);
+}
+
+}  // namespace
+
+bool fused_decode_supported(spffn_ctx* const* layers, int L, int B)
+{
+    if (L < 1 || L > kMaxFusedLayers || B < 1 || B > 2) return false;
+    const spffn_config& c0 = layers[0]->cfg;
+    if (c0.d > kMaxVPT * 8 * kConsumers) return false;
+    if (layers[0]->lay.S > kMaxG) return false;
+    if (c0.n / 32 > kMaxMaskWords) return false;
+    if (c0.H > 2048 || (B == 2 && c0.H > 1024)) return false;   // h lives in registers
+    for (int l = 1; l < L; ++l) {
+        const spffn_config& c = layers[l]->cfg;
+        if (c.d != c0.d || c.n != c0.n || c.H != c0.H || c.dtype != c0.dtype) return false;
+    }
+    if (layers[0]->lay.S != layers[0]->num_sms) return false;
+    return true;
+}
+
+void set_trace(void* buf, size_t bytes)
+{
+    g_trace = static_cast<unsigned long long*>(buf);
+    g_trace_bytes = buf ? bytes : 0;
+}
+
+int trace_marks() { return kTraceMarks; }
+
+cudaError_t launch_fused_decode(spffn_ctx* const* layers, int L, const void* x_in, int B, void* x_out, float* y,
+                                int32_t* counts, cudaStream_t st)
+{
+    const bool bf = layers[0]->cfg.dtype == SPFFN_BF16;
+    const int hvn = (layers[0]->cfg.H + 255) / 256;
+#define SPFFN_GO(TT, NBV, HVV) return launch_t<TT, NBV, HVV>(layers, L, x_in, B, x_out, y, counts, st)
+#define SPFFN_HV(TT, NBV)                                     \
+    if (hvn <= 1) SPFFN_GO(TT, NBV, 1);                       \
+    if (hvn <= 2) SPFFN_GO(TT, NBV, 2);                       \
+    if (hvn <= 4) SPFFN_GO(TT, NBV, 4);                       \
+    if (NBV == 1) SPFFN_GO(TT, 1, 8);                         \
+    return cudaErrorInvalidValue;
+    if (B == 1) {
+        if (bf) { SPFFN_HV(__nv_bfloat16, 1) } else { SPFFN_HV(__half, 1) }
+    }
+    if (bf) { SPFFN_HV(__nv_bfloat16, 2) } else { SPFFN_HV(__half, 2) }
+#undef SPFFN_HV
+#undef SPFFN_GO
+}
+
 }  // namespace spffn

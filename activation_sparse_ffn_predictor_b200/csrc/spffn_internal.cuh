@@ -28,7 +28,7 @@ struct Ctl {
 };
 
 struct Layout {
-    size_t ctl, h, mask, wcount, partial, xbuf, ybuf, idx, count, total;
+    size_t ctl, h, mask, wcount, partial, xbuf, ybuf, idx, count, mask2, ctacnt, ssbuf, total;
     int S;  // number of FFN partial sums
 };
 
@@ -48,6 +48,9 @@ inline Layout make_layout(const spffn_config& c, int S) {
     L.ybuf = take((size_t)c.max_batch * c.d * sizeof(float));
     L.idx = take((size_t)c.n * sizeof(int32_t));
     L.count = take(256);
+    L.mask2 = take((size_t)2 * (c.n / 32) * sizeof(uint32_t));
+    L.ctacnt = take((size_t)(S + 1) * sizeof(int32_t));
+    L.ssbuf = take((size_t)S * c.max_batch * sizeof(float));
     L.total = off;
     return L;
 }
@@ -72,6 +75,9 @@ struct spffn_ctx {
     float* ybuf() const { return reinterpret_cast<float*>(ws + lay.ybuf); }
     int32_t* idx() const { return reinterpret_cast<int32_t*>(ws + lay.idx); }
     int32_t* count() const { return reinterpret_cast<int32_t*>(ws + lay.count); }
+    uint32_t* mask2() const { return reinterpret_cast<uint32_t*>(ws + lay.mask2); }
+    int32_t* ctacnt() const { return reinterpret_cast<int32_t*>(ws + lay.ctacnt); }
+    float* ssbuf() const { return reinterpret_cast<float*>(ws + lay.ssbuf); }
 };
 
 namespace spffn {

@@ -161,7 +161,8 @@ def build_stack(cfg, layers, device, rate=None, reorder=True, log=print):
             Xp = wl.to_torch(wl.tokens(cfg, PROFILE_TOKENS, aux=l, tensor=wl.T_XPROF), cfg, device)
             counts = torch.zeros(cfg.n, dtype=torch.int32, device=device)
             L.profile_counts(Xp, counts)
-            perm = sp.reorder(counts.cpu().numpy().astype(np.uint32))
+            # hot-first order dealt over the decode kernel's per-CTA row ranges
+            perm = sp.reorder_dealt(counts.cpu().numpy().astype(np.uint32), L.num_partials)
             pt = torch.from_numpy(perm).to(device)
             for name in ("W1", "W2T", "Wp2"):
                 src = getattr(dl, name)
@@ -211,7 +212,7 @@ def run_ours(args, cfg, world, rank, local):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
         one_step()
-    launches_per_step = args.launches_per_step or _count_launches_per_step(L)
+    launches_per_step = sp.decode_kernel_launches(layers, B)
 
     with torch.cuda.stream(stream):
         for s in range(W):
@@ -271,7 +272,7 @@ def run_ours(args, cfg, world, rank, local):
         "config": {"workload": cfg.name, "layers": L, "d": cfg.d, "n": cfg.n, "H": cfg.H, "batch": B,
                    "activation_rate": args.rate or cfg.rate, "alpha": cfg.alpha, "global_batch": B * world,
                    "mean_active_neurons": float(ks.mean()), "parallelism": "replicas%d" % world,
-                   "reordered": True, "l2": "inputs larger than L2 (%.2f GB touched per step)"
+                   "placement": "hot-first dealt over %d CTA ranges (offline profile of %d tokens)" % (layers[0].num_partials, PROFILE_TOKENS), "l2": "inputs larger than L2 (%.2f GB touched per step)"
                    % (sum(bytes_per_step) / K / 1e9)},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": None,
@@ -282,11 +283,6 @@ def run_ours(args, cfg, world, rank, local):
         "clocks": clk.summary(),
     }
     return res, (rank == 0)
-
-
-def _count_launches_per_step(L):
-    import activation_sparse_ffn_predictor_b200 as sp
-    return sp.launches_per_decode(L) if hasattr(sp, "launches_per_decode") else 6 * L
 
 
 # ---------------------------------------------------------------------------
@@ -373,7 +369,6 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle compute for cpu_baseline")
     ap.add_argument("--ref-budget", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--launches-per-step", type=int, default=0)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -146,6 +146,11 @@ spffn_status spffn_chain(spffn_ctx* ctx, const void* x, const float* y, int32_t 
 spffn_status spffn_decode(spffn_ctx* const* layers, int32_t L, const void* x_in, int32_t B,
                           void* x_out, float* y, int32_t* counts, void* stream);
 
+/* Number of kernels one spffn_decode call with these arguments enqueues (the
+ * persistent whole-stack kernel: 1; otherwise 6 per layer), 0 on bad arguments.
+ * Pure host function. */
+int32_t spffn_decode_kernel_launches(spffn_ctx* const* layers, int32_t L, int32_t B);
+
 /* Offline profiler ([PI1] §5.1): for T profiling tokens X [T][d] (device,
  * storage dtype), counts[j] += #{t : W1[j].X_t + b1_j > 0}.  counts: device
  * uint32 [n], accumulated (caller zeroes it before the first batch). */
@@ -156,6 +161,14 @@ spffn_status spffn_profile_counts(spffn_ctx* ctx, const void* X, int32_t T, uint
  * arrays; perm[s] = original neuron placed in slot s, ordering by count
  * descending, ties by original index ascending.  Pure host function. */
 spffn_status spffn_reorder(const uint32_t* counts_host, int32_t n, int32_t* perm_host);
+
+/* Hot-first placement dealt over `parts` contiguous slot ranges (range c =
+ * slots [floor(n c / parts), floor(n (c+1) / parts))): neurons in hot-first
+ * order (as spffn_reorder) are dealt round-robin, the i-th hottest going to
+ * range i mod parts, filling each range in ascending slots.  With parts =
+ * spffn_num_partials(), every CTA of the whole-stack decode kernel owns a range
+ * with the same expected activity.  Pure host function. */
+spffn_status spffn_reorder_dealt(const uint32_t* counts_host, int32_t n, int32_t parts, int32_t* perm_host);
 
 /* Row gather applying a neuron table: dst row s = src row perm[s], for `rows`
  * rows of `row_bytes` bytes (row_bytes % 16 == 0).  src, dst, perm: device;
@@ -169,10 +182,27 @@ spffn_status spffn_permute_rows(const void* src, void* dst, int32_t rows, int32_
 spffn_status spffn_permute_vector(const void* src, void* dst, int32_t count, const int32_t* perm,
                                   void* stream);
 
+/* Tracing aid: bind a device buffer (or NULL to unbind) into which later
+ * whole-stack decode launches write %globaltimer stamps (u64 nanoseconds),
+ * laid out [CTA][layer][spffn_trace_marks()], at fixed points of each layer:
+ * 0 input formed, 1 first predictor-1 chunk ready, 2 hidden layer done,
+ * 3 after barrier, 4 h loaded, 5 first predictor-2 chunk ready, 6 own
+ * neuron list final, 7 first FFN rows ready, 8 FFN partial written, 9 after
+ * barrier, 10 reduction and table written, 11 after barrier, 12 first
+ * predictor-1 chunk computed, 13/14 later predictor-1 chunk ready/computed.
+ * A mark a CTA does not reach in a layer (no rows or no neurons) stays 0.
+ * Buffers smaller than that are ignored.  Process-wide; not thread-safe. */
+spffn_status spffn_set_trace(void* buf, size_t bytes);
+int32_t spffn_trace_marks(void);
+
 /* Read and clear the context's device error word (synchronises `stream`).
  * Returns SPFFN_OK if clean, SPFFN_ERR_DEVICE_CHECK or SPFFN_ERR_TIMEOUT;
  * *code (may be NULL) receives the raw word. */
 spffn_status spffn_last_device_error(spffn_ctx* ctx, uint32_t* code, void* stream);
+
+/* Description of the CUDA error behind the calling thread's most recent
+ * SPFFN_ERR_CUDA (static string). */
+const char* spffn_last_cuda_error_string(void);
 
 /* Static description of a status code. */
 const char* spffn_status_string(spffn_status s);

@@ -173,6 +173,27 @@ def hot_first_order(counts) -> np.ndarray:
     return np.lexsort((np.arange(c.size), -c)).astype(np.int32)
 
 
+def dealt_order(counts, parts: int) -> np.ndarray:
+    """Hot-first order dealt over ``parts`` contiguous slot ranges: range c holds
+    slots [floor(n c/parts), floor(n (c+1)/parts)); the i-th hottest neuron (per
+    hot_first_order) goes to range i mod parts, into its next free slot.  A
+    placement choice of this library (impact-ordered, [PI1] §5.2 equation (1)),
+    spreading hot neurons evenly over the ranges."""
+    hot = hot_first_order(counts)
+    n = hot.size
+    bounds = [n * c // parts for c in range(parts + 1)]
+    fill = [bounds[c] for c in range(parts)]
+    perm = np.empty(n, dtype=np.int32)
+    c = 0
+    for neuron in hot:
+        while fill[c] >= bounds[c + 1]:      # range already full: next range
+            c = (c + 1) % parts
+        perm[fill[c]] = neuron
+        fill[c] += 1
+        c = (c + 1) % parts
+    return perm
+
+
 def permute_rows(a, perm) -> np.ndarray:
     """Apply the neuron table: row ``s`` of the result is row ``perm[s]``."""
     return np.asarray(a)[np.asarray(perm, dtype=np.int64)]

@@ -86,3 +86,13 @@ def test_reorder_matches_oracle():
     for n in (1, 7, 64, 5000):
         c = r.integers(0, 6, n).astype(np.uint32)   # many ties
         assert np.array_equal(sp.reorder(c), O.hot_first_order(c))
+
+
+def test_reorder_dealt_matches_oracle():
+    r = np.random.default_rng(1)
+    for n, parts in ((7, 3), (64, 148), (4096, 148), (16384, 148), (1000, 7)):
+        c = r.integers(0, 50, n).astype(np.uint32)
+        got = sp.reorder_dealt(c, parts)
+        want = O.dealt_order(c, parts)
+        assert np.array_equal(got, want)
+        assert sorted(got.tolist()) == list(range(n))

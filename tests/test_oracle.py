@@ -233,3 +233,12 @@ def test_chain_closed_forms():
     ms = np.mean((x + y) ** 2, axis=1)
     np.testing.assert_allclose(np.sqrt(np.mean(out ** 2, axis=1)), np.sqrt(ms / (ms + O.RMS_EPS)), rtol=1e-13)
     np.testing.assert_allclose(out * np.sqrt(ms + O.RMS_EPS)[:, None], x + y, rtol=1e-13)
+
+
+def test_dealt_order_hand_example():
+    # counts: neuron 4 hottest, then 1, 6, 0, 3, 2, 5 (ties by index)
+    counts = np.array([5, 8, 1, 4, 9, 1, 7], dtype=np.uint32)
+    assert O.hot_first_order(counts).tolist() == [4, 1, 6, 0, 3, 2, 5]
+    # 3 ranges over 7 slots: [0,2) [2,4) [4,7); deal 4->r0, 1->r1, 6->r2, 0->r0, 3->r1, 2->r2, 5->r2
+    assert O.dealt_order(counts, 3).tolist() == [4, 0, 1, 3, 6, 2, 5]
+    assert O.dealt_order(counts, 1).tolist() == O.hot_first_order(counts).tolist()

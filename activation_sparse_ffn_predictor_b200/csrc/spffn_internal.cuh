@@ -18,6 +18,8 @@ enum : uint32_t {
 
 constexpr int kMaxBatch = 32;
 constexpr int kCtlBytes = 1024;    // control block at the head of the workspace
+constexpr int kMaxUnionCtas = 256;  // union path: split-K partial capacity in CTAs
+constexpr int kUnionTickets = 2048;
 
 // Control block (u32 words) at the start of every workspace.
 struct Ctl {
@@ -28,7 +30,7 @@ struct Ctl {
 };
 
 struct Layout {
-    size_t ctl, h, mask, wcount, partial, xbuf, ybuf, idx, count, mask2, ctacnt, ssbuf, total;
+    size_t ctl, h, mask, wcount, partial, xbuf, ybuf, idx, count, mask2, ctacnt, ssbuf, hsplit, asplit, upartial, utickets, total;
     int S;  // number of FFN partial sums
 };
 
@@ -51,6 +53,14 @@ inline Layout make_layout(const spffn_config& c, int S) {
     L.mask2 = take((size_t)2 * (c.n / 32) * sizeof(uint32_t));
     L.ctacnt = take((size_t)(S + 1) * sizeof(int32_t));
     L.ssbuf = take((size_t)S * c.max_batch * sizeof(float));
+    L.hsplit = take((size_t)2 * c.max_batch * c.H * 2);
+    L.asplit = take((size_t)2 * c.max_batch * c.n * 2);
+    if (c.max_batch >= 16) {
+        L.upartial = take((size_t)kMaxUnionCtas * 128 * 64 * sizeof(float));
+        L.utickets = take((size_t)kUnionTickets * sizeof(uint32_t));
+    } else {
+        L.upartial = L.utickets = 0;
+    }
     L.total = off;
     return L;
 }
@@ -78,6 +88,10 @@ struct spffn_ctx {
     uint32_t* mask2() const { return reinterpret_cast<uint32_t*>(ws + lay.mask2); }
     int32_t* ctacnt() const { return reinterpret_cast<int32_t*>(ws + lay.ctacnt); }
     float* ssbuf() const { return reinterpret_cast<float*>(ws + lay.ssbuf); }
+    void* hsplit() const { return ws + lay.hsplit; }
+    void* asplit() const { return ws + lay.asplit; }
+    float* upartial() const { return reinterpret_cast<float*>(ws + lay.upartial); }
+    uint32_t* utickets() const { return reinterpret_cast<uint32_t*>(ws + lay.utickets); }
 };
 
 namespace spffn {

@@ -6,6 +6,7 @@
 // accumulation throughout; every reduction has a fixed order.
 #include "spffn_internal.cuh"
 #include "spffn_kernels.cuh"
+#include "spffn_union.cuh"
 
 namespace spffn {
 
@@ -401,9 +402,16 @@ static cudaError_t profile_impl(const spffn_ctx& c, const void* X, int T_, uint3
     return cudaGetLastError();
 }
 
+cudaError_t launch_compact(const spffn_ctx& c, int32_t* idx, int32_t* count, int32_t* count2, cudaStream_t st)
+{
+    k_compact<<<1, 1024, 0, st>>>(c.mask(), c.wcount(), c.cfg.n / 32, idx, count, count2);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_predict(const spffn_ctx& c, const void* x, int B, int32_t* idx, int32_t* count,
                            int32_t* count2, cudaStream_t st)
 {
+    if (union_supported(c, B)) return union_predict(c, x, B, idx, count, count2, st);
     return c.cfg.dtype == SPFFN_BF16 ? predict_impl<__nv_bfloat16>(c, x, B, idx, count, count2, st)
                                      : predict_impl<__half>(c, x, B, idx, count, count2, st);
 }
@@ -411,6 +419,7 @@ cudaError_t launch_predict(const spffn_ctx& c, const void* x, int B, int32_t* id
 cudaError_t launch_forward(const spffn_ctx& c, const void* x, int B, const int32_t* idx, const int32_t* count,
                            float* y, cudaStream_t st)
 {
+    if (union_supported(c, B)) return union_forward(c, x, B, idx, count, y, st);
     return c.cfg.dtype == SPFFN_BF16 ? forward_impl<__nv_bfloat16>(c, x, B, idx, count, y, st)
                                      : forward_impl<__half>(c, x, B, idx, count, y, st);
 }

@@ -1,0 +1,568 @@
+// Union-mask tensor-core path for batches of 16..32 tokens.
+//
+// With B tokens the union of the per-token neuron sets is a dense contraction
+// over the gathered rows (each weight byte feeds B products), so every GEMM of
+// the layer runs on the 5th-generation tensor cores:
+//
+//   mode 0  predictor-1   D[H x B]   = Wp1[H x d]        . X[B x d]^T        split-K
+//   mode 1  predictor-2   D[n x 2B]  = Wp2[n x H]        . hsplit[2B x H]^T  -> mask words
+//   mode 2  FC1 (union)   D[U x B]   = W1[table][U x d]  . X[B x d]^T        split-K
+//   mode 3  FC2 (union)   D[d x 2B]  = W2T[table]^T      . asplit[2B x U]^T  split-K
+//
+// fp32 activations (h, a) enter the 16-bit MMA as a hi/lo pair of the storage
+// dtype (v ~= hi + lo, hi = round(v), lo = round(v - hi)); the epilogue adds the
+// two column halves of D.  X is already in the storage dtype (exact).
+//
+// One persistent CTA per SM; warp 0 issues TMA loads into a 6-stage ring
+// (2-D tiles for contiguous operands, tile::gather4 for the rows named by the
+// neuron table; never multicast), warp 1 issues tcgen05.mma into a double
+// buffered TMEM accumulator, warps 2..5 read TMEM (tcgen05.ld) and run the
+// epilogue.  Split-K partials are summed in fixed split order by the last CTA
+// to finish a tile (atomic ticket, no waiting), so results are deterministic.
+#include <cuda.h>
+#include <algorithm>
+#include <cstring>
+#include "spffn_internal.cuh"
+#include "spffn_union.cuh"
+
+namespace spffn {
+namespace {
+
+constexpr int kUThreads = 192;       // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kBM = 128;             // D rows per tile
+constexpr int kBK = 64;              // K per stage: one 128-byte swizzle row of 16-bit elements
+constexpr int kStages = 6;
+constexpr int kStageBytes = 24 * 1024;   // A tile 16 KB + B tile up to 8 KB
+constexpr int kTmemCols = 128;       // two accumulators of up to 64 fp32 columns
+constexpr unsigned long long kUWaitNs = 2000000000ull;
+
+struct alignas(64) UParams {
+    CUtensorMap tmA;
+    CUtensorMap tmB;
+    int mode, B, N, dtype;
+    int M;                // D rows when known on the host (modes 0, 1, 3)
+    int K;                // contraction length when known on the host (modes 0, 1, 2)
+    int n, d, H, G;
+    int splits_fixed;     // mode 0
+    const int32_t* count; // modes 2, 3: table length U (device)
+    const int32_t* idx;   // modes 2, 3: neuron table
+    const void* bias;     // bp1, bp2, b1 (by neuron), b2
+    float* partial;       // [units][kBM][N]
+    uint32_t* tickets;    // [tiles]
+    void* out_split;      // mode 0: hsplit [2B][H]; mode 2: asplit [2B][n]
+    float* out_f32;       // mode 0: h [B][H] (may be null); mode 3: y [B][d]
+    uint32_t* mask;       // mode 1
+    uint32_t* wcount;     // mode 1
+    uint32_t* err;
+};
+
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t s32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ unsigned long long now_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void ub_init(uint64_t* b, uint32_t c) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(s32(b)), "r"(c) : "memory");
+}
+__device__ __forceinline__ void ub_expect(uint64_t* b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(s32(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void ub_arrive(uint64_t* b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(s32(b)) : "memory");
+}
+__device__ __forceinline__ bool ub_try(uint64_t* b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(s32(b)), "r"(parity) : "memory");
+    return ok != 0;
+}
+// Bounded wait; false on timeout (latches the error) or when the CTA is aborting.
+__device__ __forceinline__ bool ub_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag, uint32_t* err) {
+    if (ub_try(b, parity)) return true;
+    const unsigned long long t0 = now_ns();
+    while (!ub_try(b, parity)) {
+        if (*abort_flag) return false;
+        if (now_ns() - t0 > kUWaitNs) {
+            *abort_flag = 1;
+            atomicOr(err, ERR_PIPE_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+__device__ __forceinline__ void tma_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(s32(dst)), "l"(map), "r"(x), "r"(y), "r"(s32(bar)) : "memory");
+}
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int x, int y0, int y1, int y2, int y3,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
+        ::"r"(s32(dst)), "l"(map), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(s32(bar)) : "memory");
+}
+// shared-memory matrix descriptor, 128-byte swizzle
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo16, uint32_t sbo16) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)lbo16 << 16) | ((uint64_t)sbo16 << 32) |
+           (1ull << 46) | (2ull << 61);
+}
+__device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accum) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+        ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(accum), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+}
+__device__ __forceinline__ void ucommit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(s32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+
+// Work decomposition shared by all three roles (same answer in every thread).
+struct Plan {
+    int tiles, splits, kblocks, M, K;
+};
+__device__ __forceinline__ Plan make_plan(const UParams& p) {
+    Plan q;
+    if (p.mode == 2) {
+        int U = *reinterpret_cast<const volatile int32_t*>(p.count);
+        U = U < 0 ? 0 : (U > p.n ? p.n : U);
+        q.M = U;
+        q.K = p.K;
+    } else if (p.mode == 3) {
+        int U = *reinterpret_cast<const volatile int32_t*>(p.count);
+        U = U < 0 ? 0 : (U > p.n ? p.n : U);
+        q.M = p.M;
+        q.K = U;
+    } else {
+        q.M = p.M;
+        q.K = p.K;
+    }
+    q.tiles = (q.M + kBM - 1) / kBM;
+    q.kblocks = (q.K + kBK - 1) / kBK;
+    if (p.mode == 0) {
+        q.splits = p.splits_fixed;
+    } else if (p.mode == 1) {
+        q.splits = 1;
+    } else {
+        const int s = q.tiles > 0 ? p.G / q.tiles : 1;
+        q.splits = max(1, min(s, q.kblocks));
+    }
+    if (q.kblocks > 0 && q.splits > q.kblocks) q.splits = q.kblocks;
+    return q;
+}
+
+template <typename T>
+__device__ __forceinline__ float tof(const void* base, int i) {
+    return DT<T>::f(reinterpret_cast<const T*>(base)[i]);
+}
+
+// Final epilogue for one D row (this thread's TMEM lane) and all its columns.
+template <typename T>
+__device__ void finish_row(const UParams& p, const Plan& q, int tile, int lane_row, const float* v) {
+    const int r = tile * kBM + lane_row;
+    const int B = p.B;
+    if (p.mode == 0) {                      // h = ReLU(D + bp1) -> fp32 and hi/lo pair
+        if (r < p.H) {
+            const float bias = p.bias ? tof<T>(p.bias, r) : 0.f;
+            T* hs = reinterpret_cast<T*>(p.out_split);
+            for (int t = 0; t < B; ++t) {
+                const float h = fmaxf(v[t] + bias, 0.f);
+                const T hi = DT<T>::r(h);
+                const T lo = DT<T>::r(h - DT<T>::f(hi));
+                hs[(size_t)t * p.H + r] = hi;
+                hs[(size_t)(B + t) * p.H + r] = lo;
+                if (p.out_f32) p.out_f32[(size_t)t * p.H + r] = h;
+            }
+        }
+    } else if (p.mode == 1) {               // union decision, 32 rows per mask word
+        bool any = false;
+        if (r < p.n) {
+            const float bias = p.bias ? tof<T>(p.bias, r) : 0.f;
+            for (int t = 0; t < B; ++t) any |= (v[t] + v[B + t] + bias) > 0.f;
+        }
+        const uint32_t bits = __ballot_sync(0xffffffffu, any);
+        const int word = (tile * kBM + (lane_row & ~31)) >> 5;
+        if ((threadIdx.x & 31) == 0 && word < (p.n >> 5)) {
+            p.mask[word] = bits;
+            p.wcount[word] = __popc(bits);
+        }
+    } else if (p.mode == 2) {               // a = ReLU(D + b1[j]) for table entry r (zeros past U)
+        T* as = reinterpret_cast<T*>(p.out_split);
+        if (r < p.n) {
+            const bool live = r < q.M;
+            const float bias = live ? tof<T>(p.bias, p.idx[r]) : 0.f;
+            for (int t = 0; t < B; ++t) {
+                const float a = live ? fmaxf(v[t] + bias, 0.f) : 0.f;
+                const T hi = DT<T>::r(a);
+                const T lo = DT<T>::r(a - DT<T>::f(hi));
+                as[(size_t)t * p.n + r] = hi;
+                as[(size_t)(B + t) * p.n + r] = lo;
+            }
+        }
+    } else {                                // y[t][c] = D[c][t] + D[c][B+t] + b2[c]
+        if (r < p.d) {
+            const float bias = p.bias ? tof<T>(p.bias, r) : 0.f;
+            for (int t = 0; t < B; ++t) p.out_f32[(size_t)t * p.d + r] = v[t] + v[B + t] + bias;
+        }
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ UParams p)
+{
+    extern __shared__ __align__(1024) char usm[];
+    char* base = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(usm) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + kStages * kStageBytes);
+    uint64_t* empty = full + kStages;
+    uint64_t* tfull = empty + kStages;       // [2]
+    uint64_t* tempty = tfull + 2;            // [2]
+    uint64_t* done = tempty + 2;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(done + 1);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 2);
+    int* s_last = reinterpret_cast<int*>(done + 3);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; ++i) { ub_init(&full[i], 1); ub_init(&empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { ub_init(&tfull[i], 1); ub_init(&tempty[i], 4); }
+        ub_init(done, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(s32(tmem_slot)),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const Plan q = make_plan(p);
+    const int units = q.tiles * q.splits;
+    const int N = p.N;
+    const uint32_t btile_bytes = (uint32_t)N * 128u;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------- TMA producer (whole warp)
+        int st = 0, ph = 0;
+        for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
+            const int tile = u / q.splits, sp = u % q.splits;
+            const int kb0 = (int)((long long)sp * q.kblocks / q.splits);
+            const int kb1 = (int)((long long)(sp + 1) * q.kblocks / q.splits);
+            int jr[4] = {0, 0, 0, 0};           // FC1: this lane's 4 table rows of the tile
+            if (p.mode == 2) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = tile * kBM + lane * 4 + i;
+                    jr[i] = p.idx[r < q.M ? r : 0];
+                }
+            }
+            for (int kb = kb0; kb < kb1; ++kb) {
+                bool okw = true;
+                if (lane == 0) okw = ub_wait(&empty[st], ph ^ 1, abort_flag, p.err);
+                okw = __shfl_sync(0xffffffffu, okw, 0);
+                if (!okw) break;
+                char* sa = base + st * kStageBytes;
+                char* sb = sa + 16384;
+                if (lane == 0) ub_expect(&full[st], 16384u + btile_bytes);
+                __syncwarp();
+                if (p.mode <= 1) {
+                    if (lane == 0) tma_2d(sa, &p.tmA, kb * kBK, tile * kBM, &full[st]);
+                } else if (p.mode == 2) {
+                    // 128 table rows of W1: lane l gathers rows 4l..4l+3 of this tile
+                    tma_gather4(sa + lane * 512, &p.tmA, kb * kBK, jr[0], jr[1], jr[2], jr[3], &full[st]);
+                } else {
+                    // 64 table rows (the K block) x 128 columns of W2T, as two 64-column blocks
+                    const int mb = lane >> 4, g = lane & 15;
+                    int j[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int r = kb * kBK + g * 4 + i;
+                        j[i] = p.idx[r < q.K ? r : 0];
+                    }
+                    tma_gather4(sa + mb * 8192 + g * 512, &p.tmA, tile * kBM + mb * 64, j[0], j[1], j[2], j[3],
+                                &full[st]);
+                }
+                if (lane == 0) tma_2d(sb, &p.tmB, kb * kBK, 0, &full[st]);
+                if (++st == kStages) { st = 0; ph ^= 1; }
+            }
+        }
+        // on abort, give copies already issued time to land before the CTA retires
+        if (lane == 0 && *abort_flag) {
+            const unsigned long long t0 = now_ns();
+            while (now_ns() - t0 < 200000ull) {}
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------- MMA issuer (one thread)
+        if (lane == 0) {
+            const uint32_t idesc = (1u << 4) | ((uint32_t)p.dtype << 7) | ((uint32_t)p.dtype << 10) |
+                                   ((p.mode == 3 ? 1u : 0u) << 15) | ((uint32_t)(N >> 3) << 17) |
+                                   ((uint32_t)(kBM >> 4) << 24);
+            int st = 0, ph = 0, ab = 0, aph = 0;
+            bool issued = false;
+            for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
+                const int sp = u % q.splits;
+                const int kb0 = (int)((long long)sp * q.kblocks / q.splits);
+                const int kb1 = (int)((long long)(sp + 1) * q.kblocks / q.splits);
+                if (kb1 == kb0) continue;
+                if (!ub_wait(&tempty[ab], aph ^ 1, abort_flag, p.err)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(ab * N);
+                bool okm = true;
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!ub_wait(&full[st], ph, abort_flag, p.err)) { okm = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = s32(base + st * kStageBytes), sb = sa + 16384u;
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k) {
+                        const uint64_t adesc = p.mode == 3 ? sdesc(sa + k * 2048u, 512u, 64u)
+                                                           : sdesc(sa + k * 32u, 1u, 64u);
+                        const uint64_t bdesc = sdesc(sb + k * 32u, 1u, 64u);
+                        umma(d_tmem, adesc, bdesc, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+                    }
+                    ucommit(&empty[st]);
+                    issued = true;
+                    if (++st == kStages) { st = 0; ph ^= 1; }
+                }
+                if (!okm) break;
+                ucommit(&tfull[ab]);
+                if (++ab == 2) { ab = 0; aph ^= 1; }
+            }
+            // every MMA issued by this thread has completed before TMEM is released
+            if (issued) {
+                ucommit(done);
+                const unsigned long long t0 = now_ns();
+                while (!ub_try(done, 0) && now_ns() - t0 < kUWaitNs) {}
+            }
+        }
+    } else {
+        // ------------------------------------------------------------- epilogue (warps 2..5)
+        const int quad = warp & 3;               // TMEM lanes 32*quad .. 32*quad+31
+        const int lane_row = quad * 32 + lane;
+        const int et = threadIdx.x - 64;         // 0..127
+        volatile int no_abort = 0;
+        int ab = 0, aph = 0;
+        float v[64];
+        for (int u = blockIdx.x; u < units; u += gridDim.x) {
+            const int tile = u / q.splits, sp = u % q.splits;
+            const int kb0 = (int)((long long)sp * q.kblocks / q.splits);
+            const int kb1 = (int)((long long)(sp + 1) * q.kblocks / q.splits);
+            if (kb1 > kb0) {
+                // time bound only: all four epilogue warps leave this wait the same way
+                if (!ub_wait(&tfull[ab], aph, &no_abort, p.err)) break;
+                tc_fence_after();
+                const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(ab * N);
+#pragma unroll
+                for (int c0 = 0; c0 < 64; c0 += 16)
+                    if (c0 < N) tmem_ld16(taddr + c0, v + c0);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ub_arrive(&tempty[ab]);
+                if (++ab == 2) { ab = 0; aph ^= 1; }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) v[c] = 0.f;
+            }
+            if (q.splits == 1) {
+                finish_row<T>(p, q, tile, lane_row, v);
+                continue;
+            }
+            // split-K: publish this split's partial; the last CTA on the tile reduces in split order
+            float* mine = p.partial + ((size_t)u * kBM + lane_row) * N;
+            for (int c = 0; c < N; c += 4)
+                __stcg(reinterpret_cast<float4*>(mine + c), make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]));
+            __threadfence();
+            epi_sync();
+            if (et == 0) {
+                const uint32_t old = atomicAdd(&p.tickets[tile], 1u);
+                *s_last = old == (uint32_t)(q.splits - 1);
+            }
+            epi_sync();
+            if (*s_last) {
+                __threadfence();
+                for (int c = 0; c < N; ++c) v[c] = 0.f;
+                for (int s = 0; s < q.splits; ++s) {
+                    const float* src = p.partial + ((size_t)(tile * q.splits + s) * kBM + lane_row) * N;
+                    for (int c = 0; c < N; c += 4) {
+                        const float4 w = __ldcg(reinterpret_cast<const float4*>(src + c));
+                        v[c] += w.x; v[c + 1] += w.y; v[c + 2] += w.z; v[c + 3] += w.w;
+                    }
+                }
+                finish_row<T>(p, q, tile, lane_row, v);
+                if (et == 0) p.tickets[tile] = 0u;     // ready for the next call
+            }
+            epi_sync();
+        }
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host side: tensor maps through the driver entry point (no link-time libcuda dependency)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encoder() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    return fn;
+}
+
+// 2-D row-major [rows][cols] 16-bit tensor, box {64 columns, box_rows}, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, int dtype, int64_t rows, int64_t cols, int box_rows) {
+    EncodeTiledFn enc = encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = enc(m, dtype == SPFFN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                     const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int round16(int v) { return (v + 15) / 16 * 16; }
+
+size_t smem_bytes() { return (size_t)kStages * kStageBytes + 1024 + 256; }
+
+cudaError_t launch(const UParams& p, int grid, cudaStream_t st) {
+    const size_t smem = smem_bytes();
+    cudaError_t e;
+    if (p.dtype == SPFFN_BF16) {
+        e = cudaFuncSetAttribute(k_umma<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        k_umma<__nv_bfloat16><<<grid, kUThreads, smem, st>>>(p);
+    } else {
+        e = cudaFuncSetAttribute(k_umma<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        k_umma<__half><<<grid, kUThreads, smem, st>>>(p);
+    }
+    return cudaGetLastError();
+}
+
+UParams base_params(const spffn_ctx& c, int B) {
+    UParams p;
+    memset(&p, 0, sizeof(p));
+    p.B = B;
+    p.dtype = c.cfg.dtype;
+    p.n = c.cfg.n; p.d = c.cfg.d; p.H = c.cfg.H;
+    p.G = c.num_sms;
+    p.partial = c.upartial();
+    p.tickets = c.utickets();
+    p.err = &c.ctl()->err;
+    return p;
+}
+
+}  // namespace
+
+bool union_supported(const spffn_ctx& c, int B) {
+    return B >= 16 && B <= 32 && c.cfg.d % 128 == 0 && c.cfg.max_batch >= 16 && c.lay.upartial != 0 &&
+           c.num_sms <= kMaxUnionCtas && encoder() != nullptr;
+}
+
+cudaError_t union_predict(const spffn_ctx& c, const void* x, int B, int32_t* idx, int32_t* count, int32_t* count2,
+                          cudaStream_t st)
+{
+    const auto& g = c.cfg;
+    // predictor layer 1: D[H x B] = Wp1 . X^T, split-K, -> h (fp32) and its hi/lo pair
+    UParams p = base_params(c, B);
+    p.mode = 0;
+    p.N = round16(B);
+    p.M = g.H;
+    p.K = g.d;
+    const int tiles = (g.H + kBM - 1) / kBM;
+    const int kblocks = g.d / kBK;
+    p.splits_fixed = std::max(1, std::min(kblocks, c.num_sms / tiles));
+    p.bias = c.w.bp1;
+    p.out_split = c.hsplit();
+    p.out_f32 = c.h();
+    if (!make_map(&p.tmA, c.w.Wp1, g.dtype, g.H, g.d, kBM)) return cudaErrorInvalidValue;
+    if (!make_map(&p.tmB, x, g.dtype, B, g.d, p.N)) return cudaErrorInvalidValue;
+    cudaError_t e = launch(p, c.num_sms, st);
+    if (e != cudaSuccess) return e;
+    // predictor layer 2: D[n x 2B] = Wp2 . hsplit^T -> union mask words
+    UParams q = base_params(c, B);
+    q.mode = 1;
+    q.N = round16(2 * B);
+    q.M = g.n;
+    q.K = g.H;
+    q.bias = c.w.bp2;
+    q.mask = c.mask();
+    q.wcount = c.wcount();
+    if (!make_map(&q.tmA, c.w.Wp2, g.dtype, g.n, g.H, kBM)) return cudaErrorInvalidValue;
+    if (!make_map(&q.tmB, c.hsplit(), g.dtype, 2 * B, g.H, q.N)) return cudaErrorInvalidValue;
+    e = launch(q, c.num_sms, st);
+    if (e != cudaSuccess) return e;
+    return launch_compact(c, idx, count, count2, st);
+}
+
+cudaError_t union_forward(const spffn_ctx& c, const void* x, int B, const int32_t* idx, const int32_t* count,
+                          float* y, cudaStream_t st)
+{
+    const auto& g = c.cfg;
+    // FC1 over the table rows: D[U x B] = W1[table] . X^T -> a (hi/lo pair), zeros past U
+    UParams p = base_params(c, B);
+    p.mode = 2;
+    p.N = round16(B);
+    p.K = g.d;
+    p.count = count;
+    p.idx = idx;
+    p.bias = c.w.b1;
+    p.out_split = c.asplit();
+    if (!make_map(&p.tmA, c.w.W1, g.dtype, g.n, g.d, 1)) return cudaErrorInvalidValue;
+    if (!make_map(&p.tmB, x, g.dtype, B, g.d, p.N)) return cudaErrorInvalidValue;
+    cudaError_t e = launch(p, c.num_sms, st);
+    if (e != cudaSuccess) return e;
+    // FC2: D[d x 2B] = W2T[table]^T . asplit^T -> y
+    UParams q = base_params(c, B);
+    q.mode = 3;
+    q.N = round16(2 * B);
+    q.M = g.d;
+    q.count = count;
+    q.idx = idx;
+    q.bias = c.w.b2;
+    q.out_f32 = y;
+    if (!make_map(&q.tmA, c.w.W2T, g.dtype, g.n, g.d, 1)) return cudaErrorInvalidValue;
+    if (!make_map(&q.tmB, c.asplit(), g.dtype, 2 * B, g.n, q.N)) return cudaErrorInvalidValue;
+    return launch(q, c.num_sms, st);
+}
+
+}  // namespace spffn

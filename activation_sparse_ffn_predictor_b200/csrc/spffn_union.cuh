@@ -1,0 +1,12 @@
+// Union-mask tensor-core path (spffn_union.cu).
+#pragma once
+#include "spffn_internal.cuh"
+
+namespace spffn {
+bool union_supported(const spffn_ctx& c, int B);
+cudaError_t union_predict(const spffn_ctx& c, const void* x, int B, int32_t* idx, int32_t* count, int32_t* count2,
+                          cudaStream_t st);
+cudaError_t union_forward(const spffn_ctx& c, const void* x, int B, const int32_t* idx, const int32_t* count,
+                          float* y, cudaStream_t st);
+cudaError_t launch_compact(const spffn_ctx& c, int32_t* idx, int32_t* count, int32_t* count2, cudaStream_t st);
+}  // namespace spffn

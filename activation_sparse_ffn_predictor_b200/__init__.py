@@ -27,7 +27,7 @@ EXPORTS = ("spffn_workspace_bytes", "spffn_create", "spffn_destroy", "spffn_pred
            "spffn_step", "spffn_chain", "spffn_decode", "spffn_profile_counts", "spffn_reorder",
            "spffn_permute_rows", "spffn_permute_vector", "spffn_last_device_error", "spffn_status_string",
            "spffn_num_partials", "spffn_decode_kernel_launches", "spffn_set_trace", "spffn_trace_marks",
-           "spffn_last_cuda_error_string", "spffn_reorder_dealt")
+           "spffn_last_cuda_error_string", "spffn_reorder_dealt", "spffn_forward_noalloc")
 
 
 class SpffnError(RuntimeError):
@@ -75,6 +75,7 @@ def library(path: Optional[str] = None):
         "spffn_profile_counts": (st, [vp, vp, i32, vp, vp]),
         "spffn_reorder": (st, [vp, i32, vp]),
         "spffn_reorder_dealt": (st, [vp, i32, i32, vp]),
+        "spffn_forward_noalloc": (st, [ctypes.POINTER(Config), ctypes.POINTER(Weights), vp, i32, vp, vp, vp, vp]),
         "spffn_permute_rows": (st, [vp, vp, i32, i32, vp, vp]),
         "spffn_permute_vector": (st, [vp, vp, i32, vp, vp]),
         "spffn_last_device_error": (st, [vp, ctypes.POINTER(ctypes.c_uint32), vp]),
@@ -211,6 +212,13 @@ class Layer:
         code = ctypes.c_uint32(0)
         s = library().spffn_last_device_error(self.ctx, ctypes.byref(code), _stream(stream))
         return s, int(code.value)
+
+
+def forward_noalloc(layer: Layer, x, idx, count, y, stream=None):
+    """spffn_forward for `layer`'s weights without its context or workspace
+    (scratch in the library's fixed device array; see include/spffn.h)."""
+    _check(library().spffn_forward_noalloc(ctypes.byref(layer.cfg), ctypes.byref(layer.weights), _p(x), x.shape[0],
+                                           _p(idx), _p(count), _p(y), _stream(stream)), "spffn_forward_noalloc")
 
 
 def decode(layers: Sequence[Layer], x_in, x_out, y, counts=None, stream=None):

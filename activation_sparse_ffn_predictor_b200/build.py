@@ -8,7 +8,7 @@ CSRC = os.path.join(HERE, "csrc")
 SO = os.path.join(HERE, "libspffn.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
-SOURCES = ["spffn_api.cu", "spffn_kernels.cu", "spffn_fused.cu", "spffn_union.cu"]
+SOURCES = ["spffn_api.cu", "spffn_kernels.cu", "spffn_fused.cu", "spffn_union.cu", "spffn_noalloc.cu"]
 FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
          "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall", "--expt-relaxed-constexpr"]
 

@@ -386,6 +386,33 @@ static cudaError_t forward_impl(const spffn_ctx& c, const void* x, int B, const 
     return cudaGetLastError();
 }
 
+// Same two kernels as forward_impl, with caller-chosen scratch (S partial sums
+// of B x d fp32 at `partial`, error word at `err`).
+template <typename T>
+static cudaError_t forward_scratch_impl(const spffn_config& g, const spffn_weights& w, const void* x, int B,
+                                        const int32_t* idx, const int32_t* count, float* y, float* partial, int S,
+                                        uint32_t* err, cudaStream_t st)
+{
+    const int tg = max(1, min(8, (160 * 1024) / (g.d * (int)sizeof(float))));
+    const size_t smem = (size_t)tg * g.d * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(k_ffn_partial<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k_ffn_partial<T><<<S, 256, smem, st>>>((const T*)w.W1, (const T*)w.b1, (const T*)w.W2T, (const T*)x, B, g.d, g.n,
+                                           idx, count, tg, partial, err);
+    dim3 rg((g.d + 255) / 256, B);
+    k_ffn_reduce<T><<<rg, 256, 0, st>>>(partial, S, B, g.d, (const T*)w.b2, y);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_forward_scratch(const spffn_config& g, const spffn_weights& w, const void* x, int B,
+                                   const int32_t* idx, const int32_t* count, float* y, float* partial, int S,
+                                   uint32_t* err, cudaStream_t st)
+{
+    return g.dtype == SPFFN_BF16
+               ? forward_scratch_impl<__nv_bfloat16>(g, w, x, B, idx, count, y, partial, S, err, st)
+               : forward_scratch_impl<__half>(g, w, x, B, idx, count, y, partial, S, err, st);
+}
+
 template <typename T>
 static cudaError_t chain_impl(const spffn_ctx& c, const void* x, const float* y, int B, void* xn, cudaStream_t st)
 {

@@ -195,6 +195,29 @@ spffn_status spffn_permute_vector(const void* src, void* dst, int32_t count, con
 spffn_status spffn_set_trace(void* buf, size_t bytes);
 int32_t spffn_trace_marks(void);
 
+/* Allocation-free variant of spffn_forward (no counterpart on the pages; it
+ * exists for callers that cannot allocate device memory, e.g. code running in
+ * another allocator's arena or under a fixed device-memory budget, and so
+ * cannot provide an spffn_ctx workspace).  Computes exactly what spffn_forward
+ * computes for the layer described by `cfg`/`w` (same kernels, same
+ * deterministic split reduction; cfg->H and cfg->max_batch are not used) and
+ * needs no context: the fp32 partial sums live in a fixed 1 MiB __device__
+ * array that every GPU loading this library reserves until the process exits.
+ *   Limit: B * cfg->d * 4 bytes <= 1 MiB (e.g. B = 32 needs d <= 8192), else
+ *   SPFFN_ERR_UNSUPPORTED, checked on the host before anything is enqueued;
+ *   the number of partial sums is the largest count (<= the SM count) that
+ *   fits, so results agree with spffn_forward to rounding, not bitwise.
+ *   Set-up: the first call on a device looks up the array's device address
+ *   with that device current; make that first call before any stream capture.
+ *   Every call shares the array: calls that overlap on the GPU (different
+ *   streams, or different host threads without ordering) race and must not be
+ *   issued; calls on one stream are ordered and safe.
+ *   Device-side checks still clamp the count and skip out-of-range entries,
+ *   but this entry point does not report them.
+ *   Calls no cudaMalloc, cudaFree or allocating library routine. */
+spffn_status spffn_forward_noalloc(const spffn_config* cfg, const spffn_weights* w, const void* x, int32_t B,
+                                   const int32_t* idx, const int32_t* count, float* y, void* stream);
+
 /* Read and clear the context's device error word (synchronises `stream`).
  * Returns SPFFN_OK if clean, SPFFN_ERR_DEVICE_CHECK or SPFFN_ERR_TIMEOUT;
  * *code (may be NULL) receives the raw word. */

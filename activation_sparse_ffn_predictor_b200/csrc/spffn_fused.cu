@@ -126,12 +126,12 @@ struct Shared {
     float* hs;
     unsigned char* sel;
     int32_t* nl;
-    uint32_t* maskw;         // [n/32] copy of the layer's mask words
     float* bias1;            // [max_rows_h] bp1 for the CTA's Wp1 rows
     float* bias2;            // [max_rows]   bp2 for the CTA's Wp2 rows
     float* biasy;            // [max_cols]   b2 for the CTA's output columns
     float* red;              // [2][8][NB]
     float* red2;             // [8][NB]
+    float* red1;             // [32][8][NB] GEMV1 row partials per warp
     int32_t* scan;           // [kMaxG + 1]
     float* misc;             // [16]
 };
@@ -309,12 +309,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         S.hs = reinterpret_cast<float*>(q); q += ((size_t)NB * H * 4 + 127) / 128 * 128;
         S.sel = reinterpret_cast<unsigned char*>(q); q += (p.max_rows + 127) / 128 * 128;
         S.nl = reinterpret_cast<int32_t*>(q); q += ((size_t)p.max_rows * 4 + 127) / 128 * 128;
-        S.maskw = reinterpret_cast<uint32_t*>(q); q += ((size_t)(n >> 5) * 4 + 127) / 128 * 128;
         S.bias1 = reinterpret_cast<float*>(q); q += ((size_t)(H / G + 2) * 4 + 127) / 128 * 128;
         S.bias2 = reinterpret_cast<float*>(q); q += ((size_t)p.max_rows * 4 + 127) / 128 * 128;
         S.biasy = reinterpret_cast<float*>(q); q += ((size_t)(d / G + 8) * 4 + 127) / 128 * 128;
         S.red = reinterpret_cast<float*>(q); q += 2 * 8 * 2 * NB * 4;
         S.red2 = reinterpret_cast<float*>(q); q += 8 * NB * 4;
+        S.red1 = reinterpret_cast<float*>(q); q += 32 * 8 * NB * 4;
         S.scan = reinterpret_cast<int32_t*>(q); q += (kMaxG + 1) * 4;
         S.misc = reinterpret_cast<float*>(q); q += 16 * 4;
         q = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(q) + 15) & ~uintptr_t(15));
@@ -535,50 +535,76 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         }
         consumer_sync();
         TRACE(0);
-        // GEMV1 over Wp1 rows [a0, a1): mixed-precision dot of each row with x
-        for (int r = a0; r < a1 && ok; r += R1, ++pk_) {
-            const int s = pk_ % p.pred_slots;
-            if (!cwait(S, p, &S.pfull[s], (pk_ / p.pred_slots) & 1)) { ok = false; break; }
-            if (r == a0) TRACE(1); else TRACE(13);
-            const uint4* slot = reinterpret_cast<const uint4*>(S.pring + (size_t)s * p.pred_slot_bytes);
-            const int rows = min(R1, a1 - r);
-            const int Q = R1 >= kConsumerWarps ? 1 : kConsumerWarps / R1;
-            const int rw = warp / Q, seg = warp % Q;
-            const int vlo = split_lo(nvec, Q, seg), vhi = split_lo(nvec, Q, seg + 1);
-            for (int rr = rw; rr < rows; rr += kConsumerWarps / Q) {
-                const uint4* wrow = slot + (size_t)rr * nvec;
-                float acc[NB][4];
+        // GEMV1 over Wp1 rows [a0, a1).  Warp w owns columns [w nvec/8, (w+1) nvec/8) of every
+        // row; its lanes keep that segment of x in registers as fp32 pairs, and the eight
+        // warps' partial dots of a row are added in fixed order through shared memory.
+        {
+            const int seg_lo = split_lo(nvec, kConsumerWarps, warp), seg_hi = split_lo(nvec, kConsumerWarps, warp + 1);
+            u64 xg[kMaxVPT][4][NB];
 #pragma unroll
-                for (int t = 0; t < NB; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-#pragma unroll 4
-                for (int v = vlo + lane; v < vhi; v += 32) {
-                    const uint4 w = wrow[v];
+            for (int m = 0; m < kMaxVPT; ++m) {
+                const int v = seg_lo + lane + 32 * m;
 #pragma unroll
-                    for (int t = 0; t < NB; ++t)
-                        dot_mix<T>(acc[t], w, reinterpret_cast<const uint4*>(xs + (size_t)t * d)[v]);
-                }
-                float z[NB];
-#pragma unroll
-                for (int t = 0; t < NB; ++t) z[t] = warp_sum(sum4(acc[t]));
-                if (Q == 1) {
-                    if (lane == 0) {
-                        const float bias = S.bias1[r + rr - a0];
-                        for (int t = 0; t < B; ++t) p.h[(size_t)t * H + r + rr] = fmaxf(z[t] + bias, 0.f);
+                for (int t = 0; t < NB; ++t) {
+                    if (v < seg_hi) {
+                        const uint4 xv = reinterpret_cast<const uint4*>(xs + (size_t)t * d)[v];
+                        xg[m][0][t] = Arith<T>::widen2(xv.x); xg[m][1][t] = Arith<T>::widen2(xv.y);
+                        xg[m][2][t] = Arith<T>::widen2(xv.z); xg[m][3][t] = Arith<T>::widen2(xv.w);
+                    } else {
+                        xg[m][0][t] = xg[m][1][t] = xg[m][2][t] = xg[m][3][t] = 0ull;
                     }
-                } else if (lane == 0) {
-#pragma unroll
-                    for (int t = 0; t < NB; ++t) S.red2[warp * NB + t] = z[t];
                 }
             }
-            if (r == a0) TRACE(12); else TRACE(14);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S.pempty[s]);
-            if (Q > 1) {
+            for (int r = a0; r < a1 && ok; r += R1, ++pk_) {
+                const int s = pk_ % p.pred_slots;
+                if (!cwait(S, p, &S.pfull[s], (pk_ / p.pred_slots) & 1)) { ok = false; break; }
+                if (r == a0) TRACE(1); else TRACE(13);
+                const uint4* slot = reinterpret_cast<const uint4*>(S.pring + (size_t)s * p.pred_slot_bytes);
+                const int rows = min(R1, a1 - r);
+                for (int rr = 0; rr < rows; rr += 2) {
+                    const bool two = rr + 1 < rows;
+                    const uint4* w0p = slot + (size_t)rr * nvec;
+                    const uint4* w1p = slot + (size_t)(two ? rr + 1 : rr) * nvec;
+                    u64 c0[NB], c1[NB];
+#pragma unroll
+                    for (int t = 0; t < NB; ++t) c0[t] = c1[t] = 0ull;
+#pragma unroll
+                    for (int m = 0; m < kMaxVPT; ++m) {
+                        const int v = seg_lo + lane + 32 * m;
+                        if (v < seg_hi) {
+                            const uint4 w0 = w0p[v], w1 = w1p[v];
+                            const u64 p00 = Arith<T>::widen2(w0.x), p01 = Arith<T>::widen2(w0.y);
+                            const u64 p02 = Arith<T>::widen2(w0.z), p03 = Arith<T>::widen2(w0.w);
+                            const u64 p10 = Arith<T>::widen2(w1.x), p11 = Arith<T>::widen2(w1.y);
+                            const u64 p12 = Arith<T>::widen2(w1.z), p13 = Arith<T>::widen2(w1.w);
+#pragma unroll
+                            for (int t = 0; t < NB; ++t) {
+                                ffma2(c0[t], p00, xg[m][0][t]); ffma2(c0[t], p01, xg[m][1][t]);
+                                ffma2(c0[t], p02, xg[m][2][t]); ffma2(c0[t], p03, xg[m][3][t]);
+                                ffma2(c1[t], p10, xg[m][0][t]); ffma2(c1[t], p11, xg[m][1][t]);
+                                ffma2(c1[t], p12, xg[m][2][t]); ffma2(c1[t], p13, xg[m][3][t]);
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int t = 0; t < NB; ++t) {
+                        const float2 e0 = upk(c0[t]), e1 = upk(c1[t]);
+                        const float z0 = warp_sum(e0.x + e0.y), z1 = warp_sum(e1.x + e1.y);
+                        if (lane == 0) {
+                            S.red1[(rr * kConsumerWarps + warp) * NB + t] = z0;
+                            if (two) S.red1[((rr + 1) * kConsumerWarps + warp) * NB + t] = z1;
+                        }
+                    }
+                }
+                if (r == a0) TRACE(12); else TRACE(14);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.pempty[s]);
                 consumer_sync();
                 if (tid < rows * NB) {
                     const int rr = tid / NB, t = tid % NB;
                     float zz = 0.f;
-                    for (int q = 0; q < Q; ++q) zz += S.red2[(rr * Q + q) * NB + t];
+#pragma unroll
+                    for (int q = 0; q < kConsumerWarps; ++q) zz += S.red1[(rr * kConsumerWarps + q) * NB + t];
                     if (t < B) p.h[(size_t)t * H + r + rr] = fmaxf(zz + S.bias1[r + rr - a0], 0.f);
                 }
                 consumer_sync();
@@ -934,11 +960,10 @@ Geometry geometry(const spffn_config& c, int G) {
     fixed += ((size_t)NB * c.H * 4 + 127) / 128 * 128;              // hs
     fixed += (g.max_rows + 127) / 128 * 128;                         // sel
     fixed += ((size_t)g.max_rows * 4 + 127) / 128 * 128;             // nl
-    fixed += ((size_t)(c.n / 32) * 4 + 127) / 128 * 128;             // maskw
     fixed += ((size_t)(c.H / G + 2) * 4 + 127) / 128 * 128;          // bias1
     fixed += ((size_t)g.max_rows * 4 + 127) / 128 * 128;             // bias2
     fixed += ((size_t)(c.d / G + 8) * 4 + 127) / 128 * 128;          // biasy
-    fixed += 2 * 8 * 2 * NB * 4 + 8 * NB * 4 + (kMaxG + 1) * 4 + 16 * 4 + 16;
+    fixed += 2 * 8 * 2 * NB * 4 + 8 * NB * 4 + 32 * 8 * NB * 4 + (kMaxG + 1) * 4 + 16 * 4 + 16;
     fixed += 8 * (2 * 8 + 2 * 8 + 1) + 8 * 8 + 128;                  // barriers + flags + slack
     const size_t fslot = 4 * (size_t)c.d + 128;
     g.pred_slots = 4;

@@ -256,30 +256,52 @@ __global__ void __launch_bounds__(256) k_ffn_reduce(const float* __restrict__ pa
 }
 
 // ---------------------------------------------------------------------------
-// S9  chaining: x_next = round((x + y) / sqrt(mean((x + y)^2) + eps)), one block per token.
+// S9  chaining: x_next = round((x + y) / sqrt(mean((x + y)^2) + eps)), one block
+// of 1024 threads per token; each thread keeps its 8-column vectors of u in
+// registers between the sum of squares and the write (fixed reduction tree).
 template <typename T>
-__global__ void __launch_bounds__(256) k_chain(const T* __restrict__ x, const float* __restrict__ y, int d,
-                                               T* __restrict__ xn)
+__global__ void __launch_bounds__(1024) k_chain(const T* __restrict__ x, const float* __restrict__ y, int d,
+                                                T* __restrict__ xn)
 {
-    __shared__ float ws[8];
+    constexpr int kV = 2;                         // 8-column vectors per thread (d <= 16384)
+    __shared__ float ws[32];
     const int t = blockIdx.x, tid = threadIdx.x;
-    const T* xr = x + (size_t)t * d;
-    const float* yr = y + (size_t)t * d;
+    const int nv = d >> 3;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+    const float4* yr = reinterpret_cast<const float4*>(y + (size_t)t * d);
+    float u[kV][8];
     float ss = 0.f;
-    for (int c = tid; c < d; c += blockDim.x) {
-        float u = DT<T>::f(xr[c]) + yr[c];
-        ss = fmaf(u, u, ss);
+#pragma unroll
+    for (int m = 0; m < kV; ++m) {
+        const int v = tid + m * 1024;
+        if (v < nv) {
+            float xv[8];
+            unpack8<T>(xr[v], xv);
+            const float4 a = yr[2 * v], b = yr[2 * v + 1];
+            const float yv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                u[m][q] = xv[q] + yv[q];
+                ss = fmaf(u[m][q], u[m][q], ss);
+            }
+        }
     }
     ss = warp_sum(ss);
     if ((tid & 31) == 0) ws[tid >> 5] = ss;
     __syncthreads();
     float tot = 0.f;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) tot += ws[q];
+    for (int q = 0; q < 32; ++q) tot += ws[q];
     const float rs = 1.0f / sqrtf(tot / (float)d + 1e-6f);
-    for (int c = tid; c < d; c += blockDim.x) {
-        float u = DT<T>::f(xr[c]) + yr[c];
-        xn[(size_t)t * d + c] = DT<T>::r(u * rs);
+#pragma unroll
+    for (int m = 0; m < kV; ++m) {
+        const int v = tid + m * 1024;
+        if (v < nv) {
+            T o[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) o[q] = DT<T>::r(u[m][q] * rs);
+            reinterpret_cast<uint4*>(xn + (size_t)t * d)[v] = *reinterpret_cast<const uint4*>(o);
+        }
     }
 }
 
@@ -416,7 +438,7 @@ cudaError_t launch_forward_scratch(const spffn_config& g, const spffn_weights& w
 template <typename T>
 static cudaError_t chain_impl(const spffn_ctx& c, const void* x, const float* y, int B, void* xn, cudaStream_t st)
 {
-    k_chain<T><<<B, 256, 0, st>>>((const T*)x, y, c.cfg.d, (T*)xn);
+    k_chain<T><<<B, 1024, 0, st>>>((const T*)x, y, c.cfg.d, (T*)xn);
     return cudaGetLastError();
 }
 

@@ -279,7 +279,20 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
                     jr[i] = p.idx[r < q.M ? r : 0];
                 }
             }
+            // mode 3: this lane's 4 table rows of the K block, one block ahead
+            auto k_rows = [&](int kb, int* j) {
+                const int g = lane & 15;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = kb * kBK + g * 4 + i;
+                    j[i] = p.idx[r < q.K ? r : 0];
+                }
+            };
+            int jn[4] = {0, 0, 0, 0};
+            if (p.mode == 3 && kb0 < kb1) k_rows(kb0, jn);
             for (int kb = kb0; kb < kb1; ++kb) {
+                int jc[4] = {jn[0], jn[1], jn[2], jn[3]};
+                if (p.mode == 3 && kb + 1 < kb1) k_rows(kb + 1, jn);
                 bool okw = true;
                 if (lane == 0) okw = ub_wait(&empty[st], ph ^ 1, abort_flag, p.err);
                 okw = __shfl_sync(0xffffffffu, okw, 0);
@@ -296,13 +309,7 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
                 } else {
                     // 64 table rows (the K block) x 128 columns of W2T, as two 64-column blocks
                     const int mb = lane >> 4, g = lane & 15;
-                    int j[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int r = kb * kBK + g * 4 + i;
-                        j[i] = p.idx[r < q.K ? r : 0];
-                    }
-                    tma_gather4(sa + mb * 8192 + g * 512, &p.tmA, tile * kBM + mb * 64, j[0], j[1], j[2], j[3],
+                    tma_gather4(sa + mb * 8192 + g * 512, &p.tmA, tile * kBM + mb * 64, jc[0], jc[1], jc[2], jc[3],
                                 &full[st]);
                 }
                 if (lane == 0) tma_2d(sb, &p.tmB, kb * kBK, 0, &full[st]);
@@ -392,8 +399,10 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
             }
             // split-K: publish this split's partial; the last CTA on the tile reduces in split order
             float* mine = p.partial + ((size_t)u * kBM + lane_row) * N;
-            for (int c = 0; c < N; c += 4)
-                __stcg(reinterpret_cast<float4*>(mine + c), make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]));
+#pragma unroll
+            for (int c = 0; c < 64; c += 4)
+                if (c < N)
+                    __stcg(reinterpret_cast<float4*>(mine + c), make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]));
             __threadfence();
             epi_sync();
             if (et == 0) {
@@ -403,12 +412,20 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
             epi_sync();
             if (*s_last) {
                 __threadfence();
-                for (int c = 0; c < N; ++c) v[c] = 0.f;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) v[c] = 0.f;
+                // one split at a time, its (up to 16) float4 loads issued together
                 for (int s = 0; s < q.splits; ++s) {
-                    const float* src = p.partial + ((size_t)(tile * q.splits + s) * kBM + lane_row) * N;
-                    for (int c = 0; c < N; c += 4) {
-                        const float4 w = __ldcg(reinterpret_cast<const float4*>(src + c));
-                        v[c] += w.x; v[c + 1] += w.y; v[c + 2] += w.z; v[c + 3] += w.w;
+                    const float4* src = reinterpret_cast<const float4*>(
+                        p.partial + ((size_t)(tile * q.splits + s) * kBM + lane_row) * N);
+                    float4 w[16];
+#pragma unroll
+                    for (int c4 = 0; c4 < 16; ++c4)
+                        w[c4] = c4 * 4 < N ? __ldcg(src + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int c4 = 0; c4 < 16; ++c4) {
+                        v[4 * c4] += w[c4].x; v[4 * c4 + 1] += w[c4].y;
+                        v[4 * c4 + 2] += w[c4].z; v[4 * c4 + 3] += w[c4].w;
                     }
                 }
                 finish_row<T>(p, q, tile, lane_row, v);

@@ -27,7 +27,11 @@ Readings where the pages leave a step open (all pinned by tests unless noted):
 * the neuron table is ascending in physical (stored-row) order;
 * an empty set gives ``y = b2``;
 * the layer chaining used by multi-layer runs is
-  ``x' = round_dtype((x + y) / sqrt(mean((x + y)^2) + eps))`` with eps = 1e-6.
+  ``x' = round_dtype((x + y) / sqrt(mean((x + y)^2) + eps))`` with eps = 1e-6;
+* under look-ahead prediction the set of layer l+1 comes from layer l+1's own
+  predictor applied to layer l's input (equation (-2) writes the predictor with
+  the earlier layer's index, but its outputs are layer l+1's neurons), and the
+  first layer, having no earlier input, predicts from its own.
 
 Parity of the predictor's *quality* (recall against the true active set) is
 unpinned: with random weights there is nothing to claim, and no function here
@@ -152,6 +156,17 @@ def step(layer, x):
     neuron-aware FFN over the table ([PI1] DejaVu equation (-1): S_M from the
     predictor on the FFN input, then the MLP restricted to S_M)."""
     idx, k, logits = predict(layer["Wp1"], layer["Wp2"], layer["bp2"], x, layer.get("bp1"))
+    y = sparse_ffn(layer["W1"], layer["b1"], layer["W2T"], layer.get("b2"), x, idx)
+    return idx, k, logits, y
+
+
+def step_lookahead(layer, x_pred, x):
+    """One layer under look-ahead prediction ([PI1] DejaVu appendix, equation (-2)
+    and the closing list on DejaVu's speed: the sparsity of layer l+1 is predicted
+    from layer l's input while layer l computes).  The layer's own predictor is
+    applied to ``x_pred`` (the previous layer's input; the layer's own input for
+    the first layer) and the FFN runs on ``x`` restricted to that set."""
+    idx, k, logits = predict(layer["Wp1"], layer["Wp2"], layer["bp2"], x_pred, layer.get("bp1"))
     y = sparse_ffn(layer["W1"], layer["b1"], layer["W2T"], layer.get("b2"), x, idx)
     return idx, k, logits, y
 

@@ -242,3 +242,48 @@ def test_dealt_order_hand_example():
     # 3 ranges over 7 slots: [0,2) [2,4) [4,7); deal 4->r0, 1->r1, 6->r2, 0->r0, 3->r1, 2->r2, 5->r2
     assert O.dealt_order(counts, 3).tolist() == [4, 0, 1, 3, 6, 2, 5]
     assert O.dealt_order(counts, 1).tolist() == O.hot_first_order(counts).tolist()
+
+
+# ---------------------------------------------------------------------------
+# look-ahead prediction
+def _hand_lookahead_layer():
+    # identity predictor (h = ReLU(x), logit_i = h_i): neuron i is predicted iff x_i > 0;
+    # FC1 = identity (a_j = ReLU(x_j)); FC2 rows e1*3 and e0*5: y = [5 a_1, 3 a_0]
+    return dict(W1=np.eye(2), b1=np.zeros(2), W2T=np.array([[0.0, 3.0], [5.0, 0.0]]), b2=np.zeros(2),
+                Wp1=np.eye(2), bp1=np.zeros(2), Wp2=np.eye(2), bp2=np.zeros(2))
+
+
+def test_lookahead_hand_example():
+    L = _hand_lookahead_layer()
+    x0 = np.array([1.0, -1.0])
+    # layer 0: both readings predict from x0 -> {0}; y0 = [0, 3]
+    idx0, k0, _, y0 = O.step_lookahead(L, x0, x0)
+    assert idx0.tolist() == [0] and k0 == 1
+    np.testing.assert_array_equal(y0[0], [0.0, 3.0])
+    x1 = O.chain(x0, y0)[0]
+    s = math.sqrt(2.5 + O.RMS_EPS)
+    np.testing.assert_allclose(x1, [1.0 / s, 2.0 / s], rtol=1e-15)
+    # layer 1 on x1: its own input fires both neurons, the previous input only neuron 0
+    idx_s, k_s, _, y_s = O.step(L, x1)
+    idx_l, k_l, _, y_l = O.step_lookahead(L, x0, x1)
+    assert idx_s.tolist() == [0, 1] and idx_l.tolist() == [0]
+    np.testing.assert_allclose(y_s[0], [10.0 / s, 3.0 / s], rtol=1e-15)
+    np.testing.assert_allclose(y_l[0], [0.0, 3.0 / s], rtol=1e-15)
+
+
+def test_lookahead_set_depends_only_on_predictor_input():
+    L = _tiny_layer(31)
+    r = _rng(32)
+    xp, x, x2 = r.standard_normal(8), r.standard_normal(8), r.standard_normal(8)
+    idx_a, _, log_a, y_a = O.step_lookahead(L, xp, x)
+    idx_b, _, log_b, y_b = O.step_lookahead(L, xp, x2)
+    assert idx_a.tolist() == idx_b.tolist()
+    np.testing.assert_array_equal(log_a, log_b)
+    # the FFN part is the sparse FFN of the FFN input over that set
+    np.testing.assert_array_equal(y_b, O.sparse_ffn(L["W1"], L["b1"], L["W2T"], L["b2"], x2, idx_a))
+    # same input on both sides: the plain step, bit for bit
+    i0, k0, l0, y0 = O.step(L, x)
+    i1, k1, l1, y1 = O.step_lookahead(L, x, x)
+    assert i0.tolist() == i1.tolist() and k0 == k1
+    np.testing.assert_array_equal(l0, l1)
+    np.testing.assert_array_equal(y0, y1)

@@ -27,7 +27,8 @@ EXPORTS = ("spffn_workspace_bytes", "spffn_create", "spffn_destroy", "spffn_pred
            "spffn_step", "spffn_chain", "spffn_decode", "spffn_profile_counts", "spffn_reorder",
            "spffn_permute_rows", "spffn_permute_vector", "spffn_last_device_error", "spffn_status_string",
            "spffn_num_partials", "spffn_decode_kernel_launches", "spffn_set_trace", "spffn_trace_marks",
-           "spffn_last_cuda_error_string", "spffn_reorder_dealt", "spffn_forward_noalloc")
+           "spffn_last_cuda_error_string", "spffn_reorder_dealt", "spffn_forward_noalloc",
+           "spffn_decode_lookahead", "spffn_layer_table")
 
 
 class SpffnError(RuntimeError):
@@ -72,6 +73,8 @@ def library(path: Optional[str] = None):
         "spffn_step": (st, [vp, vp, i32, vp, vp, vp, vp]),
         "spffn_chain": (st, [vp, vp, vp, i32, vp, vp]),
         "spffn_decode": (st, [ctypes.POINTER(vp), i32, vp, i32, vp, vp, vp, vp]),
+        "spffn_decode_lookahead": (st, [ctypes.POINTER(vp), i32, vp, i32, vp, vp, vp, vp]),
+        "spffn_layer_table": (st, [vp, ctypes.POINTER(vp)]),
         "spffn_profile_counts": (st, [vp, vp, i32, vp, vp]),
         "spffn_reorder": (st, [vp, i32, vp]),
         "spffn_reorder_dealt": (st, [vp, i32, i32, vp]),
@@ -208,6 +211,15 @@ class Layer:
         _check(library().spffn_profile_counts(self.ctx, _p(X), X.shape[0], _p(counts), _stream(stream)),
                "spffn_profile_counts")
 
+    def table(self, count: int):
+        """The neuron table the last decode left in this layer's workspace: an
+        int32 view of its first ``count`` entries (spffn_layer_table)."""
+        import torch
+        ptr = ctypes.c_void_p()
+        _check(library().spffn_layer_table(self.ctx, ctypes.byref(ptr)), "spffn_layer_table")
+        off = int(ptr.value) - self.workspace.data_ptr()
+        return self.workspace[off:off + 4 * int(count)].view(torch.int32)
+
     def last_device_error(self, stream=None):
         code = ctypes.c_uint32(0)
         s = library().spffn_last_device_error(self.ctx, ctypes.byref(code), _stream(stream))
@@ -221,10 +233,13 @@ def forward_noalloc(layer: Layer, x, idx, count, y, stream=None):
                                            _p(idx), _p(count), _p(y), _stream(stream)), "spffn_forward_noalloc")
 
 
-def decode(layers: Sequence[Layer], x_in, x_out, y, counts=None, stream=None):
+def decode(layers: Sequence[Layer], x_in, x_out, y, counts=None, stream=None, lookahead: bool = False):
+    """One decode step through the stack (spffn_decode; with ``lookahead`` the
+    set of layer l+1 is predicted from x_l, spffn_decode_lookahead)."""
     arr = (ctypes.c_void_p * len(layers))(*[l.ctx.value for l in layers])
-    _check(library().spffn_decode(arr, len(layers), _p(x_in), x_in.shape[0], _p(x_out), _p(y), _p(counts),
-                                  _stream(stream)), "spffn_decode")
+    fn = library().spffn_decode_lookahead if lookahead else library().spffn_decode
+    _check(fn(arr, len(layers), _p(x_in), x_in.shape[0], _p(x_out), _p(y), _p(counts), _stream(stream)),
+           "spffn_decode_lookahead" if lookahead else "spffn_decode")
 
 
 def decode_kernel_launches(layers: Sequence[Layer], B: int) -> int:

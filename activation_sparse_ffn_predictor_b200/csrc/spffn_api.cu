@@ -131,8 +131,10 @@ spffn_status spffn_chain(spffn_ctx* ctx, const void* x, const float* y, int32_t 
     return cuda_status(launch_chain(*ctx, x, y, B, x_next, (cudaStream_t)stream));
 }
 
-spffn_status spffn_decode(spffn_ctx* const* layers, int32_t L, const void* x_in, int32_t B, void* x_out,
-                          float* y, int32_t* counts, void* stream) {
+namespace {
+
+spffn_status decode_impl(spffn_ctx* const* layers, int32_t L, const void* x_in, int32_t B, void* x_out, float* y,
+                         int32_t* counts, bool lookahead, void* stream) {
     if (!layers || L < 1 || !x_in || !x_out || !y) return SPFFN_ERR_INVALID_ARG;
     const spffn_ctx* l0 = layers[0];
     if (!l0) return SPFFN_ERR_INVALID_ARG;
@@ -144,11 +146,23 @@ spffn_status spffn_decode(spffn_ctx* const* layers, int32_t L, const void* x_in,
     if (!aligned16(x_in) || !aligned16(x_out) || !aligned16(y) || x_in == x_out) return SPFFN_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     if (fused_decode_supported(layers, L, B))
-        return cuda_status(launch_fused_decode(layers, L, x_in, B, x_out, y, counts, st));
+        return cuda_status(launch_fused_decode(layers, L, x_in, B, x_out, y, counts, lookahead, st));
     const void* xcur = x_in;
+    cudaError_t e = cudaSuccess;
+    if (lookahead) {
+        const spffn_ctx& c = *layers[0];
+        e = launch_predict(c, x_in, B, c.idx(), c.count(), counts, st);
+        if (e != cudaSuccess) return cuda_status(e);
+    }
     for (int l = 0; l < L; ++l) {
         const spffn_ctx& c = *layers[l];
-        cudaError_t e = launch_predict(c, xcur, B, c.idx(), c.count(), counts ? counts + l : nullptr, st);
+        if (!lookahead) {
+            e = launch_predict(c, xcur, B, c.idx(), c.count(), counts ? counts + l : nullptr, st);
+        } else if (l + 1 < L) {
+            // the next layer's set from this layer's input
+            const spffn_ctx& cn = *layers[l + 1];
+            e = launch_predict(cn, xcur, B, cn.idx(), cn.count(), counts ? counts + l + 1 : nullptr, st);
+        }
         if (e != cudaSuccess) return cuda_status(e);
         float* yl = (l == L - 1) ? y : c.ybuf();
         e = launch_forward(c, xcur, B, c.idx(), c.count(), yl, st);
@@ -158,6 +172,24 @@ spffn_status spffn_decode(spffn_ctx* const* layers, int32_t L, const void* x_in,
         if (e != cudaSuccess) return cuda_status(e);
         xcur = xn;
     }
+    return SPFFN_OK;
+}
+
+}  // namespace
+
+spffn_status spffn_decode(spffn_ctx* const* layers, int32_t L, const void* x_in, int32_t B, void* x_out,
+                          float* y, int32_t* counts, void* stream) {
+    return decode_impl(layers, L, x_in, B, x_out, y, counts, false, stream);
+}
+
+spffn_status spffn_decode_lookahead(spffn_ctx* const* layers, int32_t L, const void* x_in, int32_t B,
+                                    void* x_out, float* y, int32_t* counts, void* stream) {
+    return decode_impl(layers, L, x_in, B, x_out, y, counts, true, stream);
+}
+
+spffn_status spffn_layer_table(spffn_ctx* ctx, const int32_t** idx) {
+    if (!ctx || !idx) return SPFFN_ERR_INVALID_ARG;
+    *idx = ctx->idx();
     return SPFFN_OK;
 }
 

@@ -1,17 +1,21 @@
 // Persistent whole-stack decode kernel for small batches (B <= 2).
 //
-// One CTA per SM runs every layer of the stack in a single launch.  Per layer,
-// four phases separated by grid barriers:
-//   A  h = ReLU(Wp1 x + bp1)          Wp1 rows split across CTAs
-//   B  logits, threshold, mask bits    Wp2 rows split across CTAs (atomicOr into
-//                                      the mask words, per-CTA counts)
-//   C  neuron table + FFN              every CTA takes an equal slice of the
-//                                      ascending table, gathers W1/W2T rows,
-//                                      FC1 (vec_dot) + ReLU, FC2 (AXPY) into a
-//                                      fixed per-CTA fp32 partial
-//   D  y = b2 + sum of partials (fixed order), u = x + y, per-CTA sum of squares
-// and the next layer's input x = round(u / rms(u)) is formed at the start of
-// its phase A.
+// One CTA per SM runs every layer of the stack in a single launch.  CTA c owns
+// a contiguous span of Wp1 rows (predictor hidden units), a contiguous span of
+// Wp2 rows (FFN neurons, placed hot-first and dealt over the spans offline) and
+// a slice of the output columns.  Per layer l:
+//   A  x_l from the previous layer's u; h = ReLU(Wp1 x + bp1) on own Wp1 rows
+//      -- grid barrier --
+//   B  logits of own neurons, threshold (union over the batch) and the CTA's
+//      ascending list of selected neurons; the FFN of exactly those neurons:
+//      FC1 vec_dot + bias + ReLU, FC2 AXPY into a per-CTA fp32 partial
+//      -- grid barrier --
+//   D  y = b2 + the G partials in fixed order on own columns, u = x + y; the
+//      neuron table (each CTA's list at its prefix position) and its count
+//      -- grid barrier --
+// With look-ahead prediction (DejaVu's asynchronous predictor) the set of layer
+// l+1 is predicted from x_l: h_{l+1} and FFN_l share one phase, logits_{l+1}
+// and the reduction of y_l the next, so a layer has two grid barriers.
 //
 // Weight bytes move with cp.async.bulk (TMA bulk copies) into shared-memory
 // rings guarded by mbarriers.  The predictor weights do not depend on the
@@ -52,12 +56,10 @@ struct Params {
     uint32_t* bar;        // grid-barrier counter
     uint32_t* err;
     uint32_t* abort;
-    uint32_t* mask;       // [2][n/32]
-    int32_t* cta_count;   // [G]
+    int32_t* cta_count;   // [2][G + 1] list lengths per CTA, by list parity
     float* h;             // [B][H]
     float* partial;       // [G][B][d]
     float* u;             // [B][d]
-    float* ss;            // [G][B]
     int pred_slots, pred_slot_bytes, ffn_slots, R1, R2, max_rows;
     unsigned long long* trace;   // optional [G][L][kTraceMarks] globaltimer stamps
     LayerW layer[kMaxFusedLayers];
@@ -118,21 +120,20 @@ struct Shared {
     uint64_t* pempty;
     uint64_t* ffull;
     uint64_t* fempty;
-    uint64_t* fready;
-    volatile int* flags;     // [0] local abort, [1] ffn_m, [2] pred issued, [3] ffn issued, [4] pred done, [5] ffn done
+    volatile int* flags;     // [0] local abort, [1] list tag|length, [2] pred issued, [3] ffn issued,
+                             // [4] pred done, [5] ffn done, [7] last final list + 1
     char* pring;
     char* fring;
     void* xs;
     float* hs;
     unsigned char* sel;
-    int32_t* nl;
+    int32_t* nl;             // [2][max_rows] neuron lists, by list parity
     float* bias1;            // [max_rows_h] bp1 for the CTA's Wp1 rows
     float* bias2;            // [max_rows]   bp2 for the CTA's Wp2 rows
     float* biasy;            // [max_cols]   b2 for the CTA's output columns
-    float* red;              // [2][8][NB]
+    float* red;              // [2][8][2][NB] FC1 partial dots of a neuron pair, by pair parity
     float* red2;             // [8][NB]
     float* red1;             // [32][8][NB] GEMV1 row partials per warp
-    int32_t* scan;           // [kMaxG + 1]
     float* misc;             // [16]
 };
 
@@ -289,7 +290,7 @@ __device__ __forceinline__ bool cwait(const Shared& S, const Params& p, uint64_t
     } while (0)
 
 // ---------------------------------------------------------------------------
-template <typename T, int NB, int HV>
+template <typename T, int NB, int HV, bool LA>
 __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ Params p)
 {
     extern __shared__ __align__(128) char smem[];
@@ -308,26 +309,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         S.xs = q; q += ((size_t)NB * d * sizeof(T) + 127) / 128 * 128;
         S.hs = reinterpret_cast<float*>(q); q += ((size_t)NB * H * 4 + 127) / 128 * 128;
         S.sel = reinterpret_cast<unsigned char*>(q); q += (p.max_rows + 127) / 128 * 128;
-        S.nl = reinterpret_cast<int32_t*>(q); q += ((size_t)p.max_rows * 4 + 127) / 128 * 128;
+        S.nl = reinterpret_cast<int32_t*>(q); q += ((size_t)2 * p.max_rows * 4 + 127) / 128 * 128;
         S.bias1 = reinterpret_cast<float*>(q); q += ((size_t)(H / G + 2) * 4 + 127) / 128 * 128;
         S.bias2 = reinterpret_cast<float*>(q); q += ((size_t)p.max_rows * 4 + 127) / 128 * 128;
         S.biasy = reinterpret_cast<float*>(q); q += ((size_t)(d / G + 8) * 4 + 127) / 128 * 128;
         S.red = reinterpret_cast<float*>(q); q += 2 * 8 * 2 * NB * 4;
         S.red2 = reinterpret_cast<float*>(q); q += 8 * NB * 4;
         S.red1 = reinterpret_cast<float*>(q); q += 32 * 8 * NB * 4;
-        S.scan = reinterpret_cast<int32_t*>(q); q += (kMaxG + 1) * 4;
         S.misc = reinterpret_cast<float*>(q); q += 16 * 4;
         q = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(q) + 15) & ~uintptr_t(15));
         uint64_t* bars = reinterpret_cast<uint64_t*>(q);
         S.pfull = bars; S.pempty = bars + p.pred_slots;
         S.ffull = S.pempty + p.pred_slots; S.fempty = S.ffull + p.ffn_slots;
-        S.fready = S.fempty + p.ffn_slots;
-        S.flags = reinterpret_cast<volatile int*>(S.fready + 1);
+        S.flags = reinterpret_cast<volatile int*>(S.fempty + p.ffn_slots);
     }
     if (tid == 0) {
         for (int i = 0; i < p.pred_slots; ++i) { mbar_init(&S.pfull[i], 1); mbar_init(&S.pempty[i], kConsumerWarps); }
         for (int i = 0; i < p.ffn_slots; ++i) { mbar_init(&S.ffull[i], 1); mbar_init(&S.fempty[i], kConsumerWarps); }
-        mbar_init(S.fready, 1);
         for (int i = 0; i < 8; ++i) S.flags[i] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -397,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
                         __threadfence_block();
                         const int s = k % p.ffn_slots;
                         if (!wait_bounded(S, p, &S.fempty[s], ((k / p.ffn_slots) & 1) ^ 1, true)) { stop = true; break; }
-                        const int j = S.nl[issued];
+                        const int j = S.nl[(l & 1) * p.max_rows + issued];
                         char* dst = S.fring + (size_t)s * fslot_bytes;
                         mbar_expect_tx(&S.ffull[s], (uint32_t)(4 * d + 16));
                         bulk_g2s(dst, w1 + (size_t)j * 2 * d, (uint32_t)(2 * d), &S.ffull[s]);
@@ -431,24 +429,29 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
     int rpar = 0;
     T* xs = reinterpret_cast<T*>(S.xs);
     const int R1 = p.R1, R2 = p.R2;
-    const int words = n >> 5;
     bool ok = true;
+    int l = 0;                 // layer whose FFN is in flight (indexes the trace rows)
 
-    for (int l = 0; l <= p.L && ok; ++l) {
-        const LayerW& W = p.layer[l < p.L ? l : 0];
-        // -------------------------------------------------------------- phase A: form x_l
-        // this layer's bias slices, in the same round trip as the input
-        if (l < p.L) {
-            const T* bp1 = reinterpret_cast<const T*>(W.bp1);
-            const T* bp2 = reinterpret_cast<const T*>(W.bp2);
-            const T* b2p = reinterpret_cast<const T*>(W.b2);
-            const int ng = d >> 2;
-            const int c0 = split_lo(ng, G, c) * 4, c1 = split_lo(ng, G, c + 1) * 4;
+    // bias slices: bp1/bp2 of predictor layer q and b2 of FFN layer f (-1: none)
+    auto load_biases = [&](int q, int f) {
+        if (q >= 0) {
+            const T* bp1 = reinterpret_cast<const T*>(p.layer[q].bp1);
+            const T* bp2 = reinterpret_cast<const T*>(p.layer[q].bp2);
             for (int i = tid; i < b1 - b0; i += kConsumers) S.bias2[i] = bp2 ? DT<T>::f(bp2[b0 + i]) : 0.f;
             if (tid < a1 - a0) S.bias1[tid] = bp1 ? DT<T>::f(bp1[a0 + tid]) : 0.f;
+        }
+        if (f >= 0) {
+            const T* b2p = reinterpret_cast<const T*>(p.layer[f].b2);
+            const int ng = d >> 2;
+            const int c0 = split_lo(ng, G, c) * 4, c1 = split_lo(ng, G, c + 1) * 4;
             if (tid < c1 - c0) S.biasy[tid] = b2p ? DT<T>::f(b2p[c0 + tid]) : 0.f;
         }
-        // Thread tid owns the 16-byte column vectors v = tid + m*256 of x.
+    };
+
+    // x of layer l into shared memory: the input itself for l == 0, else
+    // round(u / rms(u)) from the previous layer's u = x + y.  Thread tid owns the
+    // 16-byte column vectors v = tid + m*256.  For l == L the result is the output.
+    auto form_x = [&](int l) {
         if (l == 0) {
             const T* xin = reinterpret_cast<const T*>(p.x_in);
 #pragma unroll
@@ -460,457 +463,519 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
                         reinterpret_cast<uint4*>(xs + (size_t)t * d)[v] =
                             __ldcg(reinterpret_cast<const uint4*>(xin + (size_t)t * d) + v);
             }
-        } else {
-            float4 uv[kMaxVPT][2][NB];
+            return;
+        }
+        float4 uv[kMaxVPT][2][NB];
 #pragma unroll
-            for (int m = 0; m < kMaxVPT; ++m) {
-                const int v = tid + m * kConsumers;
-#pragma unroll
-                for (int t = 0; t < NB; ++t) {
-                    if (v < nvec) {
-                        const float4* up = reinterpret_cast<const float4*>(p.u + (size_t)t * d + v * 8);
-                        uv[m][0][t] = __ldcg(up);
-                        uv[m][1][t] = __ldcg(up + 1);
-                    }
-                }
-            }
-            // rms of u = x + y from the loaded values themselves (same tree in every CTA)
-            {
-                float sq[NB];
-#pragma unroll
-                for (int t = 0; t < NB; ++t) {
-                    sq[t] = 0.f;
-#pragma unroll
-                    for (int m = 0; m < kMaxVPT; ++m) {
-                        const int v = tid + m * kConsumers;
-                        if (v < nvec) {
-                            const float4 a = uv[m][0][t], b = uv[m][1][t];
-                            sq[t] = fmaf(a.x, a.x, sq[t]); sq[t] = fmaf(a.y, a.y, sq[t]);
-                            sq[t] = fmaf(a.z, a.z, sq[t]); sq[t] = fmaf(a.w, a.w, sq[t]);
-                            sq[t] = fmaf(b.x, b.x, sq[t]); sq[t] = fmaf(b.y, b.y, sq[t]);
-                            sq[t] = fmaf(b.z, b.z, sq[t]); sq[t] = fmaf(b.w, b.w, sq[t]);
-                        }
-                    }
-                    sq[t] = warp_sum(sq[t]);
-                    if (lane == 0) S.red2[warp * NB + t] = sq[t];
-                }
-                consumer_sync();
-                if (tid < NB) {
-                    float z = 0.f;
-                    for (int q = 0; q < kConsumerWarps; ++q) z += S.red2[q * NB + tid];
-                    S.misc[tid] = 1.0f / sqrtf(z / (float)d + 1e-6f);
-                }
-            }
-            consumer_sync();
+        for (int m = 0; m < kMaxVPT; ++m) {
+            const int v = tid + m * kConsumers;
 #pragma unroll
             for (int t = 0; t < NB; ++t) {
-                const float rs = S.misc[t];
+                if (v < nvec) {
+                    const float4* up = reinterpret_cast<const float4*>(p.u + (size_t)t * d + v * 8);
+                    uv[m][0][t] = __ldcg(up);
+                    uv[m][1][t] = __ldcg(up + 1);
+                }
+            }
+        }
+        // rms of u from the loaded values themselves (same tree in every CTA)
+        {
+            float sq[NB];
+#pragma unroll
+            for (int t = 0; t < NB; ++t) {
+                sq[t] = 0.f;
 #pragma unroll
                 for (int m = 0; m < kMaxVPT; ++m) {
                     const int v = tid + m * kConsumers;
                     if (v < nvec) {
-                        const float f[8] = {uv[m][0][t].x, uv[m][0][t].y, uv[m][0][t].z, uv[m][0][t].w,
-                                            uv[m][1][t].x, uv[m][1][t].y, uv[m][1][t].z, uv[m][1][t].w};
-                        T r8[8];
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) r8[q] = DT<T>::r(f[q] * rs);
-                        reinterpret_cast<uint4*>(xs + (size_t)t * d)[v] = *reinterpret_cast<const uint4*>(r8);
+                        const float4 a = uv[m][0][t], b = uv[m][1][t];
+                        sq[t] = fmaf(a.x, a.x, sq[t]); sq[t] = fmaf(a.y, a.y, sq[t]);
+                        sq[t] = fmaf(a.z, a.z, sq[t]); sq[t] = fmaf(a.w, a.w, sq[t]);
+                        sq[t] = fmaf(b.x, b.x, sq[t]); sq[t] = fmaf(b.y, b.y, sq[t]);
+                        sq[t] = fmaf(b.z, b.z, sq[t]); sq[t] = fmaf(b.w, b.w, sq[t]);
                     }
                 }
+                sq[t] = warp_sum(sq[t]);
+                if (lane == 0) S.red2[warp * NB + t] = sq[t];
             }
-            if (l == p.L) {
-                if (c == 0) {
-                    T* xo = reinterpret_cast<T*>(p.x_out);
-#pragma unroll
-                    for (int m = 0; m < kMaxVPT; ++m) {
-                        const int v = tid + m * kConsumers;
-                        for (int t = 0; t < B; ++t)
-                            if (v < nvec)
-                                reinterpret_cast<uint4*>(xo + (size_t)t * d)[v] =
-                                    reinterpret_cast<const uint4*>(xs + (size_t)t * d)[v];
-                    }
-                }
-                break;
+            consumer_sync();
+            if (tid < NB) {
+                float z = 0.f;
+                for (int q = 0; q < kConsumerWarps; ++q) z += S.red2[q * NB + tid];
+                S.misc[tid] = 1.0f / sqrtf(z / (float)d + 1e-6f);
             }
         }
         consumer_sync();
-        TRACE(0);
-        // GEMV1 over Wp1 rows [a0, a1).  Warp w owns columns [w nvec/8, (w+1) nvec/8) of every
-        // row; its lanes keep that segment of x in registers as fp32 pairs, and the eight
-        // warps' partial dots of a row are added in fixed order through shared memory.
-        {
-            const int seg_lo = split_lo(nvec, kConsumerWarps, warp), seg_hi = split_lo(nvec, kConsumerWarps, warp + 1);
-            u64 xg[kMaxVPT][4][NB];
+#pragma unroll
+        for (int t = 0; t < NB; ++t) {
+            const float rs = S.misc[t];
 #pragma unroll
             for (int m = 0; m < kMaxVPT; ++m) {
-                const int v = seg_lo + lane + 32 * m;
+                const int v = tid + m * kConsumers;
+                if (v < nvec) {
+                    const float f[8] = {uv[m][0][t].x, uv[m][0][t].y, uv[m][0][t].z, uv[m][0][t].w,
+                                        uv[m][1][t].x, uv[m][1][t].y, uv[m][1][t].z, uv[m][1][t].w};
+                    T r8[8];
 #pragma unroll
-                for (int t = 0; t < NB; ++t) {
-                    if (v < seg_hi) {
-                        const uint4 xv = reinterpret_cast<const uint4*>(xs + (size_t)t * d)[v];
-                        xg[m][0][t] = Arith<T>::widen2(xv.x); xg[m][1][t] = Arith<T>::widen2(xv.y);
-                        xg[m][2][t] = Arith<T>::widen2(xv.z); xg[m][3][t] = Arith<T>::widen2(xv.w);
-                    } else {
-                        xg[m][0][t] = xg[m][1][t] = xg[m][2][t] = xg[m][3][t] = 0ull;
-                    }
+                    for (int q = 0; q < 8; ++q) r8[q] = DT<T>::r(f[q] * rs);
+                    reinterpret_cast<uint4*>(xs + (size_t)t * d)[v] = *reinterpret_cast<const uint4*>(r8);
                 }
-            }
-            for (int r = a0; r < a1 && ok; r += R1, ++pk_) {
-                const int s = pk_ % p.pred_slots;
-                if (!cwait(S, p, &S.pfull[s], (pk_ / p.pred_slots) & 1)) { ok = false; break; }
-                if (r == a0) TRACE(1); else TRACE(13);
-                const uint4* slot = reinterpret_cast<const uint4*>(S.pring + (size_t)s * p.pred_slot_bytes);
-                const int rows = min(R1, a1 - r);
-                for (int rr = 0; rr < rows; rr += 2) {
-                    const bool two = rr + 1 < rows;
-                    const uint4* w0p = slot + (size_t)rr * nvec;
-                    const uint4* w1p = slot + (size_t)(two ? rr + 1 : rr) * nvec;
-                    u64 c0[NB], c1[NB];
-#pragma unroll
-                    for (int t = 0; t < NB; ++t) c0[t] = c1[t] = 0ull;
-#pragma unroll
-                    for (int m = 0; m < kMaxVPT; ++m) {
-                        const int v = seg_lo + lane + 32 * m;
-                        if (v < seg_hi) {
-                            const uint4 w0 = w0p[v], w1 = w1p[v];
-                            const u64 p00 = Arith<T>::widen2(w0.x), p01 = Arith<T>::widen2(w0.y);
-                            const u64 p02 = Arith<T>::widen2(w0.z), p03 = Arith<T>::widen2(w0.w);
-                            const u64 p10 = Arith<T>::widen2(w1.x), p11 = Arith<T>::widen2(w1.y);
-                            const u64 p12 = Arith<T>::widen2(w1.z), p13 = Arith<T>::widen2(w1.w);
-#pragma unroll
-                            for (int t = 0; t < NB; ++t) {
-                                ffma2(c0[t], p00, xg[m][0][t]); ffma2(c0[t], p01, xg[m][1][t]);
-                                ffma2(c0[t], p02, xg[m][2][t]); ffma2(c0[t], p03, xg[m][3][t]);
-                                ffma2(c1[t], p10, xg[m][0][t]); ffma2(c1[t], p11, xg[m][1][t]);
-                                ffma2(c1[t], p12, xg[m][2][t]); ffma2(c1[t], p13, xg[m][3][t]);
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int t = 0; t < NB; ++t) {
-                        const float2 e0 = upk(c0[t]), e1 = upk(c1[t]);
-                        const float z0 = warp_sum(e0.x + e0.y), z1 = warp_sum(e1.x + e1.y);
-                        if (lane == 0) {
-                            S.red1[(rr * kConsumerWarps + warp) * NB + t] = z0;
-                            if (two) S.red1[((rr + 1) * kConsumerWarps + warp) * NB + t] = z1;
-                        }
-                    }
-                }
-                if (r == a0) TRACE(12); else TRACE(14);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&S.pempty[s]);
-                consumer_sync();
-                if (tid < rows * NB) {
-                    const int rr = tid / NB, t = tid % NB;
-                    float zz = 0.f;
-#pragma unroll
-                    for (int q = 0; q < kConsumerWarps; ++q) zz += S.red1[(rr * kConsumerWarps + q) * NB + t];
-                    if (t < B) p.h[(size_t)t * H + r + rr] = fmaxf(zz + S.bias1[r + rr - a0], 0.f);
-                }
-                consumer_sync();
             }
         }
-        TRACE(2);
-        if (!ok || !grid_barrier(S, p, epoch)) { ok = false; break; }
-        TRACE(3);
+        if (l == p.L && c == 0) {
+            T* xo = reinterpret_cast<T*>(p.x_out);
+#pragma unroll
+            for (int m = 0; m < kMaxVPT; ++m) {
+                const int v = tid + m * kConsumers;
+                for (int t = 0; t < B; ++t)
+                    if (v < nvec)
+                        reinterpret_cast<uint4*>(xo + (size_t)t * d)[v] =
+                            reinterpret_cast<const uint4*>(xs + (size_t)t * d)[v];
+            }
+        }
+    };
 
-        // -------------------------------------------------------------- phase B: logits, own FFN
-        // Lane l keeps h's 16-byte column groups v = l + 32 i in registers as fp32 pairs.
-        // Every selected neuron of this CTA's rows is appended (ascending) to the CTA's
-        // list as soon as its chunk is done, so the FFN producer starts gathering its
-        // W1/W2T rows while the rest of Wp2 still streams.
-        int m = 0;                                  // selected neurons of this CTA in this layer
-        {
-            constexpr int kHV = HV;                // H <= 256 * HV
-            // one L2 read of h per CTA (every CTA reads the same few lines: keep that traffic small)
-            for (int i = tid; i < (NB * H) >> 2; i += kConsumers)
-                reinterpret_cast<float4*>(S.hs)[i] = __ldcg(reinterpret_cast<const float4*>(p.h) + i);
-            consumer_sync();
-            u64 hr[kHV][4][NB];
+    // h = ReLU(Wp1 x + bp1) over this CTA's Wp1 rows [a0, a1) of the next predictor
+    // layer in the ring, from the x in shared memory.  Warp w owns columns
+    // [w nvec/8, (w+1) nvec/8) of every row; its lanes keep that segment of x in
+    // registers as fp32 pairs, and the eight warps' partial dots of a row are added
+    // in fixed order through shared memory.
+    auto gemv1 = [&]() -> bool {
+        const int seg_lo = split_lo(nvec, kConsumerWarps, warp), seg_hi = split_lo(nvec, kConsumerWarps, warp + 1);
+        u64 xg[kMaxVPT][4][NB];
 #pragma unroll
-            for (int i = 0; i < kHV; ++i) {
-                const int v = lane + 32 * i;
+        for (int m = 0; m < kMaxVPT; ++m) {
+            const int v = seg_lo + lane + 32 * m;
 #pragma unroll
-                for (int t = 0; t < NB; ++t) {
-                    if (v < hv) {
-                        const float4* hp = reinterpret_cast<const float4*>(S.hs + (size_t)t * H + v * 8);
-                        const float4 a = hp[0], b = hp[1];
-                        hr[i][0][t] = pk(a.x, a.y); hr[i][1][t] = pk(a.z, a.w);
-                        hr[i][2][t] = pk(b.x, b.y); hr[i][3][t] = pk(b.z, b.w);
-                    } else {
-                        hr[i][0][t] = hr[i][1][t] = hr[i][2][t] = hr[i][3][t] = 0ull;
-                    }
-                }
-            }
-            TRACE(4);
-            for (int r = b0; r < b1 && ok; r += R2, ++pk_) {
-                const int s = pk_ % p.pred_slots;
-                if (!cwait(S, p, &S.pfull[s], (pk_ / p.pred_slots) & 1)) { ok = false; break; }
-                if (r == b0) TRACE(5);
-                const uint4* slot = reinterpret_cast<const uint4*>(S.pring + (size_t)s * p.pred_slot_bytes);
-                const int rows = min(R2, b1 - r);
-                // two rows per warp per step for independent FMA chains
-                for (int rr = warp; rr < rows; rr += 2 * kConsumerWarps) {
-                    const int rr2 = rr + kConsumerWarps;
-                    const bool two = rr2 < rows;
-                    const uint4* w0p = slot + (size_t)rr * hv;
-                    const uint4* w1p = slot + (size_t)(two ? rr2 : rr) * hv;
-                    u64 a0[2][NB], a1[2][NB];
-#pragma unroll
-                    for (int t = 0; t < NB; ++t) a0[0][t] = a0[1][t] = a1[0][t] = a1[1][t] = 0ull;
-#pragma unroll
-                    for (int i = 0; i < kHV; ++i) {
-                        const int v = lane + 32 * i;
-                        if (v < hv) {
-                            const uint4 w0 = w0p[v], w1 = w1p[v];
-                            const u64 p00 = Arith<T>::widen2(w0.x), p01 = Arith<T>::widen2(w0.y);
-                            const u64 p02 = Arith<T>::widen2(w0.z), p03 = Arith<T>::widen2(w0.w);
-                            const u64 p10 = Arith<T>::widen2(w1.x), p11 = Arith<T>::widen2(w1.y);
-                            const u64 p12 = Arith<T>::widen2(w1.z), p13 = Arith<T>::widen2(w1.w);
-#pragma unroll
-                            for (int t = 0; t < NB; ++t) {
-                                ffma2(a0[0][t], p00, hr[i][0][t]); ffma2(a0[1][t], p01, hr[i][1][t]);
-                                ffma2(a0[0][t], p02, hr[i][2][t]); ffma2(a0[1][t], p03, hr[i][3][t]);
-                                ffma2(a1[0][t], p10, hr[i][0][t]); ffma2(a1[1][t], p11, hr[i][1][t]);
-                                ffma2(a1[0][t], p12, hr[i][2][t]); ffma2(a1[1][t], p13, hr[i][3][t]);
-                            }
-                        }
-                    }
-                    bool any0 = false, any1 = false;
-#pragma unroll
-                    for (int t = 0; t < NB; ++t) {
-                        const float2 x0 = upk(a0[0][t]), x1 = upk(a0[1][t]);
-                        const float2 y0 = upk(a1[0][t]), y1 = upk(a1[1][t]);
-                        const float z0 = warp_sum((x0.x + x0.y) + (x1.x + x1.y));
-                        const float z1 = warp_sum((y0.x + y0.y) + (y1.x + y1.y));
-                        if (t < B) {
-                            any0 |= (z0 + S.bias2[r + rr - b0]) > 0.f;
-                            if (two) any1 |= (z1 + S.bias2[r + rr2 - b0]) > 0.f;
-                        }
-                    }
-                    if (lane == 0) {
-                        S.sel[rr] = any0;
-                        if (two) S.sel[rr2] = any1;
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&S.pempty[s]);
-                consumer_sync();
-                // append this chunk's selected rows in ascending order and publish the count
-                if (warp == 0) {
-                    for (int q0 = 0; q0 < rows; q0 += 32) {
-                        const bool on = q0 + lane < rows && S.sel[q0 + lane];
-                        const uint32_t bal = __ballot_sync(0xffffffffu, on);
-                        if (on) S.nl[m + __popc(bal & ((1u << lane) - 1u))] = r + q0 + lane;
-                        m += __popc(bal);
-                    }
-                    __syncwarp();
-                    if (lane == 0) {
-                        __threadfence_block();
-                        S.flags[1] = (l << 16) | m;
-                    }
+            for (int t = 0; t < NB; ++t) {
+                if (v < seg_hi) {
+                    const uint4 xv = reinterpret_cast<const uint4*>(xs + (size_t)t * d)[v];
+                    xg[m][0][t] = Arith<T>::widen2(xv.x); xg[m][1][t] = Arith<T>::widen2(xv.y);
+                    xg[m][2][t] = Arith<T>::widen2(xv.z); xg[m][3][t] = Arith<T>::widen2(xv.w);
+                } else {
+                    xg[m][0][t] = xg[m][1][t] = xg[m][2][t] = xg[m][3][t] = 0ull;
                 }
             }
         }
-        if (!ok) break;
+        for (int r = a0; r < a1; r += R1, ++pk_) {
+            const int s = pk_ % p.pred_slots;
+            if (!cwait(S, p, &S.pfull[s], (pk_ / p.pred_slots) & 1)) return false;
+            if (r == a0) TRACE(1);
+            const uint4* slot = reinterpret_cast<const uint4*>(S.pring + (size_t)s * p.pred_slot_bytes);
+            const int rows = min(R1, a1 - r);
+            for (int rr = 0; rr < rows; rr += 2) {
+                const bool two = rr + 1 < rows;
+                const uint4* w0p = slot + (size_t)rr * nvec;
+                const uint4* w1p = slot + (size_t)(two ? rr + 1 : rr) * nvec;
+                u64 c0[NB], c1[NB];
+#pragma unroll
+                for (int t = 0; t < NB; ++t) c0[t] = c1[t] = 0ull;
+#pragma unroll
+                for (int m = 0; m < kMaxVPT; ++m) {
+                    const int v = seg_lo + lane + 32 * m;
+                    if (v < seg_hi) {
+                        const uint4 w0 = w0p[v], w1 = w1p[v];
+                        const u64 p00 = Arith<T>::widen2(w0.x), p01 = Arith<T>::widen2(w0.y);
+                        const u64 p02 = Arith<T>::widen2(w0.z), p03 = Arith<T>::widen2(w0.w);
+                        const u64 p10 = Arith<T>::widen2(w1.x), p11 = Arith<T>::widen2(w1.y);
+                        const u64 p12 = Arith<T>::widen2(w1.z), p13 = Arith<T>::widen2(w1.w);
+#pragma unroll
+                        for (int t = 0; t < NB; ++t) {
+                            ffma2(c0[t], p00, xg[m][0][t]); ffma2(c0[t], p01, xg[m][1][t]);
+                            ffma2(c0[t], p02, xg[m][2][t]); ffma2(c0[t], p03, xg[m][3][t]);
+                            ffma2(c1[t], p10, xg[m][0][t]); ffma2(c1[t], p11, xg[m][1][t]);
+                            ffma2(c1[t], p12, xg[m][2][t]); ffma2(c1[t], p13, xg[m][3][t]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int t = 0; t < NB; ++t) {
+                    const float2 e0 = upk(c0[t]), e1 = upk(c1[t]);
+                    const float z0 = warp_sum(e0.x + e0.y), z1 = warp_sum(e1.x + e1.y);
+                    if (lane == 0) {
+                        S.red1[(rr * kConsumerWarps + warp) * NB + t] = z0;
+                        if (two) S.red1[((rr + 1) * kConsumerWarps + warp) * NB + t] = z1;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.pempty[s]);
+            consumer_sync();
+            if (tid < rows * NB) {
+                const int rr = tid / NB, t = tid % NB;
+                float zz = 0.f;
+#pragma unroll
+                for (int q = 0; q < kConsumerWarps; ++q) zz += S.red1[(rr * kConsumerWarps + q) * NB + t];
+                if (t < B) p.h[(size_t)t * H + r + rr] = fmaxf(zz + S.bias1[r + rr - a0], 0.f);
+            }
+            consumer_sync();
+        }
+        return true;
+    };
+
+    // Logits of predictor layer q over this CTA's Wp2 rows [b0, b1), threshold, and
+    // this CTA's list of selected neurons (ascending) into list buffer q & 1.  Lane
+    // l keeps h's 16-byte column groups v = l + 32 i in registers as fp32 pairs.  The
+    // list grows chunk by chunk and its length is published at once, so the FFN
+    // producer gathers W1/W2T rows while the rest of Wp2 still streams.  Returns the
+    // final length (-1 on a failed wait); the list is then published as final and its
+    // length stored in the per-CTA counts of parity q & 1.
+    auto gemv2 = [&](int q) -> int {
+        int m = 0;
+        int32_t* nl = S.nl + (q & 1) * p.max_rows;
+        constexpr int kHV = HV;                // H <= 256 * HV
+        // one L2 read of h per CTA (every CTA reads the same few lines: keep that traffic small)
+        for (int i = tid; i < (NB * H) >> 2; i += kConsumers)
+            reinterpret_cast<float4*>(S.hs)[i] = __ldcg(reinterpret_cast<const float4*>(p.h) + i);
+        consumer_sync();
+        u64 hr[kHV][4][NB];
+#pragma unroll
+        for (int i = 0; i < kHV; ++i) {
+            const int v = lane + 32 * i;
+#pragma unroll
+            for (int t = 0; t < NB; ++t) {
+                if (v < hv) {
+                    const float4* hp = reinterpret_cast<const float4*>(S.hs + (size_t)t * H + v * 8);
+                    const float4 a = hp[0], b = hp[1];
+                    hr[i][0][t] = pk(a.x, a.y); hr[i][1][t] = pk(a.z, a.w);
+                    hr[i][2][t] = pk(b.x, b.y); hr[i][3][t] = pk(b.z, b.w);
+                } else {
+                    hr[i][0][t] = hr[i][1][t] = hr[i][2][t] = hr[i][3][t] = 0ull;
+                }
+            }
+        }
+        TRACE(4);
+        for (int r = b0; r < b1; r += R2, ++pk_) {
+            const int s = pk_ % p.pred_slots;
+            if (!cwait(S, p, &S.pfull[s], (pk_ / p.pred_slots) & 1)) return -1;
+            if (r == b0) TRACE(5);
+            const uint4* slot = reinterpret_cast<const uint4*>(S.pring + (size_t)s * p.pred_slot_bytes);
+            const int rows = min(R2, b1 - r);
+            // two rows per warp per step for independent FMA chains
+            for (int rr = warp; rr < rows; rr += 2 * kConsumerWarps) {
+                const int rr2 = rr + kConsumerWarps;
+                const bool two = rr2 < rows;
+                const uint4* w0p = slot + (size_t)rr * hv;
+                const uint4* w1p = slot + (size_t)(two ? rr2 : rr) * hv;
+                u64 a0[2][NB], a1[2][NB];
+#pragma unroll
+                for (int t = 0; t < NB; ++t) a0[0][t] = a0[1][t] = a1[0][t] = a1[1][t] = 0ull;
+#pragma unroll
+                for (int i = 0; i < kHV; ++i) {
+                    const int v = lane + 32 * i;
+                    if (v < hv) {
+                        const uint4 w0 = w0p[v], w1 = w1p[v];
+                        const u64 p00 = Arith<T>::widen2(w0.x), p01 = Arith<T>::widen2(w0.y);
+                        const u64 p02 = Arith<T>::widen2(w0.z), p03 = Arith<T>::widen2(w0.w);
+                        const u64 p10 = Arith<T>::widen2(w1.x), p11 = Arith<T>::widen2(w1.y);
+                        const u64 p12 = Arith<T>::widen2(w1.z), p13 = Arith<T>::widen2(w1.w);
+#pragma unroll
+                        for (int t = 0; t < NB; ++t) {
+                            ffma2(a0[0][t], p00, hr[i][0][t]); ffma2(a0[1][t], p01, hr[i][1][t]);
+                            ffma2(a0[0][t], p02, hr[i][2][t]); ffma2(a0[1][t], p03, hr[i][3][t]);
+                            ffma2(a1[0][t], p10, hr[i][0][t]); ffma2(a1[1][t], p11, hr[i][1][t]);
+                            ffma2(a1[0][t], p12, hr[i][2][t]); ffma2(a1[1][t], p13, hr[i][3][t]);
+                        }
+                    }
+                }
+                bool any0 = false, any1 = false;
+#pragma unroll
+                for (int t = 0; t < NB; ++t) {
+                    const float2 x0 = upk(a0[0][t]), x1 = upk(a0[1][t]);
+                    const float2 y0 = upk(a1[0][t]), y1 = upk(a1[1][t]);
+                    const float z0 = warp_sum((x0.x + x0.y) + (x1.x + x1.y));
+                    const float z1 = warp_sum((y0.x + y0.y) + (y1.x + y1.y));
+                    if (t < B) {
+                        any0 |= (z0 + S.bias2[r + rr - b0]) > 0.f;
+                        if (two) any1 |= (z1 + S.bias2[r + rr2 - b0]) > 0.f;
+                    }
+                }
+                if (lane == 0) {
+                    S.sel[rr] = any0;
+                    if (two) S.sel[rr2] = any1;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.pempty[s]);
+            consumer_sync();
+            // append this chunk's selected rows in ascending order and publish the count
+            if (warp == 0) {
+                for (int q0 = 0; q0 < rows; q0 += 32) {
+                    const bool on = q0 + lane < rows && S.sel[q0 + lane];
+                    const uint32_t bal = __ballot_sync(0xffffffffu, on);
+                    if (on) nl[m + __popc(bal & ((1u << lane) - 1u))] = r + q0 + lane;
+                    m += __popc(bal);
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    __threadfence_block();
+                    S.flags[1] = (q << 16) | m;
+                }
+            }
+        }
         consumer_sync();
         {
             const int f = S.flags[1];
-            m = ((f >> 16) & 0x7fff) == (l & 0x7fff) ? (f & 0xffff) : 0;   // no rows (b0 == b1): empty list
+            m = ((f >> 16) & 0x7fff) == (q & 0x7fff) ? (f & 0xffff) : 0;   // no rows (b0 == b1): empty list
         }
         consumer_sync();
         if (tid == 0) {
             __threadfence_block();
-            S.flags[7] = l + 1;                       // the list of layer l is final
-            p.cta_count[c] = m;
+            S.flags[7] = q + 1;                       // list q is final
+            p.cta_count[(q & 1) * (G + 1) + c] = m;
         }
         TRACE(6);
-        {
-            // FC1 operand: this thread's x column vectors, packed storage pairs
-            uint4 xr[kMaxVPT][NB];
+        return m;
+    };
+
+    // FFN of layer l over this CTA's list (length m, buffer l & 1): FC1 (vec_dot with
+    // the storage-dtype x) + bias + ReLU, then FC2 (AXPY of the neuron's W2T row) into
+    // a fixed per-CTA fp32 partial, written to partial[c].
+    auto ffn = [&](int l, int m) -> bool {
+        const int32_t* nl = S.nl + (l & 1) * p.max_rows;
+        // FC1 operand: this thread's x column vectors, packed storage pairs
+        uint4 xr[kMaxVPT][NB];
 #pragma unroll
-            for (int a = 0; a < kMaxVPT; ++a) {
-                const int v = tid + a * kConsumers;
+        for (int a = 0; a < kMaxVPT; ++a) {
+            const int v = tid + a * kConsumers;
 #pragma unroll
-                for (int t = 0; t < NB; ++t)
-                    xr[a][t] = v < nvec ? reinterpret_cast<const uint4*>(xs + (size_t)t * d)[v] : make_uint4(0, 0, 0, 0);
-            }
-            u64 acc[kMaxVPT][4][NB];
+            for (int t = 0; t < NB; ++t)
+                xr[a][t] = v < nvec ? reinterpret_cast<const uint4*>(xs + (size_t)t * d)[v] : make_uint4(0, 0, 0, 0);
+        }
+        u64 acc[kMaxVPT][4][NB];
 #pragma unroll
-            for (int a = 0; a < kMaxVPT; ++a)
+        for (int a = 0; a < kMaxVPT; ++a)
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
+            for (int q = 0; q < 4; ++q)
 #pragma unroll
-                    for (int t = 0; t < NB; ++t) acc[a][q][t] = 0ull;
-            // neurons two at a time: one shared-memory reduction per pair
-            for (int i = 0; i < m; i += 2, fk += 2) {
-                const bool two = i + 1 < m;
-                const int s0 = fk % p.ffn_slots, s1 = (fk + 1) % p.ffn_slots;
-                if (!cwait(S, p, &S.ffull[s0], (fk / p.ffn_slots) & 1)) { ok = false; break; }
-                if (two && !cwait(S, p, &S.ffull[s1], ((fk + 1) / p.ffn_slots) & 1)) { ok = false; break; }
-                if (i == 0) TRACE(7);
-                const char* sl0 = S.fring + (size_t)s0 * fslot_bytes;
-                const char* sl1 = S.fring + (size_t)(two ? s1 : s0) * fslot_bytes;
-                float part[2][NB][4];
+                for (int t = 0; t < NB; ++t) acc[a][q][t] = 0ull;
+        // neurons two at a time: one shared-memory reduction per pair
+        for (int i = 0; i < m; i += 2, fk += 2) {
+            const bool two = i + 1 < m;
+            const int s0 = fk % p.ffn_slots, s1 = (fk + 1) % p.ffn_slots;
+            if (!cwait(S, p, &S.ffull[s0], (fk / p.ffn_slots) & 1)) return false;
+            if (two && !cwait(S, p, &S.ffull[s1], ((fk + 1) / p.ffn_slots) & 1)) return false;
+            if (i == 0) TRACE(7);
+            const char* sl0 = S.fring + (size_t)s0 * fslot_bytes;
+            const char* sl1 = S.fring + (size_t)(two ? s1 : s0) * fslot_bytes;
+            float part[2][NB][4];
 #pragma unroll
-                for (int u = 0; u < 2; ++u)
+            for (int u = 0; u < 2; ++u)
 #pragma unroll
-                    for (int t = 0; t < NB; ++t) part[u][t][0] = part[u][t][1] = part[u][t][2] = part[u][t][3] = 0.f;
-#pragma unroll
-                for (int a = 0; a < kMaxVPT; ++a) {
-                    const int v = tid + a * kConsumers;
-                    if (v < nvec) {
-                        const uint4 w0 = reinterpret_cast<const uint4*>(sl0)[v];
-                        const uint4 w1 = reinterpret_cast<const uint4*>(sl1)[v];
-#pragma unroll
-                        for (int t = 0; t < NB; ++t) {
-                            dot_mix<T>(part[0][t], w0, xr[a][t]);
-                            dot_mix<T>(part[1][t], w1, xr[a][t]);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < 2; ++u)
-#pragma unroll
-                    for (int t = 0; t < NB; ++t) {
-                        const float v = warp_sum(sum4(part[u][t]));
-                        if (lane == 0) S.red[((rpar * 8 + warp) * 2 + u) * NB + t] = v;
-                    }
-                consumer_sync();
-                u64 av[2][NB];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const char* sl = u ? sl1 : sl0;
-                    const int j = S.nl[u ? (two ? i + 1 : i) : i];
-                    const float bias = DT<T>::f(reinterpret_cast<const T*>(sl + 4 * d)[j & 7]);
-#pragma unroll
-                    for (int t = 0; t < NB; ++t) {
-                        float z = 0.f;
-#pragma unroll
-                        for (int q = 0; q < kConsumerWarps; ++q) z += S.red[((rpar * 8 + q) * 2 + u) * NB + t];
-                        float a = fmaxf(z + bias, 0.f);
-                        if (u == 1 && !two) a = 0.f;
-                        av[u][t] = pk(a, a);
-                    }
-                }
-                rpar ^= 1;
-#pragma unroll
-                for (int a = 0; a < kMaxVPT; ++a) {
-                    const int v = tid + a * kConsumers;
-                    if (v < nvec) {
-                        const uint4 w0 = reinterpret_cast<const uint4*>(sl0 + 2 * d)[v];
-                        const uint4 w1 = reinterpret_cast<const uint4*>(sl1 + 2 * d)[v];
-                        const u64 q00 = Arith<T>::widen2(w0.x), q01 = Arith<T>::widen2(w0.y);
-                        const u64 q02 = Arith<T>::widen2(w0.z), q03 = Arith<T>::widen2(w0.w);
-#pragma unroll
-                        for (int t = 0; t < NB; ++t) {
-                            ffma2(acc[a][0][t], av[0][t], q00); ffma2(acc[a][1][t], av[0][t], q01);
-                            ffma2(acc[a][2][t], av[0][t], q02); ffma2(acc[a][3][t], av[0][t], q03);
-                        }
-                        if (two) {
-                            const u64 q10 = Arith<T>::widen2(w1.x), q11 = Arith<T>::widen2(w1.y);
-                            const u64 q12 = Arith<T>::widen2(w1.z), q13 = Arith<T>::widen2(w1.w);
-#pragma unroll
-                            for (int t = 0; t < NB; ++t) {
-                                ffma2(acc[a][0][t], av[1][t], q10); ffma2(acc[a][1][t], av[1][t], q11);
-                                ffma2(acc[a][2][t], av[1][t], q12); ffma2(acc[a][3][t], av[1][t], q13);
-                            }
-                        }
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&S.fempty[s0]);
-                    if (two) mbar_arrive(&S.fempty[s1]);
-                }
-                if (!two) fk -= 1;               // only one slot consumed
-            }
-            if (!ok) break;
+                for (int t = 0; t < NB; ++t) part[u][t][0] = part[u][t][1] = part[u][t][2] = part[u][t][3] = 0.f;
 #pragma unroll
             for (int a = 0; a < kMaxVPT; ++a) {
                 const int v = tid + a * kConsumers;
                 if (v < nvec) {
+                    const uint4 w0 = reinterpret_cast<const uint4*>(sl0)[v];
+                    const uint4 w1 = reinterpret_cast<const uint4*>(sl1)[v];
 #pragma unroll
                     for (int t = 0; t < NB; ++t) {
-                        float4* dst = reinterpret_cast<float4*>(p.partial + ((size_t)c * NB + t) * d + v * 8);
-                        const float2 e0 = upk(acc[a][0][t]), e1 = upk(acc[a][1][t]);
-                        const float2 e2 = upk(acc[a][2][t]), e3 = upk(acc[a][3][t]);
-                        __stcg(dst, make_float4(e0.x, e0.y, e1.x, e1.y));
-                        __stcg(dst + 1, make_float4(e2.x, e2.y, e3.x, e3.y));
+                        dot_mix<T>(part[0][t], w0, xr[a][t]);
+                        dot_mix<T>(part[1][t], w1, xr[a][t]);
                     }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int t = 0; t < NB; ++t) {
+                    const float v = warp_sum(sum4(part[u][t]));
+                    if (lane == 0) S.red[((rpar * 8 + warp) * 2 + u) * NB + t] = v;
+                }
+            consumer_sync();
+            u64 av[2][NB];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const char* sl = u ? sl1 : sl0;
+                const int j = nl[u ? (two ? i + 1 : i) : i];
+                const float bias = DT<T>::f(reinterpret_cast<const T*>(sl + 4 * d)[j & 7]);
+#pragma unroll
+                for (int t = 0; t < NB; ++t) {
+                    float z = 0.f;
+#pragma unroll
+                    for (int q = 0; q < kConsumerWarps; ++q) z += S.red[((rpar * 8 + q) * 2 + u) * NB + t];
+                    float a = fmaxf(z + bias, 0.f);
+                    if (u == 1 && !two) a = 0.f;
+                    av[u][t] = pk(a, a);
+                }
+            }
+            rpar ^= 1;
+#pragma unroll
+            for (int a = 0; a < kMaxVPT; ++a) {
+                const int v = tid + a * kConsumers;
+                if (v < nvec) {
+                    const uint4 w0 = reinterpret_cast<const uint4*>(sl0 + 2 * d)[v];
+                    const uint4 w1 = reinterpret_cast<const uint4*>(sl1 + 2 * d)[v];
+                    const u64 q00 = Arith<T>::widen2(w0.x), q01 = Arith<T>::widen2(w0.y);
+                    const u64 q02 = Arith<T>::widen2(w0.z), q03 = Arith<T>::widen2(w0.w);
+#pragma unroll
+                    for (int t = 0; t < NB; ++t) {
+                        ffma2(acc[a][0][t], av[0][t], q00); ffma2(acc[a][1][t], av[0][t], q01);
+                        ffma2(acc[a][2][t], av[0][t], q02); ffma2(acc[a][3][t], av[0][t], q03);
+                    }
+                    if (two) {
+                        const u64 q10 = Arith<T>::widen2(w1.x), q11 = Arith<T>::widen2(w1.y);
+                        const u64 q12 = Arith<T>::widen2(w1.z), q13 = Arith<T>::widen2(w1.w);
+#pragma unroll
+                        for (int t = 0; t < NB; ++t) {
+                            ffma2(acc[a][0][t], av[1][t], q10); ffma2(acc[a][1][t], av[1][t], q11);
+                            ffma2(acc[a][2][t], av[1][t], q12); ffma2(acc[a][3][t], av[1][t], q13);
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&S.fempty[s0]);
+                if (two) mbar_arrive(&S.fempty[s1]);
+            }
+            if (!two) fk -= 1;               // only one slot consumed
+        }
+#pragma unroll
+        for (int a = 0; a < kMaxVPT; ++a) {
+            const int v = tid + a * kConsumers;
+            if (v < nvec) {
+#pragma unroll
+                for (int t = 0; t < NB; ++t) {
+                    float4* dst = reinterpret_cast<float4*>(p.partial + ((size_t)c * NB + t) * d + v * 8);
+                    const float2 e0 = upk(acc[a][0][t]), e1 = upk(acc[a][1][t]);
+                    const float2 e2 = upk(acc[a][2][t]), e3 = upk(acc[a][3][t]);
+                    __stcg(dst, make_float4(e0.x, e0.y, e1.x, e1.y));
+                    __stcg(dst + 1, make_float4(e2.x, e2.y, e3.x, e3.y));
                 }
             }
         }
         TRACE(8);
-        if (!grid_barrier(S, p, epoch)) { ok = false; break; }
-        TRACE(9);
+        return true;
+    };
 
-        // -------------------------------------------------------------- phase D: reduce, u = x + y
-        {
-            // neuron table of layer l: this CTA's ascending entries at their global positions
-            {
-                const int v = tid < G ? __ldcg(p.cta_count + tid) : 0;
-                if (tid < G) S.scan[tid] = v;
+    // y of layer l for this CTA's column groups: b2 + the G partials added in fixed
+    // order, and u = x + y for the next layer (y itself kept for the last layer).
+    auto reduce = [&](int l) {
+        const int NG = d >> 2;                         // float4 column groups
+        const int g0 = split_lo(NG, G, c), g1 = split_lo(NG, G, c + 1);
+        const int tasks = (g1 - g0) * NB;
+        for (int task = warp; task < tasks; task += kConsumerWarps) {
+            const int g = g0 + task / NB, t = task % NB;
+            float4 v[kMaxG / 32];
+#pragma unroll
+            for (int i = 0; i < kMaxG / 32; ++i) {
+                const int s = lane + 32 * i;
+                v[i] = s < G ? __ldcg(reinterpret_cast<const float4*>(p.partial + ((size_t)s * NB + t) * d + g * 4))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
             }
-        }
-        {
-            const int NG = d >> 2;                         // float4 column groups
-            const int g0 = split_lo(NG, G, c), g1 = split_lo(NG, G, c + 1);
-            const int tasks = (g1 - g0) * NB;
-            for (int task = warp; task < tasks; task += kConsumerWarps) {
-                const int g = g0 + task / NB, t = task % NB;
-                float4 v[kMaxG / 32];
+            float4 a = v[0];
 #pragma unroll
-                for (int i = 0; i < kMaxG / 32; ++i) {
-                    const int s = lane + 32 * i;
-                    v[i] = s < G ? __ldcg(reinterpret_cast<const float4*>(p.partial + ((size_t)s * NB + t) * d + g * 4))
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-                float4 a = v[0];
-#pragma unroll
-                for (int i = 1; i < kMaxG / 32; ++i) { a.x += v[i].x; a.y += v[i].y; a.z += v[i].z; a.w += v[i].w; }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    a.x += __shfl_xor_sync(0xffffffffu, a.x, o);
-                    a.y += __shfl_xor_sync(0xffffffffu, a.y, o);
-                    a.z += __shfl_xor_sync(0xffffffffu, a.z, o);
-                    a.w += __shfl_xor_sync(0xffffffffu, a.w, o);
-                }
-                if (lane == 0 && t < B) {
-                    float yv[4] = {a.x, a.y, a.z, a.w};
-                    float uv[4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int col = g * 4 + q;
-                        yv[q] += S.biasy[col - g0 * 4];
-                        uv[q] = DT<T>::f(xs[(size_t)t * d + col]) + yv[q];
-                    }
-                    if (l == p.L - 1)
-                        *reinterpret_cast<float4*>(p.y + (size_t)t * d + g * 4) = make_float4(yv[0], yv[1], yv[2], yv[3]);
-                    __stcg(reinterpret_cast<float4*>(p.u + (size_t)t * d + g * 4), make_float4(uv[0], uv[1], uv[2], uv[3]));
-                }
-            }
-        }
-        consumer_sync();
-        if (warp == 0) {
-            int off = 0, tot = 0;
-            for (int g = lane; g < G; g += 32) {
-                const int v = S.scan[g];
-                off += g < c ? v : 0;
-                tot += v;
-            }
+            for (int i = 1; i < kMaxG / 32; ++i) { a.x += v[i].x; a.y += v[i].y; a.z += v[i].z; a.w += v[i].w; }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
-                off += __shfl_xor_sync(0xffffffffu, off, o);
-                tot += __shfl_xor_sync(0xffffffffu, tot, o);
+                a.x += __shfl_xor_sync(0xffffffffu, a.x, o);
+                a.y += __shfl_xor_sync(0xffffffffu, a.y, o);
+                a.z += __shfl_xor_sync(0xffffffffu, a.z, o);
+                a.w += __shfl_xor_sync(0xffffffffu, a.w, o);
             }
-            for (int i = lane; i < m; i += 32) W.idx[off + i] = S.nl[i];
-            if (c == 0 && lane == 0 && p.counts) p.counts[l] = tot;
+            if (lane == 0 && t < B) {
+                float yv[4] = {a.x, a.y, a.z, a.w};
+                float uv[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int col = g * 4 + q;
+                    yv[q] += S.biasy[col - g0 * 4];
+                    uv[q] = DT<T>::f(xs[(size_t)t * d + col]) + yv[q];
+                }
+                if (l == p.L - 1)
+                    *reinterpret_cast<float4*>(p.y + (size_t)t * d + g * 4) = make_float4(yv[0], yv[1], yv[2], yv[3]);
+                __stcg(reinterpret_cast<float4*>(p.u + (size_t)t * d + g * 4), make_float4(uv[0], uv[1], uv[2], uv[3]));
+            }
         }
-        TRACE(10);
-        if (!grid_barrier(S, p, epoch)) { ok = false; break; }
-        TRACE(11);
+    };
+
+    // neuron table of layer l: this CTA's ascending entries (list buffer l & 1) at
+    // their global positions, from every CTA's count of that list; CTA 0 stores the
+    // total.  The last consumer warp only (it has no reduction task at B = 1 when a
+    // CTA owns fewer than 8 column groups, so the count loads overlap the reduction).
+    auto table = [&](int l, int m) {
+        if (warp != kConsumerWarps - 1) return;
+        const int32_t* cnt = p.cta_count + (l & 1) * (G + 1);
+        const int32_t* nl = S.nl + (l & 1) * p.max_rows;
+        int off = 0, tot = 0;
+        for (int g = lane; g < G; g += 32) {
+            const int v = __ldcg(cnt + g);
+            off += g < c ? v : 0;
+            tot += v;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            off += __shfl_xor_sync(0xffffffffu, off, o);
+            tot += __shfl_xor_sync(0xffffffffu, tot, o);
+        }
+        int32_t* idx = p.layer[l].idx;
+        for (int i = lane; i < m; i += 32) idx[off + i] = nl[i];
+        if (c == 0 && lane == 0 && p.counts) p.counts[l] = tot;
+    };
+
+    if constexpr (!LA) {
+        // Per layer l: A  x_l, h_l (Wp1 rows)            | grid barrier
+        //              B  logits_l, list_l, FFN_l -> partial | grid barrier
+        //              D  y_l, u_l, table_l                | grid barrier
+        for (l = 0; l < p.L && ok; ++l) {
+            load_biases(l, l);
+            form_x(l);
+            consumer_sync();
+            TRACE(0);
+            if (!gemv1()) { ok = false; break; }
+            TRACE(2);
+            if (!grid_barrier(S, p, epoch)) { ok = false; break; }
+            TRACE(3);
+            const int m = gemv2(l);
+            if (m < 0) { ok = false; break; }
+            if (!ffn(l, m)) { ok = false; break; }
+            if (!grid_barrier(S, p, epoch)) { ok = false; break; }
+            TRACE(9);
+            table(l, m);
+            reduce(l);
+            TRACE(10);
+            if (!grid_barrier(S, p, epoch)) { ok = false; break; }
+            TRACE(11);
+        }
+    } else {
+        // Look-ahead: the neuron set of layer l+1 is predicted from x_l, so each layer
+        // has two grid barriers and the FFN rows of layer l are gathered while layer
+        // l-1's grid still runs.  Prologue: x_0, h_0 | barrier | logits_0, list_0.
+        // Per layer l: x_l, h_{l+1}, FFN_l -> partial      | grid barrier
+        //              logits_{l+1}, list_{l+1}; y_l, u_l, table_l | grid barrier
+        int m = 0;
+        load_biases(0, -1);
+        form_x(0);
+        consumer_sync();
+        if (!gemv1() || !grid_barrier(S, p, epoch)) ok = false;
+        if (ok) {
+            m = gemv2(0);
+            if (m < 0) ok = false;
+        }
+        for (l = 0; l < p.L && ok; ++l) {
+            const bool next = l + 1 < p.L;
+            load_biases(next ? l + 1 : -1, l);
+            if (l > 0) form_x(l);
+            consumer_sync();
+            TRACE(0);
+            if (next && !gemv1()) { ok = false; break; }
+            TRACE(2);
+            if (!ffn(l, m)) { ok = false; break; }
+            if (!grid_barrier(S, p, epoch)) { ok = false; break; }
+            TRACE(3);
+            const int m_next = next ? gemv2(l + 1) : 0;
+            if (m_next < 0) { ok = false; break; }
+            table(l, m);
+            reduce(l);
+            m = m_next;
+            TRACE(10);
+            if (!grid_barrier(S, p, epoch)) { ok = false; break; }
+            TRACE(11);
+        }
     }
+    if (ok) form_x(p.L);
 
     // ---- drain: never leave a bulk copy in flight
     if (!ok) {
@@ -946,7 +1011,7 @@ struct Geometry {
 };
 
 template <typename T, int NB>
-Geometry geometry(const spffn_config& c, int G) {
+Geometry geometry(const spffn_config& c, int G, bool lookahead) {
     Geometry g;
     const int budget = 227 * 1024;
     g.pred_slot_bytes = 32 * 1024;
@@ -959,15 +1024,17 @@ Geometry geometry(const spffn_config& c, int G) {
     fixed += ((size_t)NB * c.d * sizeof(T) + 127) / 128 * 128;      // xs
     fixed += ((size_t)NB * c.H * 4 + 127) / 128 * 128;              // hs
     fixed += (g.max_rows + 127) / 128 * 128;                         // sel
-    fixed += ((size_t)g.max_rows * 4 + 127) / 128 * 128;             // nl
+    fixed += ((size_t)2 * g.max_rows * 4 + 127) / 128 * 128;         // nl, two lists
     fixed += ((size_t)(c.H / G + 2) * 4 + 127) / 128 * 128;          // bias1
     fixed += ((size_t)g.max_rows * 4 + 127) / 128 * 128;             // bias2
     fixed += ((size_t)(c.d / G + 8) * 4 + 127) / 128 * 128;          // biasy
-    fixed += 2 * 8 * 2 * NB * 4 + 8 * NB * 4 + 32 * 8 * NB * 4 + (kMaxG + 1) * 4 + 16 * 4 + 16;
-    fixed += 8 * (2 * 8 + 2 * 8 + 1) + 8 * 8 + 128;                  // barriers + flags + slack
+    fixed += 2 * 8 * 2 * NB * 4 + 8 * NB * 4 + 32 * 8 * NB * 4 + 16 * 4 + 16;
+    fixed += 8 * (2 * 8 + 2 * 8) + 8 * 8 + 128;                      // barriers + flags + slack
     const size_t fslot = 4 * (size_t)c.d + 128;
-    g.pred_slots = 4;
-    g.ffn_slots = 8;
+    // look-ahead gathers a layer's FFN rows while the previous layer still runs, so
+    // it trades a predictor slot for more FFN slots
+    g.pred_slots = lookahead ? 3 : 4;
+    g.ffn_slots = lookahead ? 10 : 8;
     auto total = [&]() { return fixed + (size_t)g.pred_slots * g.pred_slot_bytes + g.ffn_slots * fslot; };
     while (total() > (size_t)budget && g.ffn_slots > 3) --g.ffn_slots;
     while (total() > (size_t)budget && g.pred_slots > 3) --g.pred_slots;
@@ -977,13 +1044,13 @@ Geometry geometry(const spffn_config& c, int G) {
     return g;
 }
 
-template <typename T, int NB, int HV>
+template <typename T, int NB, int HV, bool LA>
 cudaError_t launch_t(spffn_ctx* const* layers, int L, const void* x_in, int B, void* x_out, float* y,
                      int32_t* counts, cudaStream_t st)
 {
     const spffn_ctx& c0 = *layers[0];
     const int G = c0.lay.S;
-    Geometry g = geometry<T, NB>(c0.cfg, G);
+    Geometry g = geometry<T, NB>(c0.cfg, G, LA);
     if (g.smem > 227 * 1024) return cudaErrorInvalidConfiguration;
     static Params p;   // host staging copy; the launch copies it into the kernel's parameter space
     p.L = L; p.B = B; p.d = c0.cfg.d; p.n = c0.cfg.n; p.H = c0.cfg.H; p.G = G;
@@ -992,12 +1059,10 @@ cudaError_t launch_t(spffn_ctx* const* layers, int L, const void* x_in, int B, v
     p.bar = &ctl->barrier[0];
     p.err = &ctl->err;
     p.abort = &ctl->barrier[1];
-    p.mask = c0.mask2();
     p.cta_count = c0.ctacnt();
     p.h = c0.h();
     p.partial = c0.partial();
     p.u = c0.ybuf();
-    p.ss = c0.ssbuf();
     p.pred_slots = g.pred_slots; p.pred_slot_bytes = g.pred_slot_bytes; p.ffn_slots = g.ffn_slots;
     p.R1 = g.R1; p.R2 = g.R2; p.max_rows = g.max_rows;
     p.trace = (g_trace && g_trace_bytes >= (size_t)G * L * kTraceMarks * 8) ? g_trace : nullptr;
@@ -1005,7 +1070,7 @@ cudaError_t launch_t(spffn_ctx* const* layers, int L, const void* x_in, int B, v
         const spffn_ctx& c = *layers[l];
         p.layer[l] = LayerW{c.w.W1, c.w.b1, c.w.W2T, c.w.b2, c.w.Wp1, c.w.bp1, c.w.Wp2, c.w.bp2, c.idx()};
     }
-    cudaError_t e = cudaFuncSetAttribute(k_decode<T, NB, HV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem);
+    cudaError_t e = cudaFuncSetAttribute(k_decode<T, NB, HV, LA>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem);
     if (e != cudaSuccess) return e;
     e = cudaMemsetAsync(&ctl->barrier[0], 0, 2 * sizeof(uint32_t), st);
     if (e != cudaSuccess) return e;
@@ -1019,7 +1084,7 @@ cudaError_t launch_t(spffn_ctx* const* layers, int L, const void* x_in, int B, v
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_decode<T, NB, HV>, p);
+    return cudaLaunchKernelEx(&cfg, k_decode<T, NB, HV, LA>, p);
 }
 
 }  // namespace
@@ -1049,11 +1114,13 @@ void set_trace(void* buf, size_t bytes)
 int trace_marks() { return kTraceMarks; }
 
 cudaError_t launch_fused_decode(spffn_ctx* const* layers, int L, const void* x_in, int B, void* x_out, float* y,
-                                int32_t* counts, cudaStream_t st)
+                                int32_t* counts, bool lookahead, cudaStream_t st)
 {
     const bool bf = layers[0]->cfg.dtype == SPFFN_BF16;
     const int hvn = (layers[0]->cfg.H + 255) / 256;
-#define SPFFN_GO(TT, NBV, HVV) return launch_t<TT, NBV, HVV>(layers, L, x_in, B, x_out, y, counts, st)
+#define SPFFN_GO(TT, NBV, HVV)                                                                        \
+    return lookahead ? launch_t<TT, NBV, HVV, true>(layers, L, x_in, B, x_out, y, counts, st)         \
+                     : launch_t<TT, NBV, HVV, false>(layers, L, x_in, B, x_out, y, counts, st)
 #define SPFFN_HV(TT, NBV)                                     \
     if (hvn <= 1) SPFFN_GO(TT, NBV, 1);                       \
     if (hvn <= 2) SPFFN_GO(TT, NBV, 2);                       \

@@ -30,7 +30,7 @@ struct Ctl {
 };
 
 struct Layout {
-    size_t ctl, h, mask, wcount, partial, xbuf, ybuf, idx, count, mask2, ctacnt, ssbuf, hsplit, asplit, upartial, utickets, total;
+    size_t ctl, h, mask, wcount, partial, xbuf, ybuf, idx, count, ctacnt, hsplit, asplit, upartial, utickets, total;
     int S;  // number of FFN partial sums
 };
 
@@ -50,9 +50,7 @@ inline Layout make_layout(const spffn_config& c, int S) {
     L.ybuf = take((size_t)c.max_batch * c.d * sizeof(float));
     L.idx = take((size_t)c.n * sizeof(int32_t));
     L.count = take(256);
-    L.mask2 = take((size_t)2 * (c.n / 32) * sizeof(uint32_t));
-    L.ctacnt = take((size_t)(S + 1) * sizeof(int32_t));
-    L.ssbuf = take((size_t)S * c.max_batch * sizeof(float));
+    L.ctacnt = take((size_t)2 * (S + 1) * sizeof(int32_t));    // two lists' per-CTA lengths
     L.hsplit = take((size_t)2 * c.max_batch * c.H * 2);
     L.asplit = take((size_t)2 * c.max_batch * c.n * 2);
     if (c.max_batch >= 16) {
@@ -85,9 +83,7 @@ struct spffn_ctx {
     float* ybuf() const { return reinterpret_cast<float*>(ws + lay.ybuf); }
     int32_t* idx() const { return reinterpret_cast<int32_t*>(ws + lay.idx); }
     int32_t* count() const { return reinterpret_cast<int32_t*>(ws + lay.count); }
-    uint32_t* mask2() const { return reinterpret_cast<uint32_t*>(ws + lay.mask2); }
     int32_t* ctacnt() const { return reinterpret_cast<int32_t*>(ws + lay.ctacnt); }
-    float* ssbuf() const { return reinterpret_cast<float*>(ws + lay.ssbuf); }
     void* hsplit() const { return ws + lay.hsplit; }
     void* asplit() const { return ws + lay.asplit; }
     float* upartial() const { return reinterpret_cast<float*>(ws + lay.upartial); }

@@ -8,8 +8,11 @@ weights generated in HBM, hot-first reordered offline (untimed), then K decode
 steps timed with CUDA events.  One step = spffn_decode over all layers:
 predictor (two GEMVs + threshold + compaction), sparse FC1/FC2 with the
 deterministic split reduction, and the chaining into the next layer.
+With --lookahead the step is spffn_decode_lookahead instead (layer l+1's set
+predicted from layer l's input, DejaVu's asynchronous predictor), reported
+under its own workload name.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1] [--lookahead] [--impl ours|reference]
 
 Under torchrun each rank runs its own replica on its own decode stream
 (independent requests: weak scaling, no data-path collective); the reported time
@@ -37,6 +40,12 @@ import workload as wl  # noqa: E402
 METRIC = "sparse-FFN decode tokens/s per layer-stack"
 UNIT = "tokens/s"
 PROFILE_TOKENS = 256
+PREDICTION = {False: "each layer's set predicted from its own input",
+              True: "look-ahead: layer l+1's set predicted from layer l's input"}
+
+
+def workload_name(cfg, args) -> str:
+    return cfg.name + ("-lookahead" if args.lookahead else "")
 
 
 # ---------------------------------------------------------------------------
@@ -92,6 +101,40 @@ def ffn_bytes_per_neuron(cfg) -> int:
 
 def step_bytes(cfg, counts_sum: int, layers: int) -> int:
     return layers * predictor_bytes(cfg) + counts_sum * ffn_bytes_per_neuron(cfg)
+
+
+# DRAM traffic (ncu dram__bytes_read.sum + dram__bytes_write.sum) of the
+# persistent decode kernel per layer, from one capture of a 4-layer stack of the
+# OPT-6.7B-shaped workload at batch 1 (traffic grows with layers, so a launch
+# over L layers is L times this).  It holds only for the kernel sources it was
+# captured on: any change to them and the bench reports null.
+DECODE_SOURCES = ("spffn_fused.cu", "spffn_fused.cuh", "spffn_internal.cuh")
+DECODE_TRAFFIC = {
+    "sha256": "c8d612a3911afc4fa903bbd7678236d3b50a76f446f701dcdba51a16cf9d809a",
+    "workload": "opt6.7b-d4096-n16384-L32", "batch": 1, "rate": 0.05,
+    "bytes_per_layer": (223.093504e6 + 4.497920e6) / 4,
+    "summary": "profiles/k_decode_opt6.7b-d4096-n16384_b1.md",
+}
+
+
+def decode_sources_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "activation_sparse_ffn_predictor_b200", "csrc")
+    for f in DECODE_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def decode_traffic(cfg, layers: int, batch: int, rate, lookahead: bool):
+    """Measured DRAM bytes per launch of the decode kernel for this run, or None."""
+    t = DECODE_TRAFFIC
+    if lookahead or cfg.name != t["workload"] or batch != t["batch"] or (rate or cfg.rate) != t["rate"]:
+        return None
+    if decode_sources_sha256() != t["sha256"]:
+        return None
+    return t["bytes_per_layer"] * layers
 
 
 # ---------------------------------------------------------------------------
@@ -203,7 +246,7 @@ def run_ours(args, cfg, world, rank, local):
     stream = torch.cuda.Stream(device)
 
     def one_step():
-        sp.decode(layers, x_in, x_out, y, counts, stream=stream)
+        sp.decode(layers, x_in, x_out, y, counts, stream=stream, lookahead=args.lookahead)
 
     # CUDA graph of one decode step (removes host launch cost from the timed region)
     with torch.cuda.stream(stream):
@@ -269,13 +312,15 @@ def run_ours(args, cfg, world, rank, local):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": t_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": cfg.dtype, "data": "synthetic",
-        "config": {"workload": cfg.name, "layers": L, "d": cfg.d, "n": cfg.n, "H": cfg.H, "batch": B,
+        "config": {"workload": workload_name(cfg, args), "layers": L, "d": cfg.d, "n": cfg.n, "H": cfg.H, "batch": B,
+                   "prediction": PREDICTION[args.lookahead],
                    "activation_rate": args.rate or cfg.rate, "alpha": cfg.alpha, "global_batch": B * world,
                    "mean_active_neurons": float(ks.mean()), "parallelism": "replicas%d" % world,
                    "placement": "hot-first dealt over %d CTA ranges (offline profile of %d tokens)" % (layers[0].num_partials, PROFILE_TOKENS), "l2": "inputs larger than L2 (%.2f GB touched per step)"
                    % (sum(bytes_per_step) / K / 1e9)},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak,
+                     "traffic": decode_traffic(cfg, L, B, args.rate, args.lookahead) if launches_per_step == 1 else None,
                      "kernel": "spffn decode step (one replay per step)", "peak_kind": peak_kind},
         "e2e": {"value": world * B * K / (e2e_ms * 1e-3), "unit": UNIT,
                 "h2d_bytes_per_step": B * cfg.d * 2, "d2h_bytes_per_step": B * cfg.d * 4},
@@ -346,8 +391,9 @@ def run_reference(args, cfg, world, rank, local):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": cfg.name, "layers": cfg.layers, "d": cfg.d, "n": cfg.n, "H": cfg.H,
-                   "batch": cfg.batch, "activation_rate": args.rate or cfg.rate, "alpha": cfg.alpha},
+        "config": {"workload": workload_name(cfg, args), "layers": cfg.layers, "d": cfg.d, "n": cfg.n, "H": cfg.H,
+                   "batch": cfg.batch, "activation_rate": args.rate or cfg.rate, "alpha": cfg.alpha,
+                   "prediction": PREDICTION[args.lookahead]},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": "%d (layer, step) samples of the first 2 layers, %.1f s of oracle compute, "
                                    "extrapolated to %d layers" % (samples, spent, cfg.layers)},
@@ -369,6 +415,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle compute for cpu_baseline")
     ap.add_argument("--ref-budget", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--lookahead", action="store_true",
+                    help="predict layer l+1's neuron set from layer l's input (DejaVu look-ahead)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

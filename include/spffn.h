@@ -146,8 +146,27 @@ spffn_status spffn_chain(spffn_ctx* ctx, const void* x, const float* y, int32_t 
 spffn_status spffn_decode(spffn_ctx* const* layers, int32_t L, const void* x_in, int32_t B,
                           void* x_out, float* y, int32_t* counts, void* stream);
 
-/* Number of kernels one spffn_decode call with these arguments enqueues (the
- * persistent whole-stack kernel: 1; otherwise 6 per layer), 0 on bad arguments.
+/* spffn_decode with look-ahead prediction (DejaVu's asynchronous predictor,
+ * equation (-2) in the DejaVu appendix of "LLM模型之PowerInfer1.0"): the
+ * neuron set of layer l+1 is predicted from layer l's input, so the predictor
+ * of the next layer runs beside the FFN of this one:
+ *   (idx_0, count_0) = predict_0(x_0)
+ *   for l = 0..L-1:  (idx_{l+1}, count_{l+1}) = predict_{l+1}(x_l)   [l+1 < L]
+ *                    y_l = forward_l(x_l; idx_l);  x_{l+1} = chain(x_l, y_l)
+ * Layer l+1's own predictor weights (Wp1, bp1, Wp2, bp2 of layers[l+1]) are the
+ * ones applied to x_l.  Arguments, outputs and errors as for spffn_decode. */
+spffn_status spffn_decode_lookahead(spffn_ctx* const* layers, int32_t L, const void* x_in, int32_t B,
+                                    void* x_out, float* y, int32_t* counts, void* stream);
+
+/* Device pointer to the neuron table that the last spffn_decode or
+ * spffn_decode_lookahead left in this layer's workspace (ascending neuron
+ * indices; its length is that call's counts[l]).  Valid until the next call
+ * that uses ctx.  Pure host function; INVALID_ARG on a NULL argument. */
+spffn_status spffn_layer_table(spffn_ctx* ctx, const int32_t** idx);
+
+/* Number of kernels one spffn_decode (or spffn_decode_lookahead) call with these
+ * arguments enqueues (the persistent whole-stack kernel: 1; otherwise 6 per
+ * layer), 0 on bad arguments.
  * Pure host function. */
 int32_t spffn_decode_kernel_launches(spffn_ctx* const* layers, int32_t L, int32_t B);
 

@@ -1,0 +1,114 @@
+"""Whole-stack decode, plain (spffn_decode) and with look-ahead prediction
+(spffn_decode_lookahead, DejaVu appendix equation (-2) of "LLM模型之PowerInfer1.0"),
+against the oracle chaining its own layer inputs: every layer's neuron table
+(bit-exact outside the near-threshold band) and count, the last layer's y and
+the final x.  Covers the persistent kernel (B <= 2), the per-layer path (B = 3)
+and the union tensor-core path (B = 16)."""
+import numpy as np
+import pytest
+
+import activation_sparse_ffn_predictor_b200 as sp
+import oracle as O
+import workload as wl
+from _gpu import REL_L2_BAR, ambiguous, check_table, oracle_layer, rel_l2, torch_layer, x_tokens
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "block-d1024-n4096-L4": (wl.CONFIGS[0], 4),
+    "ragged-bf16-d1088-n4128-H320-L3": (wl.FFNConfig("ragged", 1, 1088, 4128, 320, "bf16", 1.0, 0.2), 3),
+    "tiny-d64-n32-H64-L3": (wl.FFNConfig("tiny", 1, 64, 32, 64, "f16", 1.2, 0.3), 3),
+    "wide-d10240-n2048-H64-L2": (wl.FFNConfig("wide", 1, 10240, 2048, 64, "f16", 1.2, 0.1), 2),
+    "bigH-d512-n1024-H8192-L2": (wl.FFNConfig("bigH", 1, 512, 1024, 8192, "bf16", 1.0, 0.1), 2),
+}
+
+
+def oracle_chain(cfg, hs, x64, lookahead):
+    """Oracle per layer on its own chained (rounded) inputs: (idx, k, logits, y) and x_0..x_L."""
+    xs, out = [x64], []
+    for l, h in enumerate(hs):
+        xp = xs[max(l - 1, 0)] if lookahead else xs[l]
+        r = O.step_lookahead(oracle_layer(h), xp, xs[l])
+        out.append(r)
+        xs.append(wl.widen(wl.round_to(O.chain(xs[l], r[3]), cfg.bf16), cfg.bf16))
+    return out, xs
+
+
+def run_and_check(cfg, Lc, B, aux, lookahead, max_batch=None):
+    hs = [wl.host_layer(cfg, l) for l in range(Lc)]
+    layers = [sp.Layer(**torch_layer(h), max_batch=max_batch or B) for h in hs]
+    xb, x64 = x_tokens(cfg, B, aux=aux)
+    dt = torch.bfloat16 if cfg.bf16 else torch.float16
+    x_out = torch.empty(B, cfg.d, dtype=dt, device="cuda")
+    y = torch.empty(B, cfg.d, dtype=torch.float32, device="cuda")
+    counts = torch.full((Lc,), -1, dtype=torch.int32, device="cuda")
+    sp.decode(layers, wl.to_torch(xb, cfg), x_out, y, counts, lookahead=lookahead)
+    torch.cuda.synchronize()
+    for L in layers:
+        assert L.last_device_error() == (sp.OK, 0)
+    want, xs = oracle_chain(cfg, hs, x64, lookahead)
+    kc = counts.cpu().numpy()
+    exact, checked = True, 0
+    for l in range(Lc):
+        idx_or, k_or, logits, y_or = want[l]
+        if not exact:
+            break
+        tab = layers[l].table(int(kc[l])).cpu().numpy()
+        diff = check_table(tab, int(kc[l]), idx_or, logits)
+        assert abs(int(kc[l]) - k_or) <= len(diff)
+        checked += 1
+        # a near-threshold neuron taken differently changes y and every later input
+        exact = not diff
+    if exact:
+        assert rel_l2(y.cpu().numpy(), want[-1][3]) <= REL_L2_BAR
+        got = wl.widen(x_out.cpu().view(torch.int16).numpy().view(np.uint16), cfg.bf16)
+        assert rel_l2(got, xs[-1]) <= REL_L2_BAR
+    assert checked >= 1
+    return kc, want
+
+
+@pytest.mark.parametrize("lookahead", [False, True])
+@pytest.mark.parametrize("B", [1, 2, 3])
+@pytest.mark.parametrize("name", list(CASES))
+def test_decode_tables_match_oracle(name, B, lookahead):
+    cfg, Lc = CASES[name]
+    run_and_check(cfg, Lc, B, aux=500 + B, lookahead=lookahead)
+
+
+@pytest.mark.parametrize("lookahead", [False, True])
+def test_union_decode_tables_match_oracle(lookahead):
+    run_and_check(wl.CONFIGS[0], 3, 16, aux=516, lookahead=lookahead, max_batch=16)
+
+
+def test_lookahead_changes_the_sets():
+    # the two modes agree on layer 0 and (for this seed) differ on a later layer
+    cfg, Lc = CASES["block-d1024-n4096-L4"]
+    k_std, _ = run_and_check(cfg, Lc, 1, aux=9, lookahead=False)
+    k_la, want = run_and_check(cfg, Lc, 1, aux=9, lookahead=True)
+    assert k_std[0] == k_la[0]
+    assert any(k_std[l] != k_la[l] for l in range(1, Lc))
+
+
+def test_lookahead_decode_in_cuda_graph_is_repeatable():
+    cfg, Lc = CASES["block-d1024-n4096-L4"]
+    hs = [wl.host_layer(cfg, l) for l in range(Lc)]
+    layers = [sp.Layer(**torch_layer(h), max_batch=1) for h in hs]
+    x_in = torch.empty(1, cfg.d, dtype=torch.float16, device="cuda")
+    x_out = torch.empty_like(x_in)
+    y = torch.empty(1, cfg.d, dtype=torch.float32, device="cuda")
+    counts = torch.zeros(Lc, dtype=torch.int32, device="cuda")
+    s = torch.cuda.Stream()
+    x_in.copy_(wl.to_torch(wl.tokens(cfg, 1, aux=3), cfg))
+    with torch.cuda.stream(s):
+        sp.decode(layers, x_in, x_out, y, counts, stream=s, lookahead=True)
+    s.synchronize()
+    first = (y.cpu(), x_out.cpu(), counts.cpu())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        sp.decode(layers, x_in, x_out, y, counts, stream=s, lookahead=True)
+    for _ in range(2):
+        g.replay()
+        torch.cuda.synchronize()
+        assert all(torch.equal(a, b) for a, b in zip(first, (y.cpu(), x_out.cpu(), counts.cpu())))
+    del g

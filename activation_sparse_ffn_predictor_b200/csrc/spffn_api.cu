@@ -6,12 +6,16 @@
 #include "spffn_internal.cuh"
 #include "spffn_kernels.cuh"
 #include "spffn_fused.cuh"
+#include "spffn_union.cuh"
 
 using namespace spffn;
 
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Batches above the per-phase kernels' limit run only on the union tensor-core path.
+bool batch_supported(const spffn_ctx& c, int B) { return B <= kMaxPhaseBatch || union_supported(c, B); }
 
 bool valid_config(const spffn_config* c) {
     if (!c) return false;
@@ -107,6 +111,7 @@ spffn_status spffn_predict(spffn_ctx* ctx, const void* x, int32_t B, int32_t* id
                            void* stream) {
     if (!ctx || !x || !idx || !count || B < 1 || B > ctx->cfg.max_batch) return SPFFN_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(idx)) return SPFFN_ERR_INVALID_ARG;
+    if (!batch_supported(*ctx, B)) return SPFFN_ERR_UNSUPPORTED;
     return cuda_status(launch_predict(*ctx, x, B, idx, count, nullptr, (cudaStream_t)stream));
 }
 
@@ -114,6 +119,7 @@ spffn_status spffn_forward(spffn_ctx* ctx, const void* x, int32_t B, const int32
                            const int32_t* count, float* y, void* stream) {
     if (!ctx || !x || !idx || !count || !y || B < 1 || B > ctx->cfg.max_batch) return SPFFN_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(y)) return SPFFN_ERR_INVALID_ARG;
+    if (!batch_supported(*ctx, B)) return SPFFN_ERR_UNSUPPORTED;
     return cuda_status(launch_forward(*ctx, x, B, idx, count, y, (cudaStream_t)stream));
 }
 
@@ -142,6 +148,7 @@ spffn_status decode_impl(spffn_ctx* const* layers, int32_t L, const void* x_in, 
         const spffn_ctx* c = layers[l];
         if (!c || c->cfg.d != l0->cfg.d || c->cfg.dtype != l0->cfg.dtype) return SPFFN_ERR_INVALID_ARG;
         if (B < 1 || B > c->cfg.max_batch) return SPFFN_ERR_INVALID_ARG;
+        if (!batch_supported(*c, B)) return SPFFN_ERR_UNSUPPORTED;
     }
     if (!aligned16(x_in) || !aligned16(x_out) || !aligned16(y) || x_in == x_out) return SPFFN_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
@@ -197,7 +204,14 @@ int32_t spffn_decode_kernel_launches(spffn_ctx* const* layers, int32_t L, int32_
     if (!layers || L < 1 || !layers[0] || B < 1 || B > layers[0]->cfg.max_batch) return 0;
     for (int l = 0; l < L; ++l)
         if (!layers[l]) return 0;
-    return fused_decode_supported(layers, L, B) ? 1 : 6 * L;
+    if (fused_decode_supported(layers, L, B)) return 1;
+    // per layer: predictor hidden, logits (per token group), compaction, FC1, FC2 (per group), chaining
+    int n = 0;
+    for (int l = 0; l < L; ++l) {
+        const int g = union_supported(*layers[l], B) ? union_groups(B).groups : 1;
+        n += 4 + 2 * g;
+    }
+    return n;
 }
 
 spffn_status spffn_set_trace(void* buf, size_t bytes) {

@@ -16,7 +16,8 @@ enum : uint32_t {
     ERR_PIPE_TIMEOUT = 1u << 3,    // a copy-completion wait hit its iteration limit
 };
 
-constexpr int kMaxBatch = 32;
+constexpr int kMaxBatch = 256;       // union tensor-core path (B >= 16, d % 128 == 0)
+constexpr int kMaxPhaseBatch = 32;   // per-phase kernels and the split-FFN partial buffer
 constexpr int kCtlBytes = 1024;    // control block at the head of the workspace
 constexpr int kMaxUnionCtas = 256;  // union path: split-K partial capacity in CTAs
 constexpr int kUnionTickets = 2048;
@@ -30,7 +31,7 @@ struct Ctl {
 };
 
 struct Layout {
-    size_t ctl, h, mask, wcount, partial, xbuf, ybuf, idx, count, ctacnt, hsplit, asplit, upartial, utickets, total;
+    size_t ctl, h, mask, partial, xbuf, ybuf, idx, count, ctacnt, hsplit, asplit, upartial, utickets, total;
     int S;  // number of FFN partial sums
 };
 
@@ -44,17 +45,20 @@ inline Layout make_layout(const spffn_config& c, int S) {
     L.ctl = take(kCtlBytes);
     L.h = take((size_t)c.max_batch * c.H * sizeof(float));
     L.mask = take((size_t)(c.n / 32) * sizeof(uint32_t));
-    L.wcount = take((size_t)(c.n / 32) * sizeof(uint32_t));
-    L.partial = take((size_t)S * c.max_batch * c.d * sizeof(float));
+    const int pb = c.max_batch < kMaxPhaseBatch ? c.max_batch : kMaxPhaseBatch;
+    L.partial = take((size_t)S * pb * c.d * sizeof(float));
     L.xbuf = take((size_t)2 * c.max_batch * c.d * 2);
     L.ybuf = take((size_t)c.max_batch * c.d * sizeof(float));
     L.idx = take((size_t)c.n * sizeof(int32_t));
     L.count = take(256);
     L.ctacnt = take((size_t)2 * (S + 1) * sizeof(int32_t));    // two lists' per-CTA lengths
-    L.hsplit = take((size_t)2 * c.max_batch * c.H * 2);
-    L.asplit = take((size_t)2 * c.max_batch * c.n * 2);
+    // hi/lo activation rows of the union path: token groups of at most 128 (padded to 16)
+    const int srows = 2 * (c.max_batch <= 128 ? (c.max_batch + 15) / 16 * 16 : (c.max_batch + 127) / 128 * 128);
+    L.hsplit = take((size_t)srows * c.H * 2);
+    L.asplit = take((size_t)srows * c.n * 2);
     if (c.max_batch >= 16) {
-        L.upartial = take((size_t)kMaxUnionCtas * 128 * 64 * sizeof(float));
+        const int nmax = c.max_batch > 32 ? 256 : 64;    // widest MMA N of a union launch
+        L.upartial = take((size_t)kMaxUnionCtas * 128 * nmax * sizeof(float));
         L.utickets = take((size_t)kUnionTickets * sizeof(uint32_t));
     } else {
         L.upartial = L.utickets = 0;
@@ -77,7 +81,6 @@ struct spffn_ctx {
     spffn::Ctl* ctl() const { return reinterpret_cast<spffn::Ctl*>(ws + lay.ctl); }
     float* h() const { return reinterpret_cast<float*>(ws + lay.h); }
     uint32_t* mask() const { return reinterpret_cast<uint32_t*>(ws + lay.mask); }
-    uint32_t* wcount() const { return reinterpret_cast<uint32_t*>(ws + lay.wcount); }
     float* partial() const { return reinterpret_cast<float*>(ws + lay.partial); }
     void* xbuf(int i) const { return ws + lay.xbuf + (size_t)i * cfg.max_batch * cfg.d * 2; }
     float* ybuf() const { return reinterpret_cast<float*>(ws + lay.ybuf); }

@@ -60,7 +60,7 @@ __global__ void __launch_bounds__(256) k_hidden(const T* __restrict__ Wp1, const
 template <typename T>
 __global__ void __launch_bounds__(256) k_logits(const T* __restrict__ Wp2, const T* __restrict__ bp2,
                                                 const float* __restrict__ h, int B, int H, int n,
-                                                uint32_t* __restrict__ mask, uint32_t* __restrict__ wcount)
+                                                uint32_t* __restrict__ mask)
 {
     __shared__ int sel[32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(256) k_logits(const T* __restrict__ Wp2, const
         __syncthreads();
         if (warp == 0) {
             uint32_t bits = __ballot_sync(0xffffffffu, sel[lane] != 0);
-            if (lane == 0) { mask[word] = bits; wcount[word] = __popc(bits); }
+            if (lane == 0) mask[word] = bits;
         }
         __syncthreads();
     }
@@ -109,8 +109,7 @@ __global__ void __launch_bounds__(256) k_logits(const T* __restrict__ Wp2, const
 // ---------------------------------------------------------------------------
 // S3  compaction: ascending neuron table from the mask words.  One block of
 // 1024 threads; thread q owns words [q*per, (q+1)*per).
-__global__ void __launch_bounds__(1024) k_compact(const uint32_t* __restrict__ mask,
-                                                  const uint32_t* __restrict__ wcount, int words,
+__global__ void __launch_bounds__(1024) k_compact(const uint32_t* __restrict__ mask, int words,
                                                   int32_t* __restrict__ idx, int32_t* __restrict__ count,
                                                   int32_t* __restrict__ count2)
 {
@@ -119,7 +118,7 @@ __global__ void __launch_bounds__(1024) k_compact(const uint32_t* __restrict__ m
     const int per = (words + 1023) / 1024;
     const int w0 = min(words, tid * per), w1 = min(words, w0 + per);
     uint32_t local = 0;
-    for (int w = w0; w < w1; ++w) local += wcount[w];
+    for (int w = w0; w < w1; ++w) local += __popc(mask[w]);
     // inclusive warp scan
     uint32_t incl = local;
 #pragma unroll
@@ -377,9 +376,8 @@ static cudaError_t predict_impl(const spffn_ctx& c, const void* x, int B, int32_
     const int hb = min((g.H + 7) / 8, c.num_sms * 8);
     k_hidden<T><<<hb, 256, 0, st>>>((const T*)c.w.Wp1, (const T*)c.w.bp1, (const T*)x, B, g.d, g.H, c.h());
     const int words = g.n / 32;
-    k_logits<T><<<words, 256, 0, st>>>((const T*)c.w.Wp2, (const T*)c.w.bp2, c.h(), B, g.H, g.n, c.mask(),
-                                       c.wcount());
-    k_compact<<<1, 1024, 0, st>>>(c.mask(), c.wcount(), words, idx, count, count2);
+    k_logits<T><<<words, 256, 0, st>>>((const T*)c.w.Wp2, (const T*)c.w.bp2, c.h(), B, g.H, g.n, c.mask());
+    k_compact<<<1, 1024, 0, st>>>(c.mask(), words, idx, count, count2);
     return cudaGetLastError();
 }
 
@@ -453,7 +451,7 @@ static cudaError_t profile_impl(const spffn_ctx& c, const void* X, int T_, uint3
 
 cudaError_t launch_compact(const spffn_ctx& c, int32_t* idx, int32_t* count, int32_t* count2, cudaStream_t st)
 {
-    k_compact<<<1, 1024, 0, st>>>(c.mask(), c.wcount(), c.cfg.n / 32, idx, count, count2);
+    k_compact<<<1, 1024, 0, st>>>(c.mask(), c.cfg.n / 32, idx, count, count2);
     return cudaGetLastError();
 }
 

@@ -54,7 +54,7 @@ extern "C" spffn_status spffn_forward_noalloc(const spffn_config* cfg, const spf
     if (cfg->d < 64 || cfg->d > 16384 || cfg->d % 64 || cfg->n < 32 || cfg->n % 32 || cfg->n > 131072)
         return SPFFN_ERR_INVALID_ARG;
     if (cfg->dtype != SPFFN_F16 && cfg->dtype != SPFFN_BF16) return SPFFN_ERR_INVALID_ARG;
-    if (B < 1 || B > spffn::kMaxBatch) return SPFFN_ERR_INVALID_ARG;
+    if (B < 1 || B > spffn::kMaxPhaseBatch) return SPFFN_ERR_INVALID_ARG;
     if (!w->W1 || !w->b1 || !w->W2T) return SPFFN_ERR_INVALID_ARG;
     if (!aligned16(w->W1) || !aligned16(w->W2T) || !aligned16(x) || !aligned16(y)) return SPFFN_ERR_INVALID_ARG;
     // one partial sum is B x d fp32; at least one must fit the fixed scratch

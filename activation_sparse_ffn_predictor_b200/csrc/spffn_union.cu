@@ -31,9 +31,9 @@ namespace {
 constexpr int kUThreads = 192;       // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int kBM = 128;             // D rows per tile
 constexpr int kBK = 64;              // K per stage: one 128-byte swizzle row of 16-bit elements
-constexpr int kStages = 6;
-constexpr int kStageBytes = 24 * 1024;   // A tile 16 KB + B tile up to 8 KB
-constexpr int kTmemCols = 128;       // two accumulators of up to 64 fp32 columns
+constexpr int kMaxStages = 6;       // stage = A tile 16 KB + B tile N x 128 B (N <= 256)
+constexpr int kMaxN = 256;           // MMA N per launch; TMEM holds two accumulators of N columns
+constexpr int kGroup = 128;          // tokens per group of the split-activation modes (1, 3)
 constexpr unsigned long long kUWaitNs = 2000000000ull;
 
 struct alignas(64) UParams {
@@ -44,15 +44,18 @@ struct alignas(64) UParams {
     int K;                // contraction length when known on the host (modes 0, 1, 2)
     int n, d, H, G;
     int splits_fixed;     // mode 0
+    int stages, stage_bytes, tmem_cols;
+    int Gs;               // modes 0, 2: token-group size of the split buffer written (hsplit, asplit)
+    int Gt, Bt, t_base, b_row0, mask_or;   // modes 1, 3: this group's size (hi/lo column offset),
+                                           // valid tokens, first token, first B-operand row, OR mask
     const int32_t* count; // modes 2, 3: table length U (device)
     const int32_t* idx;   // modes 2, 3: neuron table
     const void* bias;     // bp1, bp2, b1 (by neuron), b2
     float* partial;       // [units][kBM][N]
     uint32_t* tickets;    // [tiles]
-    void* out_split;      // mode 0: hsplit [2B][H]; mode 2: asplit [2B][n]
+    void* out_split;      // mode 0: hsplit, mode 2: asplit: [groups][2][Gs][H or n] hi/lo pairs
     float* out_f32;       // mode 0: h [B][H] (may be null); mode 3: y [B][d]
     uint32_t* mask;       // mode 1
-    uint32_t* wcount;     // mode 1
     uint32_t* err;
 };
 
@@ -177,53 +180,52 @@ __device__ __forceinline__ float tof(const void* base, int i) {
     return DT<T>::f(reinterpret_cast<const T*>(base)[i]);
 }
 
-// Final epilogue for one D row (this thread's TMEM lane) and all its columns.
+// Final epilogue for one D row (this thread's TMEM lane) and 16 columns c0..c0+15
+// of each half.  Modes 0 and 2 keep one column per token; modes 1 and 3 hold each
+// token's hi and lo halves Gt columns apart.  Mode 1 ORs its union decision into *any.
 template <typename T>
-__device__ void finish_row(const UParams& p, const Plan& q, int tile, int lane_row, const float* v) {
+__device__ void finish_chunk(const UParams& p, const Plan& q, int tile, int lane_row, int c0, const float* hi,
+                             const float* lo, bool* any)
+{
     const int r = tile * kBM + lane_row;
-    const int B = p.B;
-    if (p.mode == 0) {                      // h = ReLU(D + bp1) -> fp32 and hi/lo pair
+    if (p.mode == 0) {                      // h = ReLU(D + bp1) -> fp32 and its hi/lo pair
         if (r < p.H) {
             const float bias = p.bias ? tof<T>(p.bias, r) : 0.f;
             T* hs = reinterpret_cast<T*>(p.out_split);
-            for (int t = 0; t < B; ++t) {
-                const float h = fmaxf(v[t] + bias, 0.f);
-                const T hi = DT<T>::r(h);
-                const T lo = DT<T>::r(h - DT<T>::f(hi));
-                hs[(size_t)t * p.H + r] = hi;
-                hs[(size_t)(B + t) * p.H + r] = lo;
+            for (int i = 0; i < 16 && c0 + i < p.B; ++i) {
+                const int t = c0 + i, g = t / p.Gs, tt = t - g * p.Gs;
+                const float h = fmaxf(hi[i] + bias, 0.f);
+                const T h1 = DT<T>::r(h);
+                const T h2 = DT<T>::r(h - DT<T>::f(h1));
+                hs[(size_t)(2 * g * p.Gs + tt) * p.H + r] = h1;
+                hs[(size_t)(2 * g * p.Gs + p.Gs + tt) * p.H + r] = h2;
                 if (p.out_f32) p.out_f32[(size_t)t * p.H + r] = h;
             }
         }
-    } else if (p.mode == 1) {               // union decision, 32 rows per mask word
-        bool any = false;
+    } else if (p.mode == 1) {               // union decision over this group's tokens
         if (r < p.n) {
             const float bias = p.bias ? tof<T>(p.bias, r) : 0.f;
-            for (int t = 0; t < B; ++t) any |= (v[t] + v[B + t] + bias) > 0.f;
-        }
-        const uint32_t bits = __ballot_sync(0xffffffffu, any);
-        const int word = (tile * kBM + (lane_row & ~31)) >> 5;
-        if ((threadIdx.x & 31) == 0 && word < (p.n >> 5)) {
-            p.mask[word] = bits;
-            p.wcount[word] = __popc(bits);
+            for (int i = 0; i < 16 && c0 + i < p.Bt; ++i) *any |= (hi[i] + lo[i] + bias) > 0.f;
         }
     } else if (p.mode == 2) {               // a = ReLU(D + b1[j]) for table entry r (zeros past U)
         T* as = reinterpret_cast<T*>(p.out_split);
         if (r < p.n) {
             const bool live = r < q.M;
             const float bias = live ? tof<T>(p.bias, p.idx[r]) : 0.f;
-            for (int t = 0; t < B; ++t) {
-                const float a = live ? fmaxf(v[t] + bias, 0.f) : 0.f;
-                const T hi = DT<T>::r(a);
-                const T lo = DT<T>::r(a - DT<T>::f(hi));
-                as[(size_t)t * p.n + r] = hi;
-                as[(size_t)(B + t) * p.n + r] = lo;
+            for (int i = 0; i < 16 && c0 + i < p.B; ++i) {
+                const int t = c0 + i, g = t / p.Gs, tt = t - g * p.Gs;
+                const float a = live ? fmaxf(hi[i] + bias, 0.f) : 0.f;
+                const T a1 = DT<T>::r(a);
+                const T a2 = DT<T>::r(a - DT<T>::f(a1));
+                as[(size_t)(2 * g * p.Gs + tt) * p.n + r] = a1;
+                as[(size_t)(2 * g * p.Gs + p.Gs + tt) * p.n + r] = a2;
             }
         }
-    } else {                                // y[t][c] = D[c][t] + D[c][B+t] + b2[c]
+    } else {                                // y[t][c] = D[c][t] + D[c][Gt+t] + b2[c]
         if (r < p.d) {
             const float bias = p.bias ? tof<T>(p.bias, r) : 0.f;
-            for (int t = 0; t < B; ++t) p.out_f32[(size_t)t * p.d + r] = v[t] + v[B + t] + bias;
+            for (int i = 0; i < 16 && c0 + i < p.Bt; ++i)
+                p.out_f32[(size_t)(p.t_base + c0 + i) * p.d + r] = hi[i] + lo[i] + bias;
         }
     }
 }
@@ -233,9 +235,10 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
 {
     extern __shared__ __align__(1024) char usm[];
     char* base = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(usm) + 1023) & ~uintptr_t(1023));
+    const int kStages = p.stages, kStageBytes = p.stage_bytes;
     uint64_t* full = reinterpret_cast<uint64_t*>(base + kStages * kStageBytes);
-    uint64_t* empty = full + kStages;
-    uint64_t* tfull = empty + kStages;       // [2]
+    uint64_t* empty = full + kMaxStages;
+    uint64_t* tfull = empty + kMaxStages;    // [2]
     uint64_t* tempty = tfull + 2;            // [2]
     uint64_t* done = tempty + 2;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(done + 1);
@@ -252,7 +255,7 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(s32(tmem_slot)),
-                     "r"(kTmemCols));
+                     "r"(p.tmem_cols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     tc_fence_before();
@@ -312,7 +315,7 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
                     tma_gather4(sa + mb * 8192 + g * 512, &p.tmA, tile * kBM + mb * 64, jc[0], jc[1], jc[2], jc[3],
                                 &full[st]);
                 }
-                if (lane == 0) tma_2d(sb, &p.tmB, kb * kBK, 0, &full[st]);
+                if (lane == 0) tma_2d(sb, &p.tmB, kb * kBK, p.b_row0, &full[st]);
                 if (++st == kStages) { st = 0; ph ^= 1; }
             }
         }
@@ -366,43 +369,72 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
         }
     } else {
         // ------------------------------------------------------------- epilogue (warps 2..5)
+        // The accumulator row is read from TMEM 16 columns at a time (with the matching
+        // lo chunk in modes 1 and 3), so registers do not grow with N.
         const int quad = warp & 3;               // TMEM lanes 32*quad .. 32*quad+31
         const int lane_row = quad * 32 + lane;
         const int et = threadIdx.x - 64;         // 0..127
         volatile int no_abort = 0;
         int ab = 0, aph = 0;
-        float v[64];
+        const bool pair = p.mode == 1 || p.mode == 3;
+        const int half = pair ? p.Gt : N;        // columns of one half, a multiple of 16
         for (int u = blockIdx.x; u < units; u += gridDim.x) {
             const int tile = u / q.splits, sp = u % q.splits;
             const int kb0 = (int)((long long)sp * q.kblocks / q.splits);
             const int kb1 = (int)((long long)(sp + 1) * q.kblocks / q.splits);
-            if (kb1 > kb0) {
+            const bool has = kb1 > kb0;
+            uint32_t taddr = 0;
+            if (has) {
                 // time bound only: all four epilogue warps leave this wait the same way
                 if (!ub_wait(&tfull[ab], aph, &no_abort, p.err)) break;
                 tc_fence_after();
-                const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(ab * N);
+                taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(ab * N);
+            }
+            if (q.splits == 1) {
+                bool any = false;
+                for (int c0 = 0; c0 < half; c0 += 16) {
+                    float hi[16], lo[16];
 #pragma unroll
-                for (int c0 = 0; c0 < 64; c0 += 16)
-                    if (c0 < N) tmem_ld16(taddr + c0, v + c0);
-                tmem_wait_ld();
+                    for (int i = 0; i < 16; ++i) hi[i] = lo[i] = 0.f;
+                    if (has) {
+                        tmem_ld16(taddr + c0, hi);
+                        if (pair) tmem_ld16(taddr + half + c0, lo);
+                        tmem_wait_ld();
+                    }
+                    finish_chunk<T>(p, q, tile, lane_row, c0, hi, lo, &any);
+                }
+                if (p.mode == 1) {                   // one mask word per 32 rows
+                    const uint32_t bits = __ballot_sync(0xffffffffu, any);
+                    const int word = (tile * kBM + (lane_row & ~31)) >> 5;
+                    if (lane == 0 && word < (p.n >> 5)) {
+                        if (p.mask_or) atomicOr(&p.mask[word], bits);
+                        else p.mask[word] = bits;
+                    }
+                }
+            } else {
+                // split-K: publish this split's partial
+                float* mine = p.partial + ((size_t)u * kBM + lane_row) * N;
+                for (int c0 = 0; c0 < N; c0 += 16) {
+                    float v[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = 0.f;
+                    if (has) {
+                        tmem_ld16(taddr + c0, v);
+                        tmem_wait_ld();
+                    }
+#pragma unroll
+                    for (int c = 0; c < 16; c += 4)
+                        __stcg(reinterpret_cast<float4*>(mine + c0 + c), make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]));
+                }
+            }
+            if (has) {
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ub_arrive(&tempty[ab]);
                 if (++ab == 2) { ab = 0; aph ^= 1; }
-            } else {
-#pragma unroll
-                for (int c = 0; c < 64; ++c) v[c] = 0.f;
             }
-            if (q.splits == 1) {
-                finish_row<T>(p, q, tile, lane_row, v);
-                continue;
-            }
-            // split-K: publish this split's partial; the last CTA on the tile reduces in split order
-            float* mine = p.partial + ((size_t)u * kBM + lane_row) * N;
-#pragma unroll
-            for (int c = 0; c < 64; c += 4)
-                if (c < N)
-                    __stcg(reinterpret_cast<float4*>(mine + c), make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]));
+            if (q.splits == 1) continue;
+            // the last CTA on the tile reduces the splits in split order
             __threadfence();
             epi_sync();
             if (et == 0) {
@@ -412,23 +444,30 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
             epi_sync();
             if (*s_last) {
                 __threadfence();
+                bool any = false;
+                for (int c0 = 0; c0 < half; c0 += 16) {
+                    float hi[16], lo[16];
 #pragma unroll
-                for (int c = 0; c < 64; ++c) v[c] = 0.f;
-                // one split at a time, its (up to 16) float4 loads issued together
-                for (int s = 0; s < q.splits; ++s) {
-                    const float4* src = reinterpret_cast<const float4*>(
-                        p.partial + ((size_t)(tile * q.splits + s) * kBM + lane_row) * N);
-                    float4 w[16];
+                    for (int i = 0; i < 16; ++i) hi[i] = lo[i] = 0.f;
+                    for (int s = 0; s < q.splits; ++s) {
+                        const float4* src = reinterpret_cast<const float4*>(
+                            p.partial + ((size_t)(tile * q.splits + s) * kBM + lane_row) * N + c0);
+                        float4 w[8];
 #pragma unroll
-                    for (int c4 = 0; c4 < 16; ++c4)
-                        w[c4] = c4 * 4 < N ? __ldcg(src + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+                        for (int c4 = 0; c4 < 4; ++c4) {
+                            w[c4] = __ldcg(src + c4);
+                            w[4 + c4] = pair ? __ldcg(src + half / 4 + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+                        }
 #pragma unroll
-                    for (int c4 = 0; c4 < 16; ++c4) {
-                        v[4 * c4] += w[c4].x; v[4 * c4 + 1] += w[c4].y;
-                        v[4 * c4 + 2] += w[c4].z; v[4 * c4 + 3] += w[c4].w;
+                        for (int c4 = 0; c4 < 4; ++c4) {
+                            hi[4 * c4] += w[c4].x; hi[4 * c4 + 1] += w[c4].y;
+                            hi[4 * c4 + 2] += w[c4].z; hi[4 * c4 + 3] += w[c4].w;
+                            lo[4 * c4] += w[4 + c4].x; lo[4 * c4 + 1] += w[4 + c4].y;
+                            lo[4 * c4 + 2] += w[4 + c4].z; lo[4 * c4 + 3] += w[4 + c4].w;
+                        }
                     }
+                    finish_chunk<T>(p, q, tile, lane_row, c0, hi, lo, &any);
                 }
-                finish_row<T>(p, q, tile, lane_row, v);
                 if (et == 0) p.tickets[tile] = 0u;     // ready for the next call
             }
             epi_sync();
@@ -439,7 +478,7 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(p.tmem_cols));
     }
 }
 
@@ -478,10 +517,19 @@ bool make_map(CUtensorMap* m, const void* ptr, int dtype, int64_t rows, int64_t 
 
 int round16(int v) { return (v + 15) / 16 * 16; }
 
-size_t smem_bytes() { return (size_t)kStages * kStageBytes + 1024 + 256; }
+// stage ring and TMEM allocation for an MMA of N columns
+void size_launch(UParams& p) {
+    p.stage_bytes = 16384 + p.N * 128;
+    p.stages = std::min(kMaxStages, (200 * 1024) / p.stage_bytes);
+    int cols = 32;
+    while (cols < 2 * p.N) cols *= 2;
+    p.tmem_cols = cols;
+}
 
-cudaError_t launch(const UParams& p, int grid, cudaStream_t st) {
-    const size_t smem = smem_bytes();
+cudaError_t launch(UParams& p, int grid, cudaStream_t st) {
+    size_launch(p);
+    if (p.N > kMaxN || p.stages < 2) return cudaErrorInvalidValue;
+    const size_t smem = (size_t)p.stages * p.stage_bytes + 1024 + 256;
     cudaError_t e;
     if (p.dtype == SPFFN_BF16) {
         e = cudaFuncSetAttribute(k_umma<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -510,8 +558,18 @@ UParams base_params(const spffn_ctx& c, int B) {
 
 }  // namespace
 
+// Token groups of the split-activation modes: B tokens in ceil(B / 128) groups of
+// Gt tokens (a multiple of 16); group g's hi rows start at 2 g Gt, its lo rows at
+// 2 g Gt + Gt, so one B-operand box of 2 Gt rows covers a group.
+UnionGroups union_groups(int B) {
+    UnionGroups u;
+    u.groups = (B + kGroup - 1) / kGroup;
+    u.Gt = round16((B + u.groups - 1) / u.groups);
+    return u;
+}
+
 bool union_supported(const spffn_ctx& c, int B) {
-    return B >= 16 && B <= 32 && c.cfg.d % 128 == 0 && c.cfg.max_batch >= 16 && c.lay.upartial != 0 &&
+    return B >= 16 && B <= kMaxBatch && B <= c.cfg.max_batch && c.cfg.d % 128 == 0 && c.lay.upartial != 0 &&
            c.num_sms <= kMaxUnionCtas && encoder() != nullptr;
 }
 
@@ -519,12 +577,14 @@ cudaError_t union_predict(const spffn_ctx& c, const void* x, int B, int32_t* idx
                           cudaStream_t st)
 {
     const auto& g = c.cfg;
-    // predictor layer 1: D[H x B] = Wp1 . X^T, split-K, -> h (fp32) and its hi/lo pair
+    const UnionGroups ug = union_groups(B);
+    // predictor layer 1: D[H x B] = Wp1 . X^T, split-K, -> h (fp32) and its hi/lo pairs
     UParams p = base_params(c, B);
     p.mode = 0;
     p.N = round16(B);
     p.M = g.H;
     p.K = g.d;
+    p.Gs = ug.Gt;
     const int tiles = (g.H + kBM - 1) / kBM;
     const int kblocks = g.d / kBK;
     p.splits_fixed = std::max(1, std::min(kblocks, c.num_sms / tiles));
@@ -535,19 +595,24 @@ cudaError_t union_predict(const spffn_ctx& c, const void* x, int B, int32_t* idx
     if (!make_map(&p.tmB, x, g.dtype, B, g.d, p.N)) return cudaErrorInvalidValue;
     cudaError_t e = launch(p, c.num_sms, st);
     if (e != cudaSuccess) return e;
-    // predictor layer 2: D[n x 2B] = Wp2 . hsplit^T -> union mask words
-    UParams q = base_params(c, B);
-    q.mode = 1;
-    q.N = round16(2 * B);
-    q.M = g.n;
-    q.K = g.H;
-    q.bias = c.w.bp2;
-    q.mask = c.mask();
-    q.wcount = c.wcount();
-    if (!make_map(&q.tmA, c.w.Wp2, g.dtype, g.n, g.H, kBM)) return cudaErrorInvalidValue;
-    if (!make_map(&q.tmB, c.hsplit(), g.dtype, 2 * B, g.H, q.N)) return cudaErrorInvalidValue;
-    e = launch(q, c.num_sms, st);
-    if (e != cudaSuccess) return e;
+    // predictor layer 2, one token group at a time: D[n x 2Gt] = Wp2 . hsplit_g^T -> union mask words
+    for (int gi = 0; gi < ug.groups; ++gi) {
+        UParams q = base_params(c, B);
+        q.mode = 1;
+        q.N = 2 * ug.Gt;
+        q.M = g.n;
+        q.K = g.H;
+        q.Gt = ug.Gt;
+        q.Bt = std::min(ug.Gt, B - gi * ug.Gt);
+        q.b_row0 = 2 * gi * ug.Gt;
+        q.mask_or = gi > 0;
+        q.bias = c.w.bp2;
+        q.mask = c.mask();
+        if (!make_map(&q.tmA, c.w.Wp2, g.dtype, g.n, g.H, kBM)) return cudaErrorInvalidValue;
+        if (!make_map(&q.tmB, c.hsplit(), g.dtype, 2 * ug.groups * ug.Gt, g.H, q.N)) return cudaErrorInvalidValue;
+        e = launch(q, c.num_sms, st);
+        if (e != cudaSuccess) return e;
+    }
     return launch_compact(c, idx, count, count2, st);
 }
 
@@ -555,11 +620,13 @@ cudaError_t union_forward(const spffn_ctx& c, const void* x, int B, const int32_
                           float* y, cudaStream_t st)
 {
     const auto& g = c.cfg;
-    // FC1 over the table rows: D[U x B] = W1[table] . X^T -> a (hi/lo pair), zeros past U
+    const UnionGroups ug = union_groups(B);
+    // FC1 over the table rows: D[U x B] = W1[table] . X^T -> a (hi/lo pairs), zeros past U
     UParams p = base_params(c, B);
     p.mode = 2;
     p.N = round16(B);
     p.K = g.d;
+    p.Gs = ug.Gt;
     p.count = count;
     p.idx = idx;
     p.bias = c.w.b1;
@@ -568,18 +635,26 @@ cudaError_t union_forward(const spffn_ctx& c, const void* x, int B, const int32_
     if (!make_map(&p.tmB, x, g.dtype, B, g.d, p.N)) return cudaErrorInvalidValue;
     cudaError_t e = launch(p, c.num_sms, st);
     if (e != cudaSuccess) return e;
-    // FC2: D[d x 2B] = W2T[table]^T . asplit^T -> y
-    UParams q = base_params(c, B);
-    q.mode = 3;
-    q.N = round16(2 * B);
-    q.M = g.d;
-    q.count = count;
-    q.idx = idx;
-    q.bias = c.w.b2;
-    q.out_f32 = y;
-    if (!make_map(&q.tmA, c.w.W2T, g.dtype, g.n, g.d, 1)) return cudaErrorInvalidValue;
-    if (!make_map(&q.tmB, c.asplit(), g.dtype, 2 * B, g.n, q.N)) return cudaErrorInvalidValue;
-    return launch(q, c.num_sms, st);
+    // FC2, one token group at a time: D[d x 2Gt] = W2T[table]^T . asplit_g^T -> y
+    for (int gi = 0; gi < ug.groups; ++gi) {
+        UParams q = base_params(c, B);
+        q.mode = 3;
+        q.N = 2 * ug.Gt;
+        q.M = g.d;
+        q.Gt = ug.Gt;
+        q.Bt = std::min(ug.Gt, B - gi * ug.Gt);
+        q.t_base = gi * ug.Gt;
+        q.b_row0 = 2 * gi * ug.Gt;
+        q.count = count;
+        q.idx = idx;
+        q.bias = c.w.b2;
+        q.out_f32 = y;
+        if (!make_map(&q.tmA, c.w.W2T, g.dtype, g.n, g.d, 1)) return cudaErrorInvalidValue;
+        if (!make_map(&q.tmB, c.asplit(), g.dtype, 2 * ug.groups * ug.Gt, g.n, q.N)) return cudaErrorInvalidValue;
+        e = launch(q, c.num_sms, st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace spffn

@@ -3,6 +3,10 @@
 #include "spffn_internal.cuh"
 
 namespace spffn {
+struct UnionGroups {
+    int groups, Gt;   // token groups of the split-activation modes, tokens per group (multiple of 16)
+};
+UnionGroups union_groups(int B);
 bool union_supported(const spffn_ctx& c, int B);
 cudaError_t union_predict(const spffn_ctx& c, const void* x, int B, int32_t* idx, int32_t* count, int32_t* count2,
                           cudaStream_t st);

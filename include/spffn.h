@@ -62,7 +62,9 @@ typedef enum { SPFFN_F16 = 0, SPFFN_BF16 = 1 } spffn_dtype;
  *   d          model width; d % 64 == 0, 64 <= d <= 16384
  *   n          FFN neurons;  n % 32 == 0, 32 <= n <= 131072
  *   H          predictor hidden width; H % 64 == 0, 64 <= H <= 8192
- *   max_batch  largest batch B the context will see; 1 <= max_batch <= 32
+ *   max_batch  largest batch B the context will see; 1 <= max_batch <= 256.  Batches
+ *              of 16..256 tokens run on the union tensor-core path, which needs
+ *              d % 128 == 0; without it a batch above 32 is SPFFN_ERR_UNSUPPORTED
  *   dtype      storage type of weights and of x (accumulation is always fp32)
  *   flags      0 (reserved) */
 typedef struct {
@@ -108,7 +110,8 @@ spffn_status spffn_destroy(spffn_ctx* ctx);
  *   l_t,i = Wp2[i] . h_t + bp2_i                 (fp32)
  *   neuron i selected  <=>  l_t,i > 0 for some token t  (sigmoid > 0.5)
  *   idx[0..count) = selected neurons, ascending; *count written on device.
- * x: device [B][d] storage dtype; 1 <= B <= max_batch.
+ * x: device [B][d] storage dtype; 1 <= B <= max_batch (B > 32 only on the union
+ * path, see spffn_config; else SPFFN_ERR_UNSUPPORTED).
  * idx: device int32, capacity n.  count: device int32 scalar. */
 spffn_status spffn_predict(spffn_ctx* ctx, const void* x, int32_t B,
                            int32_t* idx, int32_t* count, void* stream);
@@ -165,8 +168,9 @@ spffn_status spffn_decode_lookahead(spffn_ctx* const* layers, int32_t L, const v
 spffn_status spffn_layer_table(spffn_ctx* ctx, const int32_t** idx);
 
 /* Number of kernels one spffn_decode (or spffn_decode_lookahead) call with these
- * arguments enqueues (the persistent whole-stack kernel: 1; otherwise 6 per
- * layer), 0 on bad arguments.
+ * arguments enqueues (the persistent whole-stack kernel: 1; otherwise per layer
+ * 4 + 2 x the union path's token groups, ceil(B / 128), or 6 off that path), 0 on
+ * bad arguments.
  * Pure host function. */
 int32_t spffn_decode_kernel_launches(spffn_ctx* const* layers, int32_t L, int32_t B);
 

@@ -48,8 +48,9 @@ def test_workspace_bytes_validation():
     ok = sp.workspace_bytes(4096, 16384, 1024, 1)
     assert ok > 16384 // 32 * 4 + 1024 * 4
     assert sp.workspace_bytes(4096, 16384, 1024, 32) > ok
+    assert sp.workspace_bytes(4096, 16384, 1024, 256) > sp.workspace_bytes(4096, 16384, 1024, 32)
     for bad in [(4000, 16384, 1024, 1), (4096, 16383, 1024, 1), (4096, 16384, 1000, 1),
-                (4096, 16384, 1024, 0), (4096, 16384, 1024, 33), (32, 64, 64, 1)]:
+                (4096, 16384, 1024, 0), (4096, 16384, 1024, 257), (32, 64, 64, 1)]:
         assert sp.workspace_bytes(*bad) == 0, bad
     assert sp.workspace_bytes(4096, 16384, 1024, 1, dtype=2) == 0
 

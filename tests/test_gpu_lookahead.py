@@ -3,7 +3,7 @@
 against the oracle chaining its own layer inputs: every layer's neuron table
 (bit-exact outside the near-threshold band) and count, the last layer's y and
 the final x.  Covers the persistent kernel (B <= 2), the per-layer path (B = 3)
-and the union tensor-core path (B = 16)."""
+and the union tensor-core path (B = 16, 64 and 200)."""
 import numpy as np
 import pytest
 
@@ -76,9 +76,10 @@ def test_decode_tables_match_oracle(name, B, lookahead):
     run_and_check(cfg, Lc, B, aux=500 + B, lookahead=lookahead)
 
 
+@pytest.mark.parametrize("B", [16, 64, 200])
 @pytest.mark.parametrize("lookahead", [False, True])
-def test_union_decode_tables_match_oracle(lookahead):
-    run_and_check(wl.CONFIGS[0], 3, 16, aux=516, lookahead=lookahead, max_batch=16)
+def test_union_decode_tables_match_oracle(lookahead, B):
+    run_and_check(wl.CONFIGS[0], 3, B, aux=516 + B, lookahead=lookahead, max_batch=B)
 
 
 def test_lookahead_changes_the_sets():

@@ -13,11 +13,14 @@
 // dtype (v ~= hi + lo, hi = round(v), lo = round(v - hi)); the epilogue adds the
 // two column halves of D.  X is already in the storage dtype (exact).
 //
-// One persistent CTA per SM; warp 0 issues TMA loads into a 6-stage ring
-// (2-D tiles for contiguous operands, tile::gather4 for the rows named by the
-// neuron table; never multicast), warp 1 issues tcgen05.mma into a double
-// buffered TMEM accumulator, warps 2..5 read TMEM (tcgen05.ld) and run the
-// epilogue.  Split-K partials are summed in fixed split order by the last CTA
+// One persistent CTA per SM; warp 0 issues TMA loads into a ring of 4..6 stages
+// (2-D tiles for the contiguous operands, tile::gather4 for FC2's table rows; never
+// multicast), warps 6..9 gather FC1's table rows with coalesced 16-byte cp.async
+// into the same 128-byte swizzled image (each thread fences its landed copies into
+// the async proxy before it arrives; twice the rate of gather4 for these 128-byte
+// row pieces, while FC2's 256-byte pieces go faster through gather4), warp 1
+// issues tcgen05.mma into a double buffered TMEM accumulator, warps 2..5 read TMEM
+// (tcgen05.ld) and run the epilogue.  Split-K partials are summed in fixed split order by the last CTA
 // to finish a tile (atomic ticket, no waiting), so results are deterministic.
 #include <cuda.h>
 #include <algorithm>
@@ -28,7 +31,8 @@
 namespace spffn {
 namespace {
 
-constexpr int kUThreads = 192;       // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kUThreads = 320;       // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue, 6..9 row gathers
+constexpr int kGatherThreads = 128;
 constexpr int kBM = 128;             // D rows per tile
 constexpr int kBK = 64;              // K per stage: one 128-byte swizzle row of 16-bit elements
 constexpr int kMaxStages = 6;       // stage = A tile 16 KB + B tile N x 128 B (N <= 256)
@@ -50,6 +54,7 @@ struct alignas(64) UParams {
                                            // valid tokens, first token, first B-operand row, OR mask
     const int32_t* count; // modes 2, 3: table length U (device)
     const int32_t* idx;   // modes 2, 3: neuron table
+    const void* W;        // mode 2: W1, rows gathered by the table
     const void* bias;     // bp1, bp2, b1 (by neuron), b2
     float* partial;       // [units][kBM][N]
     uint32_t* tickets;    // [tiles]
@@ -110,6 +115,16 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, i
         " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
         ::"r"(s32(dst)), "l"(map), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(s32(bar)) : "memory");
 }
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// make this thread's completed generic-proxy writes to shared memory visible to the
+// tensor cores (async proxy) before it signals them
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 // shared-memory matrix descriptor, 128-byte swizzle
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo16, uint32_t sbo16) {
     return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)lbo16 << 16) | ((uint64_t)sbo16 << 32) |
@@ -210,8 +225,9 @@ __device__ void finish_chunk(const UParams& p, const Plan& q, int tile, int lane
     } else if (p.mode == 2) {               // a = ReLU(D + b1[j]) for table entry r (zeros past U)
         T* as = reinterpret_cast<T*>(p.out_split);
         if (r < p.n) {
-            const bool live = r < q.M;
-            const float bias = live ? tof<T>(p.bias, p.idx[r]) : 0.f;
+            const int j = r < q.M ? p.idx[r] : -1;
+            const bool live = (unsigned)j < (unsigned)p.n;     // past U or out of range: zero
+            const float bias = live ? tof<T>(p.bias, j) : 0.f;
             for (int i = 0; i < 16 && c0 + i < p.B; ++i) {
                 const int t = c0 + i, g = t / p.Gs, tt = t - g * p.Gs;
                 const float a = live ? fmaxf(hi[i] + bias, 0.f) : 0.f;
@@ -247,7 +263,9 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kStages; ++i) { ub_init(&full[i], 1); ub_init(&empty[i], 1); }
+        // mode 2: the TMA warp's B tile plus one arrival per gathering thread
+        const uint32_t fc = (p.mode == 2) ? 1u + kGatherThreads : 1u;
+        for (int i = 0; i < kStages; ++i) { ub_init(&full[i], fc); ub_init(&empty[i], 1); }
         for (int i = 0; i < 2; ++i) { ub_init(&tfull[i], 1); ub_init(&tempty[i], 4); }
         ub_init(done, 1);
         *abort_flag = 0;
@@ -263,54 +281,51 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const Plan q = make_plan(p);
+    if (p.mode == 2 && blockIdx.x == 0 && threadIdx.x == 0) {
+        const int U = *p.count;
+        if (U < 0 || U > p.n) atomicOr(p.err, ERR_COUNT_CLAMPED);    // clamped by make_plan
+    }
     const int units = q.tiles * q.splits;
     const int N = p.N;
     const uint32_t btile_bytes = (uint32_t)N * 128u;
 
     if (warp == 0) {
         // ------------------------------------------------------------- TMA producer (whole warp)
+        // modes 0, 1: A and B tiles (2-D); mode 2: the B tile only (the gather warps copy
+        // the A rows); mode 3: the B tile and the K block's 64 table rows of W2T, which
+        // lane l fetches with tile::gather4 (rows 4(l%16)..+3, 64-column block l/16)
         int st = 0, ph = 0;
         for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
             const int tile = u / q.splits, sp = u % q.splits;
             const int kb0 = (int)((long long)sp * q.kblocks / q.splits);
             const int kb1 = (int)((long long)(sp + 1) * q.kblocks / q.splits);
-            int jr[4] = {0, 0, 0, 0};           // FC1: this lane's 4 table rows of the tile
-            if (p.mode == 2) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int r = tile * kBM + lane * 4 + i;
-                    jr[i] = p.idx[r < q.M ? r : 0];
-                }
-            }
-            // mode 3: this lane's 4 table rows of the K block, one block ahead
+            // mode 3: this lane's 4 table rows of a K block (entries outside [0, n) read row 0;
+            // FC1 latched them and gave them activation zero), one block ahead
             auto k_rows = [&](int kb, int* j) {
                 const int g = lane & 15;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int r = kb * kBK + g * 4 + i;
-                    j[i] = p.idx[r < q.K ? r : 0];
+                    const int e = p.idx[r < q.K ? r : 0];
+                    j[i] = (unsigned)e < (unsigned)p.n ? e : 0;
                 }
             };
             int jn[4] = {0, 0, 0, 0};
             if (p.mode == 3 && kb0 < kb1) k_rows(kb0, jn);
+            bool okw = true;
             for (int kb = kb0; kb < kb1; ++kb) {
                 int jc[4] = {jn[0], jn[1], jn[2], jn[3]};
                 if (p.mode == 3 && kb + 1 < kb1) k_rows(kb + 1, jn);
-                bool okw = true;
                 if (lane == 0) okw = ub_wait(&empty[st], ph ^ 1, abort_flag, p.err);
                 okw = __shfl_sync(0xffffffffu, okw, 0);
                 if (!okw) break;
                 char* sa = base + st * kStageBytes;
                 char* sb = sa + 16384;
-                if (lane == 0) ub_expect(&full[st], 16384u + btile_bytes);
+                if (lane == 0) ub_expect(&full[st], (p.mode == 2 ? 0u : 16384u) + btile_bytes);
                 __syncwarp();
                 if (p.mode <= 1) {
                     if (lane == 0) tma_2d(sa, &p.tmA, kb * kBK, tile * kBM, &full[st]);
-                } else if (p.mode == 2) {
-                    // 128 table rows of W1: lane l gathers rows 4l..4l+3 of this tile
-                    tma_gather4(sa + lane * 512, &p.tmA, kb * kBK, jr[0], jr[1], jr[2], jr[3], &full[st]);
-                } else {
-                    // 64 table rows (the K block) x 128 columns of W2T, as two 64-column blocks
+                } else if (p.mode == 3) {
                     const int mb = lane >> 4, g = lane & 15;
                     tma_gather4(sa + mb * 8192 + g * 512, &p.tmA, tile * kBM + mb * 64, jc[0], jc[1], jc[2], jc[3],
                                 &full[st]);
@@ -318,11 +333,67 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
                 if (lane == 0) tma_2d(sb, &p.tmB, kb * kBK, p.b_row0, &full[st]);
                 if (++st == kStages) { st = 0; ph ^= 1; }
             }
+            if (!okw) break;
         }
         // on abort, give copies already issued time to land before the CTA retires
         if (lane == 0 && *abort_flag) {
             const unsigned long long t0 = now_ns();
             while (now_ns() - t0 < 200000ull) {}
+        }
+    } else if (warp >= 6) {
+        // ------------------------------------------------------------- row gathers (mode 2)
+        // 128 threads copy the stage's 128 table rows of W1 (128 bytes each) with 16-byte
+        // cp.async into the same 128-byte swizzled image a TMA tile would leave (16-byte
+        // chunk c of row r at r*128 + ((c ^ (r & 7)) << 4)); eight consecutive lanes cover
+        // one row.  Each thread commits one group per stage and, kLag - 1 stages later, once
+        // that group has landed, fences it into the async proxy and arrives on the stage's
+        // full barrier.
+        if (p.mode == 2) {
+            constexpr int kLag = 4;                      // stages in flight per thread (kStages >= 4)
+            const int t = threadIdx.x - 6 * 32;          // 0..127
+            const int c = t & 7;
+            int st = 0, ph = 0, lag_st[kLag] = {0, 0, 0, 0}, nlag = 0;
+            bool okg = true;
+            for (int u = blockIdx.x; u < units && okg; u += gridDim.x) {
+                const int tile = u / q.splits, sp = u % q.splits;
+                const int kb0 = (int)((long long)sp * q.kblocks / q.splits);
+                const int kb1 = (int)((long long)(sp + 1) * q.kblocks / q.splits);
+                // rows 16 i + t / 8 of the tile; a table entry outside [0, n) is latched and read
+                // as row 0 (its activation is zero)
+                const char* rows[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = tile * kBM + i * 16 + (t >> 3);
+                    int j = p.idx[r < q.M ? r : 0];
+                    if ((unsigned)j >= (unsigned)p.n) { atomicOr(p.err, ERR_IDX_RANGE); j = 0; }
+                    rows[i] = reinterpret_cast<const char*>(p.W) + (size_t)j * p.d * 2 + c * 16;
+                }
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!ub_wait(&empty[st], ph ^ 1, abort_flag, p.err)) { okg = false; break; }
+                    char* sa = base + st * kStageBytes;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int r = i * 16 + (t >> 3);
+                        cp_async16(sa + r * 128 + ((c ^ (r & 7)) << 4), rows[i] + (size_t)kb * kBK * 2);
+                    }
+                    cp_async_commit();
+                    lag_st[nlag++] = st;
+                    if (nlag == kLag) {
+                        // all but the newest kLag - 1 groups have landed: signal the oldest stage
+                        cp_async_wait<kLag - 1>();
+                        fence_async_smem();
+                        ub_arrive(&full[lag_st[0]]);
+#pragma unroll
+                        for (int i = 0; i + 1 < kLag; ++i) lag_st[i] = lag_st[i + 1];
+                        nlag = kLag - 1;
+                    }
+                    if (++st == kStages) { st = 0; ph ^= 1; }
+                }
+            }
+            // land and signal what is still in flight
+            cp_async_wait<0>();
+            fence_async_smem();
+            for (int i = 0; i < nlag; ++i) ub_arrive(&full[lag_st[i]]);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------- MMA issuer (one thread)
@@ -367,7 +438,7 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
                 while (!ub_try(done, 0) && now_ns() - t0 < kUWaitNs) {}
             }
         }
-    } else {
+    } else if (warp >= 2 && warp <= 5) {
         // ------------------------------------------------------------- epilogue (warps 2..5)
         // The accumulator row is read from TMEM 16 columns at a time (with the matching
         // lo chunk in modes 1 and 3), so registers do not grow with N.
@@ -631,7 +702,7 @@ cudaError_t union_forward(const spffn_ctx& c, const void* x, int B, const int32_
     p.idx = idx;
     p.bias = c.w.b1;
     p.out_split = c.asplit();
-    if (!make_map(&p.tmA, c.w.W1, g.dtype, g.n, g.d, 1)) return cudaErrorInvalidValue;
+    p.W = c.w.W1;
     if (!make_map(&p.tmB, x, g.dtype, B, g.d, p.N)) return cudaErrorInvalidValue;
     cudaError_t e = launch(p, c.num_sms, st);
     if (e != cudaSuccess) return e;

@@ -100,3 +100,32 @@ def test_batch_above_32_needs_the_union_path():
     L.predict(wl.to_torch(wl.tokens(cfg, 32, aux=2), cfg), idx, cnt)
     torch.cuda.synchronize()
     assert L.last_device_error() == (sp.OK, 0)
+
+
+def _mixed_tables(n, seed):
+    r = np.random.default_rng(seed)
+    dense = np.arange(256, 512)                                          # two full blocks
+    edge = 1024 + np.sort(r.choice(128, 64, replace=False))             # a block exactly half full
+    below = 1280 + np.sort(r.choice(128, 63, replace=False))            # one member short of dense
+    sparse = np.sort(r.choice(np.arange(2048, n), 300, replace=False))
+    tab = np.concatenate([dense, edge, below, sparse])
+    shuffled = r.permutation(tab)
+    return tab, shuffled
+
+
+@pytest.mark.parametrize("B", [16, 64])
+def test_union_forward_dense_and_sparse_blocks(B):
+    # tables mixing full, half-full and sparse 128-neuron blocks, in ascending and in
+    # shuffled order (a table is a set): dense blocks load as 2-D tiles, the rest gathered
+    cfg, h, OL, T, L = setup("f16-d1024-n4096-H256")
+    xb, x64 = x_tokens(cfg, B, aux=900 + B)
+    x = wl.to_torch(xb, cfg)
+    tab, shuffled = _mixed_tables(cfg.n, B)
+    y_or = O.sparse_ffn(OL["W1"], OL["b1"], OL["W2T"], OL["b2"], x64, np.sort(tab))
+    for t in (tab, shuffled):
+        idx = torch.from_numpy(np.ascontiguousarray(t, dtype=np.int32)).cuda()
+        cnt = torch.tensor([len(t)], dtype=torch.int32, device="cuda")
+        y = torch.empty(B, cfg.d, dtype=torch.float32, device="cuda")
+        L.forward(x, idx, cnt, y)
+        assert rel_l2(y.cpu().numpy(), y_or) <= REL_L2_BAR
+    assert L.last_device_error() == (sp.OK, 0)

@@ -83,3 +83,30 @@ def test_union_is_deterministic():
         outs.append((y.cpu(), idx[:k].cpu(), cnt.cpu()))   # entries past the count are not written
     for o in outs[1:]:
         assert all(torch.equal(a, b) for a, b in zip(outs[0], o))
+
+
+def test_union_edge_cases_empty_clamped_and_out_of_range():
+    cfg, h, OL, T, L = setup("f16-d1024-n4096-H256", 16)
+    xb, x64 = x_tokens(cfg, 16, aux=31)
+    x = wl.to_torch(xb, cfg)
+    y = torch.empty(16, cfg.d, dtype=torch.float32, device="cuda")
+    idx = torch.arange(cfg.n, dtype=torch.int32, device="cuda")
+    L.last_device_error()
+    # empty table: y = b2 (zero here), no error
+    L.forward(x, idx, torch.tensor([0], dtype=torch.int32, device="cuda"), y)
+    assert torch.count_nonzero(y).item() == 0
+    assert L.last_device_error() == (sp.OK, 0)
+    # count > n: clamped to n (the dense FFN), latched
+    L.forward(x, idx, torch.tensor([cfg.n + 9], dtype=torch.int32, device="cuda"), y)
+    yd = O.dense_ffn(OL["W1"], OL["b1"], OL["W2T"], OL["b2"], x64)
+    assert rel_l2(y.cpu().numpy(), yd) <= REL_L2_BAR
+    s, code = L.last_device_error()
+    assert s == sp.ERR_DEVICE_CHECK and code & 1
+    # out-of-range entries are skipped and latched
+    bad = torch.tensor([3, cfg.n + 4, 7, -1, 9], dtype=torch.int32, device="cuda")
+    L.forward(x, bad, torch.tensor([5], dtype=torch.int32, device="cuda"), y)
+    y_or = O.sparse_ffn(OL["W1"], OL["b1"], OL["W2T"], OL["b2"], x64, [3, 7, 9])
+    assert rel_l2(y.cpu().numpy(), y_or) <= REL_L2_BAR
+    s, code = L.last_device_error()
+    assert s == sp.ERR_DEVICE_CHECK and code & 2
+    assert L.last_device_error() == (sp.OK, 0)

@@ -131,7 +131,8 @@ struct Shared {
     float* bias1;            // [max_rows_h] bp1 for the CTA's Wp1 rows
     float* bias2;            // [max_rows]   bp2 for the CTA's Wp2 rows
     float* biasy;            // [max_cols]   b2 for the CTA's output columns
-    float* red;              // [2][8][2][NB] FC1 partial dots of a neuron pair, by pair parity
+    float* red;              // FC1 partial dots: [2][4][8] for neuron quads (B = 1), then
+                             // [2][8][2][NB] for pairs, each by step parity
     float* red2;             // [8][NB]
     float* red1;             // [32][8][NB] GEMV1 row partials per warp
     float* misc;             // [16]
@@ -313,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         S.bias1 = reinterpret_cast<float*>(q); q += ((size_t)(H / G + 2) * 4 + 127) / 128 * 128;
         S.bias2 = reinterpret_cast<float*>(q); q += ((size_t)p.max_rows * 4 + 127) / 128 * 128;
         S.biasy = reinterpret_cast<float*>(q); q += ((size_t)(d / G + 8) * 4 + 127) / 128 * 128;
-        S.red = reinterpret_cast<float*>(q); q += 2 * 8 * 2 * NB * 4;
+        S.red = reinterpret_cast<float*>(q); q += (2 * 4 * 8 + 2 * 8 * 2 * NB) * 4;
         S.red2 = reinterpret_cast<float*>(q); q += 8 * NB * 4;
         S.red1 = reinterpret_cast<float*>(q); q += 32 * 8 * NB * 4;
         S.misc = reinterpret_cast<float*>(q); q += 16 * 4;
@@ -749,8 +750,71 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
             for (int q = 0; q < 4; ++q)
 #pragma unroll
                 for (int t = 0; t < NB; ++t) acc[a][q][t] = 0ull;
-        // neurons two at a time: one shared-memory reduction per pair
-        for (int i = 0; i < m; i += 2, fk += 2) {
+        int i = 0;
+        if constexpr (NB == 1) {
+            // four neurons per step while four remain (one shared-memory reduction per quad;
+            // four independent dot chains hide more latency than two)
+            float* redq = S.red;
+            if (p.ffn_slots >= 4) {
+                for (; i + 4 <= m; i += 4, fk += 4) {
+                    const char* sl[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        if (!cwait(S, p, &S.ffull[(fk + u) % p.ffn_slots], ((fk + u) / p.ffn_slots) & 1)) return false;
+                        sl[u] = S.fring + (size_t)((fk + u) % p.ffn_slots) * fslot_bytes;
+                    }
+                    if (i == 0) TRACE(7);
+                    float part[4][4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) part[u][0] = part[u][1] = part[u][2] = part[u][3] = 0.f;
+#pragma unroll
+                    for (int a = 0; a < kMaxVPT; ++a) {
+                        const int v = tid + a * kConsumers;
+                        if (v < nvec) {
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) dot_mix<T>(part[u], reinterpret_cast<const uint4*>(sl[u])[v], xr[a][0]);
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float v = warp_sum(sum4(part[u]));
+                        if (lane == 0) redq[(rpar * 4 + u) * 8 + warp] = v;
+                    }
+                    consumer_sync();
+                    u64 av[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float4* rp = reinterpret_cast<const float4*>(redq + (rpar * 4 + u) * 8);
+                        const float4 r0 = rp[0], r1 = rp[1];
+                        const float z = ((r0.x + r0.y) + (r0.z + r0.w)) + ((r1.x + r1.y) + (r1.z + r1.w));
+                        const float bias = DT<T>::f(reinterpret_cast<const T*>(sl[u] + 4 * d)[nl[i + u] & 7]);
+                        const float a = fmaxf(z + bias, 0.f);
+                        av[u] = pk(a, a);
+                    }
+                    rpar ^= 1;
+#pragma unroll
+                    for (int a = 0; a < kMaxVPT; ++a) {
+                        const int v = tid + a * kConsumers;
+                        if (v < nvec) {
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const uint4 w = reinterpret_cast<const uint4*>(sl[u] + 2 * d)[v];
+                                ffma2(acc[a][0][0], av[u], Arith<T>::widen2(w.x));
+                                ffma2(acc[a][1][0], av[u], Arith<T>::widen2(w.y));
+                                ffma2(acc[a][2][0], av[u], Arith<T>::widen2(w.z));
+                                ffma2(acc[a][3][0], av[u], Arith<T>::widen2(w.w));
+                            }
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0)
+                        for (int u = 0; u < 4; ++u) mbar_arrive(&S.fempty[(fk + u) % p.ffn_slots]);
+                }
+            }
+        }
+        float* redp = S.red + 2 * 4 * 8;
+        // the rest two at a time: one shared-memory reduction per pair
+        for (; i < m; i += 2, fk += 2) {
             const bool two = i + 1 < m;
             const int s0 = fk % p.ffn_slots, s1 = (fk + 1) % p.ffn_slots;
             if (!cwait(S, p, &S.ffull[s0], (fk / p.ffn_slots) & 1)) return false;
@@ -781,7 +845,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
 #pragma unroll
                 for (int t = 0; t < NB; ++t) {
                     const float v = warp_sum(sum4(part[u][t]));
-                    if (lane == 0) S.red[((rpar * 8 + warp) * 2 + u) * NB + t] = v;
+                    if (lane == 0) redp[((rpar * 8 + warp) * 2 + u) * NB + t] = v;
                 }
             consumer_sync();
             u64 av[2][NB];
@@ -794,7 +858,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
                 for (int t = 0; t < NB; ++t) {
                     float z = 0.f;
 #pragma unroll
-                    for (int q = 0; q < kConsumerWarps; ++q) z += S.red[((rpar * 8 + q) * 2 + u) * NB + t];
+                    for (int q = 0; q < kConsumerWarps; ++q) z += redp[((rpar * 8 + q) * 2 + u) * NB + t];
                     float a = fmaxf(z + bias, 0.f);
                     if (u == 1 && !two) a = 0.f;
                     av[u][t] = pk(a, a);
@@ -1028,7 +1092,7 @@ Geometry geometry(const spffn_config& c, int G, bool lookahead) {
     fixed += ((size_t)(c.H / G + 2) * 4 + 127) / 128 * 128;          // bias1
     fixed += ((size_t)g.max_rows * 4 + 127) / 128 * 128;             // bias2
     fixed += ((size_t)(c.d / G + 8) * 4 + 127) / 128 * 128;          // biasy
-    fixed += 2 * 8 * 2 * NB * 4 + 8 * NB * 4 + 32 * 8 * NB * 4 + 16 * 4 + 16;
+    fixed += (2 * 4 * 8 + 2 * 8 * 2 * NB) * 4 + 8 * NB * 4 + 32 * 8 * NB * 4 + 16 * 4 + 16;
     fixed += 8 * (2 * 8 + 2 * 8) + 8 * 8 + 128;                      // barriers + flags + slack
     const size_t fslot = 4 * (size_t)c.d + 128;
     // look-ahead gathers a layer's FFN rows while the previous layer still runs, so

@@ -28,7 +28,7 @@ EXPORTS = ("spffn_workspace_bytes", "spffn_create", "spffn_destroy", "spffn_pred
            "spffn_permute_rows", "spffn_permute_vector", "spffn_last_device_error", "spffn_status_string",
            "spffn_num_partials", "spffn_decode_kernel_launches", "spffn_set_trace", "spffn_trace_marks",
            "spffn_last_cuda_error_string", "spffn_reorder_dealt", "spffn_forward_noalloc",
-           "spffn_decode_lookahead", "spffn_layer_table")
+           "spffn_decode_lookahead", "spffn_layer_table", "spffn_decode_tables")
 
 
 class SpffnError(RuntimeError):
@@ -75,6 +75,7 @@ def library(path: Optional[str] = None):
         "spffn_decode": (st, [ctypes.POINTER(vp), i32, vp, i32, vp, vp, vp, vp]),
         "spffn_decode_lookahead": (st, [ctypes.POINTER(vp), i32, vp, i32, vp, vp, vp, vp]),
         "spffn_layer_table": (st, [vp, ctypes.POINTER(vp)]),
+        "spffn_decode_tables": (st, [ctypes.POINTER(vp), i32, vp, i32, ctypes.POINTER(vp), vp, vp, vp, vp, vp]),
         "spffn_profile_counts": (st, [vp, vp, i32, vp, vp]),
         "spffn_reorder": (st, [vp, i32, vp]),
         "spffn_reorder_dealt": (st, [vp, i32, i32, vp]),
@@ -240,6 +241,16 @@ def decode(layers: Sequence[Layer], x_in, x_out, y, counts=None, stream=None, lo
     fn = library().spffn_decode_lookahead if lookahead else library().spffn_decode
     _check(fn(arr, len(layers), _p(x_in), x_in.shape[0], _p(x_out), _p(y), _p(counts), _stream(stream)),
            "spffn_decode_lookahead" if lookahead else "spffn_decode")
+
+
+def decode_tables(layers: Sequence[Layer], x_in, tables, tab_counts, x_out, y, counts=None, stream=None):
+    """One decode step on caller-supplied neuron tables, no predictor
+    (spffn_decode_tables): ``tables`` is a sequence of L int32 CUDA tensors,
+    ``tab_counts`` an int32 CUDA tensor [L] of their lengths."""
+    arr = (ctypes.c_void_p * len(layers))(*[l.ctx.value for l in layers])
+    tabs = (ctypes.c_void_p * len(tables))(*[_p(t) for t in tables])
+    _check(library().spffn_decode_tables(arr, len(layers), _p(x_in), x_in.shape[0], tabs, _p(tab_counts),
+                                         _p(x_out), _p(y), _p(counts), _stream(stream)), "spffn_decode_tables")
 
 
 def decode_kernel_launches(layers: Sequence[Layer], B: int) -> int:

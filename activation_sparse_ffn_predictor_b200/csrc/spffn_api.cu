@@ -120,6 +120,13 @@ spffn_status spffn_forward(spffn_ctx* ctx, const void* x, int32_t B, const int32
     if (!ctx || !x || !idx || !count || !y || B < 1 || B > ctx->cfg.max_batch) return SPFFN_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(y)) return SPFFN_ERR_INVALID_ARG;
     if (!batch_supported(*ctx, B)) return SPFFN_ERR_UNSUPPORTED;
+    spffn_ctx* one[1] = {ctx};
+    if (fused_tables_supported(one, 1, B)) {
+        // one persistent launch: gathered rows, FC1 + AXPY, fixed-order reduction
+        const int32_t* tabs[1] = {idx};
+        const int32_t* cnts[1] = {count};
+        return cuda_status(launch_fused_tables(one, 1, x, B, tabs, cnts, nullptr, y, nullptr, (cudaStream_t)stream));
+    }
     return cuda_status(launch_forward(*ctx, x, B, idx, count, y, (cudaStream_t)stream));
 }
 
@@ -192,6 +199,42 @@ spffn_status spffn_decode(spffn_ctx* const* layers, int32_t L, const void* x_in,
 spffn_status spffn_decode_lookahead(spffn_ctx* const* layers, int32_t L, const void* x_in, int32_t B,
                                     void* x_out, float* y, int32_t* counts, void* stream) {
     return decode_impl(layers, L, x_in, B, x_out, y, counts, true, stream);
+}
+
+spffn_status spffn_decode_tables(spffn_ctx* const* layers, int32_t L, const void* x_in, int32_t B,
+                                 const int32_t* const* tables, const int32_t* tab_counts, void* x_out, float* y,
+                                 int32_t* counts, void* stream) {
+    if (!layers || L < 1 || !x_in || !x_out || !y || !tables || !tab_counts) return SPFFN_ERR_INVALID_ARG;
+    const spffn_ctx* l0 = layers[0];
+    if (!l0) return SPFFN_ERR_INVALID_ARG;
+    for (int l = 0; l < L; ++l) {
+        const spffn_ctx* c = layers[l];
+        if (!c || !tables[l] || c->cfg.d != l0->cfg.d || c->cfg.dtype != l0->cfg.dtype) return SPFFN_ERR_INVALID_ARG;
+        if (B < 1 || B > c->cfg.max_batch) return SPFFN_ERR_INVALID_ARG;
+        if (!batch_supported(*c, B)) return SPFFN_ERR_UNSUPPORTED;
+    }
+    if (!aligned16(x_in) || !aligned16(x_out) || !aligned16(y) || x_in == x_out) return SPFFN_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    std::vector<const int32_t*> cnt(L);
+    for (int l = 0; l < L; ++l) cnt[l] = tab_counts + l;
+    if (fused_tables_supported(layers, L, B))
+        return cuda_status(launch_fused_tables(layers, L, x_in, B, tables, cnt.data(), x_out, y, counts, st));
+    const void* xcur = x_in;
+    for (int l = 0; l < L; ++l) {
+        const spffn_ctx& c = *layers[l];
+        float* yl = (l == L - 1) ? y : c.ybuf();
+        cudaError_t e = launch_forward(c, xcur, B, tables[l], cnt[l], yl, st);
+        if (e != cudaSuccess) return cuda_status(e);
+        if (counts) {
+            e = cudaMemcpyAsync(counts + l, cnt[l], sizeof(int32_t), cudaMemcpyDeviceToDevice, st);
+            if (e != cudaSuccess) return cuda_status(e);
+        }
+        void* xn = (l == L - 1) ? x_out : c.xbuf(l & 1);
+        e = launch_chain(c, xcur, yl, B, xn, st);
+        if (e != cudaSuccess) return cuda_status(e);
+        xcur = xn;
+    }
+    return SPFFN_OK;
 }
 
 spffn_status spffn_layer_table(spffn_ctx* ctx, const int32_t** idx) {

@@ -45,6 +45,8 @@ constexpr int kMaxMaskWords = 2048;             // n <= 65536 on this path
 struct LayerW {
     const void *W1, *b1, *W2T, *b2, *Wp1, *bp1, *Wp2, *bp2;
     int32_t* idx;
+    const int32_t* tab;        // caller-tables mode: this layer's neuron table and its length (device)
+    const int32_t* tab_count;
 };
 
 struct Params {
@@ -61,6 +63,7 @@ struct Params {
     float* partial;       // [G][B][d]
     float* u;             // [B][d]
     int pred_slots, pred_slot_bytes, ffn_slots, R1, R2, max_rows;
+    int tables;                  // 1: no predictor, each layer's neuron table comes from the caller
     unsigned long long* trace;   // optional [G][L][kTraceMarks] globaltimer stamps
     LayerW layer[kMaxFusedLayers];
 };
@@ -343,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
     if (warp == kConsumerWarps) {
         if (lane == 0) {
             int k = 0;
-            for (int l = 0; l < p.L && !aborted(S, p); ++l) {
+            for (int l = 0; l < p.L && !aborted(S, p) && !p.tables; ++l) {
                 for (int part = 0; part < 2; ++part) {
                     const int r0 = part ? b0 : a0, r1 = part ? b1 : a1, R = part ? p.R2 : p.R1;
                     const size_t rb = part ? (size_t)H * 2 : (size_t)d * 2;
@@ -523,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
                 }
             }
         }
-        if (l == p.L && c == 0) {
+        if (l == p.L && c == 0 && p.x_out) {
             T* xo = reinterpret_cast<T*>(p.x_out);
 #pragma unroll
             for (int m = 0; m < kMaxVPT; ++m) {
@@ -979,7 +982,61 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         if (c == 0 && lane == 0 && p.counts) p.counts[l] = tot;
     };
 
-    if constexpr (!LA) {
+    // caller-tables mode: this CTA's equal slice of layer l's table into list buffer l & 1
+    // (entries outside [0, n) are skipped and latched, the length is clamped to [0, n) and
+    // latched), published as final for the FFN producer; returns the list length
+    auto take_table = [&](int l) -> int {
+        int32_t* nl = S.nl + (l & 1) * p.max_rows;
+        int m = 0;
+        if (warp == 0) {
+            int U = __ldcg(p.layer[l].tab_count);
+            if (U < 0 || U > n) {
+                if (c == 0 && lane == 0) atomicOr(p.err, ERR_COUNT_CLAMPED);
+                U = U < 0 ? 0 : n;
+            }
+            const int lo = split_lo(U, G, c), hi = split_lo(U, G, c + 1);
+            for (int i0 = lo; i0 < hi; i0 += 32) {
+                const int i = i0 + lane;
+                const int j = i < hi ? __ldcg(p.layer[l].tab + i) : -1;
+                const bool bad = i < hi && (j < 0 || j >= n);
+                if (bad) atomicOr(p.err, ERR_IDX_RANGE);
+                const bool on = i < hi && !bad;
+                const uint32_t bal = __ballot_sync(0xffffffffu, on);
+                if (on) nl[m + __popc(bal & ((1u << lane) - 1u))] = j;
+                m += __popc(bal);
+            }
+            __syncwarp();
+            if (lane == 0) {
+                __threadfence_block();
+                S.flags[1] = (l << 16) | m;
+                S.flags[7] = l + 1;                    // the list of layer l is final
+                if (c == 0 && p.counts) p.counts[l] = U;
+                S.misc[15] = __int_as_float(m);
+            }
+        }
+        consumer_sync();
+        return __float_as_int(S.misc[15]);
+    };
+
+    if (p.tables) {
+        // Per layer l: x_l, this CTA's slice of the caller's table, FFN -> partial | grid barrier
+        //              y_l, u_l                                                      | grid barrier
+        for (l = 0; l < p.L && ok; ++l) {
+            load_biases(-1, l);
+            form_x(l);
+            consumer_sync();
+            TRACE(0);
+            const int m = take_table(l);
+            TRACE(6);
+            if (!ffn(l, m)) { ok = false; break; }
+            if (!grid_barrier(S, p, epoch)) { ok = false; break; }
+            TRACE(9);
+            reduce(l);
+            TRACE(10);
+            if (!grid_barrier(S, p, epoch)) { ok = false; break; }
+            TRACE(11);
+        }
+    } else if constexpr (!LA) {
         // Per layer l: A  x_l, h_l (Wp1 rows)            | grid barrier
         //              B  logits_l, list_l, FFN_l -> partial | grid barrier
         //              D  y_l, u_l, table_l                | grid barrier
@@ -1075,7 +1132,7 @@ struct Geometry {
 };
 
 template <typename T, int NB>
-Geometry geometry(const spffn_config& c, int G, bool lookahead) {
+Geometry geometry(const spffn_config& c, int G, bool lookahead, bool tables = false) {
     Geometry g;
     const int budget = 227 * 1024;
     g.pred_slot_bytes = 32 * 1024;
@@ -1097,8 +1154,8 @@ Geometry geometry(const spffn_config& c, int G, bool lookahead) {
     const size_t fslot = 4 * (size_t)c.d + 128;
     // look-ahead gathers a layer's FFN rows while the previous layer still runs, so
     // it trades a predictor slot for more FFN slots
-    g.pred_slots = lookahead ? 3 : 4;
-    g.ffn_slots = lookahead ? 10 : 8;
+    g.pred_slots = tables ? 1 : (lookahead ? 3 : 4);     // no predictor weights to stream with tables
+    g.ffn_slots = (tables || lookahead) ? 10 : 8;
     auto total = [&]() { return fixed + (size_t)g.pred_slots * g.pred_slot_bytes + g.ffn_slots * fslot; };
     while (total() > (size_t)budget && g.ffn_slots > 3) --g.ffn_slots;
     while (total() > (size_t)budget && g.pred_slots > 3) --g.pred_slots;
@@ -1110,11 +1167,13 @@ Geometry geometry(const spffn_config& c, int G, bool lookahead) {
 
 template <typename T, int NB, int HV, bool LA>
 cudaError_t launch_t(spffn_ctx* const* layers, int L, const void* x_in, int B, void* x_out, float* y,
-                     int32_t* counts, cudaStream_t st)
+                     int32_t* counts, cudaStream_t st, const int32_t* const* tabs = nullptr,
+                     const int32_t* const* tab_counts = nullptr)
 {
     const spffn_ctx& c0 = *layers[0];
     const int G = c0.lay.S;
-    Geometry g = geometry<T, NB>(c0.cfg, G, LA);
+    const bool tables = tabs != nullptr;
+    Geometry g = geometry<T, NB>(c0.cfg, G, LA, tables);
     if (g.smem > 227 * 1024) return cudaErrorInvalidConfiguration;
     static Params p;   // host staging copy; the launch copies it into the kernel's parameter space
     p.L = L; p.B = B; p.d = c0.cfg.d; p.n = c0.cfg.n; p.H = c0.cfg.H; p.G = G;
@@ -1132,8 +1191,10 @@ cudaError_t launch_t(spffn_ctx* const* layers, int L, const void* x_in, int B, v
     p.trace = (g_trace && g_trace_bytes >= (size_t)G * L * kTraceMarks * 8) ? g_trace : nullptr;
     for (int l = 0; l < L; ++l) {
         const spffn_ctx& c = *layers[l];
-        p.layer[l] = LayerW{c.w.W1, c.w.b1, c.w.W2T, c.w.b2, c.w.Wp1, c.w.bp1, c.w.Wp2, c.w.bp2, c.idx()};
+        p.layer[l] = LayerW{c.w.W1, c.w.b1, c.w.W2T, c.w.b2, c.w.Wp1, c.w.bp1, c.w.Wp2, c.w.bp2, c.idx(),
+                            tables ? tabs[l] : nullptr, tables ? tab_counts[l] : nullptr};
     }
+    p.tables = tables ? 1 : 0;
     cudaError_t e = cudaFuncSetAttribute(k_decode<T, NB, HV, LA>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem);
     if (e != cudaSuccess) return e;
     e = cudaMemsetAsync(&ctl->barrier[0], 0, 2 * sizeof(uint32_t), st);
@@ -1152,6 +1213,21 @@ cudaError_t launch_t(spffn_ctx* const* layers, int L, const void* x_in, int B, v
 }
 
 }  // namespace
+
+bool fused_tables_supported(spffn_ctx* const* layers, int L, int B)
+{
+    if (L < 1 || L > kMaxFusedLayers || B < 1 || B > 2) return false;
+    const spffn_config& c0 = layers[0]->cfg;
+    if (c0.d > kMaxVPT * 8 * kConsumers) return false;
+    if (layers[0]->lay.S > kMaxG || layers[0]->lay.S != layers[0]->num_sms) return false;
+    for (int l = 1; l < L; ++l) {
+        const spffn_config& c = layers[l]->cfg;
+        if (c.d != c0.d || c.n != c0.n || c.dtype != c0.dtype) return false;
+    }
+    const Geometry g = c0.dtype == SPFFN_BF16 ? geometry<__nv_bfloat16, 2>(c0, layers[0]->lay.S, false, true)
+                                          : geometry<__half, 2>(c0, layers[0]->lay.S, false, true);
+    return g.smem <= 227 * 1024;
+}
 
 bool fused_decode_supported(spffn_ctx* const* layers, int L, int B)
 {
@@ -1197,6 +1273,20 @@ cudaError_t launch_fused_decode(spffn_ctx* const* layers, int L, const void* x_i
     if (bf) { SPFFN_HV(__nv_bfloat16, 2) } else { SPFFN_HV(__half, 2) }
 #undef SPFFN_HV
 #undef SPFFN_GO
+}
+
+cudaError_t launch_fused_tables(spffn_ctx* const* layers, int L, const void* x_in, int B,
+                                const int32_t* const* tabs, const int32_t* const* tab_counts, void* x_out,
+                                float* y, int32_t* counts, cudaStream_t st)
+{
+    // the logits GEMV does not run: any hidden width fits (HV only sizes its registers)
+    const bool bf = layers[0]->cfg.dtype == SPFFN_BF16;
+    if (B == 1) {
+        return bf ? launch_t<__nv_bfloat16, 1, 1, false>(layers, L, x_in, B, x_out, y, counts, st, tabs, tab_counts)
+                  : launch_t<__half, 1, 1, false>(layers, L, x_in, B, x_out, y, counts, st, tabs, tab_counts);
+    }
+    return bf ? launch_t<__nv_bfloat16, 2, 1, false>(layers, L, x_in, B, x_out, y, counts, st, tabs, tab_counts)
+              : launch_t<__half, 2, 1, false>(layers, L, x_in, B, x_out, y, counts, st, tabs, tab_counts);
 }
 
 }  // namespace spffn

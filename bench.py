@@ -13,6 +13,7 @@ predicted from layer l's input, DejaVu's asynchronous predictor), reported
 under its own workload name.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1] [--lookahead] [--impl ours|reference]
+    python bench.py --config 3 --rate 0.05 --true-mask     # sparse FFN on the true set, no predictor
 
 Under torchrun each rank runs its own replica on its own decode stream
 (independent requests: weak scaling, no data-path collective); the reported time
@@ -330,6 +331,124 @@ def run_ours(args, cfg, world, rank, local):
     return res, (rank == 0)
 
 
+def run_true_mask(args, cfg, world, rank, local):
+    """The sparse FFN alone on each token's true activation set (z > 0), no predictor:
+    one spffn_decode_tables per step (per layer the FFN over the true table, then
+    the chaining).  The tables come
+    from an untimed pass of the same deterministic steps (the library's profile
+    kernel on one step's layer input gives that input's z > 0 set); the timed
+    replays then see exactly the inputs the tables were taken from."""
+    import torch
+    import activation_sparse_ffn_predictor_b200 as sp
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist_init(world, "nccl")
+    L = cfg.layers
+    B, K, W = cfg.batch, args.steps, args.warmup
+    if B >= 16:
+        raise SystemExit("--true-mask measures the per-phase FFN kernels: batch < 16")
+    stack = build_stack(cfg, L, device, rate=args.rate)
+    layers = [s_[1] for s_ in stack]
+    seed = rank_seed(rank)
+    dt = torch.bfloat16 if cfg.bf16 else torch.float16
+    xs = torch.stack([wl.to_torch(wl.tokens(cfg, B, aux=s_, seed=seed), cfg, device) for s_ in range(K + W)])
+    xl = torch.empty(L + 1, B, cfg.d, dtype=dt, device=device)
+    y = torch.empty(B, cfg.d, dtype=torch.float32, device=device)
+    idx = torch.zeros(K + W, L, cfg.n, dtype=torch.int32, device=device)
+    cnt = torch.zeros(K + W, L, 1, dtype=torch.int32, device=device)
+    prof = torch.zeros(cfg.n, dtype=torch.int32, device=device)
+    stream = torch.cuda.Stream(device)
+
+    tabs = [[idx[s_, l] for l in range(L)] for s_ in range(K + W)]
+    tcnt = cnt[:, :, 0].contiguous()
+
+    def ffn_step(s_):
+        sp.decode_tables(layers, xl[0], tabs[s_], tcnt[s_], xl[L], y, stream=stream)
+
+    graphs = []
+    with torch.cuda.stream(stream):
+        for s_ in range(K + W):
+            xl[0].copy_(xs[s_])
+            for l, Ly in enumerate(layers):
+                prof.zero_()
+                Ly.profile_counts(xl[l], prof, stream=stream)
+                sel = torch.nonzero(prof > 0).flatten().to(torch.int32)
+                idx[s_, l, :sel.numel()] = sel
+                cnt[s_, l, 0] = sel.numel()
+                Ly.forward(xl[l], idx[s_, l], cnt[s_, l], y, stream=stream)
+                Ly.chain(xl[l], y, xl[l + 1], stream=stream)
+    stream.synchronize()
+    tcnt = cnt[:, :, 0].contiguous()
+    for s_ in range(K + W):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            ffn_step(s_)
+        graphs.append(g)
+    with torch.cuda.stream(stream):
+        for s_ in range(W):
+            xl[0].copy_(xs[s_])
+            graphs[s_].replay()
+    stream.synchronize()
+    barrier(world, device)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(local) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for k in range(K):
+                xl[0].copy_(xs[W + k])
+                ev[k][0].record(stream)
+                graphs[W + k].replay()
+                ev[k][1].record(stream)
+            e1.record(stream)
+        stream.synchronize()
+    torch.cuda.synchronize()
+    barrier(world, device)
+    t_max = max_over_ranks(e0.elapsed_time(e1), world, device)
+    ks = cnt[W:, :, 0].cpu().numpy()
+    bytes_per_step = [int(ks[k].sum()) * ffn_bytes_per_neuron(cfg) for k in range(K)]
+    mean_launch_ms = sum(a.elapsed_time(b) for a, b in ev) / K
+    achieved = (sum(bytes_per_step) / K) / (mean_launch_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+    # end to end: pinned host x in, the last layer's y out, every step
+    xh = torch.empty(K, B, cfg.d, dtype=dt).pin_memory()
+    xh.copy_(xs[W:].cpu())
+    yh = torch.empty(K, B, cfg.d, dtype=torch.float32).pin_memory()
+    barrier(world, device)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for k in range(K):
+            xl[0].copy_(xh[k], non_blocking=True)
+            graphs[W + k].replay()
+            yh[k].copy_(y, non_blocking=True)
+        f1.record(stream)
+    stream.synchronize()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world, device)
+    del graphs
+    rate = args.rate or cfg.rate
+    res = {
+        "metric": METRIC, "value": world * B * K / (t_max * 1e-3), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": t_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": cfg.dtype, "data": "synthetic",
+        "config": {"workload": "%s-truemask-r%g" % (cfg.name, rate), "layers": L, "d": cfg.d, "n": cfg.n,
+                   "batch": B, "activation_rate": rate, "alpha": cfg.alpha, "global_batch": B * world,
+                   "mean_active_neurons": float(ks.mean()), "parallelism": "replicas%d" % world,
+                   "prediction": "none: each token's true activation set (z > 0), taken before timing",
+                   "l2": "%.2f GB touched per step" % (sum(bytes_per_step) / K / 1e9)},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "kernel": "spffn_decode_tables (one graph per step)", "peak_kind": peak_kind},
+        "e2e": {"value": world * B * K / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": B * cfg.d * 2,
+                "d2h_bytes_per_step": B * cfg.d * 4},
+        # the persistent kernel at B <= 2 (d <= 10240): one launch per step; else FFN + reduction + chaining per layer
+        "gpu_launches": (1 if B <= 2 and cfg.d <= 10240 else 3 * L) * K,
+        "clocks": clk.summary(),
+    }
+    return res, (rank == 0)
+
+
 # ---------------------------------------------------------------------------
 def cpu_threads() -> int:
     try:
@@ -417,6 +536,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--lookahead", action="store_true",
                     help="predict layer l+1's neuron set from layer l's input (DejaVu look-ahead)")
+    ap.add_argument("--true-mask", action="store_true",
+                    help="time the sparse FFN alone on each token's true activation set (no predictor)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -428,6 +549,8 @@ def main(argv=None):
     world, rank, local = dist_env()
     if args.impl == "reference":
         res, show = run_reference(args, cfg, world, rank, local)
+    elif args.true_mask:
+        res, show = run_true_mask(args, cfg, world, rank, local)
     else:
         res, show = run_ours(args, cfg, world, rank, local)
         if show and world == 1 and not args.no_cpu_baseline:

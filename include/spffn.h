@@ -161,6 +161,19 @@ spffn_status spffn_decode(spffn_ctx* const* layers, int32_t L, const void* x_in,
 spffn_status spffn_decode_lookahead(spffn_ctx* const* layers, int32_t L, const void* x_in, int32_t B,
                                     void* x_out, float* y, int32_t* counts, void* stream);
 
+/* One decode step through L layers on caller-supplied neuron tables, no predictor
+ * (e.g. each token's true activation set, or any other mask):
+ *   for l = 0..L-1:  y_l = forward_l(x_l; tables[l][0..tab_counts[l]));  x_{l+1} = chain(x_l, y_l)
+ * tables: host array of L device pointers to int32 tables, entries as for
+ * spffn_forward (distinct, in [0,n); out-of-range entries skipped and latched).
+ * tab_counts: device int32 [L] (each clamped to [0,n], latched).  x_in, x_out,
+ * y, counts (which receives the clamped lengths, may be NULL) as for
+ * spffn_decode.  At B <= 2 the whole stack is one persistent kernel (two grid
+ * barriers per layer); otherwise per-layer launches. */
+spffn_status spffn_decode_tables(spffn_ctx* const* layers, int32_t L, const void* x_in, int32_t B,
+                                 const int32_t* const* tables, const int32_t* tab_counts, void* x_out, float* y,
+                                 int32_t* counts, void* stream);
+
 /* Device pointer to the neuron table that the last spffn_decode or
  * spffn_decode_lookahead left in this layer's workspace (ascending neuron
  * indices; its length is that call's counts[l]).  Valid until the next call

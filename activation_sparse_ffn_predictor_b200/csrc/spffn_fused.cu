@@ -294,7 +294,7 @@ __device__ __forceinline__ bool cwait(const Shared& S, const Params& p, uint64_t
     } while (0)
 
 // ---------------------------------------------------------------------------
-template <typename T, int NB, int HV, bool LA>
+template <typename T, int NB, int HV, bool LA, bool TAB>
 __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ Params p)
 {
     extern __shared__ __align__(128) char smem[];
@@ -346,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
     if (warp == kConsumerWarps) {
         if (lane == 0) {
             int k = 0;
-            for (int l = 0; l < p.L && !aborted(S, p) && !p.tables; ++l) {
+            for (int l = 0; l < p.L && !aborted(S, p) && !TAB; ++l) {
                 for (int part = 0; part < 2; ++part) {
                     const int r0 = part ? b0 : a0, r1 = part ? b1 : a1, R = part ? p.R2 : p.R1;
                     const size_t rb = part ? (size_t)H * 2 : (size_t)d * 2;
@@ -567,38 +567,79 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
             if (r == a0) TRACE(1);
             const uint4* slot = reinterpret_cast<const uint4*>(S.pring + (size_t)s * p.pred_slot_bytes);
             const int rows = min(R1, a1 - r);
-            for (int rr = 0; rr < rows; rr += 2) {
-                const bool two = rr + 1 < rows;
-                const uint4* w0p = slot + (size_t)rr * nvec;
-                const uint4* w1p = slot + (size_t)(two ? rr + 1 : rr) * nvec;
-                u64 c0[NB], c1[NB];
-#pragma unroll
-                for (int t = 0; t < NB; ++t) c0[t] = c1[t] = 0ull;
-#pragma unroll
-                for (int m = 0; m < kMaxVPT; ++m) {
-                    const int v = seg_lo + lane + 32 * m;
-                    if (v < seg_hi) {
-                        const uint4 w0 = w0p[v], w1 = w1p[v];
-                        const u64 p00 = Arith<T>::widen2(w0.x), p01 = Arith<T>::widen2(w0.y);
-                        const u64 p02 = Arith<T>::widen2(w0.z), p03 = Arith<T>::widen2(w0.w);
-                        const u64 p10 = Arith<T>::widen2(w1.x), p11 = Arith<T>::widen2(w1.y);
-                        const u64 p12 = Arith<T>::widen2(w1.z), p13 = Arith<T>::widen2(w1.w);
-#pragma unroll
-                        for (int t = 0; t < NB; ++t) {
-                            ffma2(c0[t], p00, xg[m][0][t]); ffma2(c0[t], p01, xg[m][1][t]);
-                            ffma2(c0[t], p02, xg[m][2][t]); ffma2(c0[t], p03, xg[m][3][t]);
-                            ffma2(c1[t], p10, xg[m][0][t]); ffma2(c1[t], p11, xg[m][1][t]);
-                            ffma2(c1[t], p12, xg[m][2][t]); ffma2(c1[t], p13, xg[m][3][t]);
+            if constexpr (NB == 1) {
+                // B = 1: four rows at a time (four independent dot chains); rows past the end
+                // repeat the last row and their results are dropped.  B = 2: two rows at a time.
+                constexpr int kR = 4;
+                for (int rr = 0; rr < rows; rr += kR) {
+                    const uint4* wp[kR];
+    #pragma unroll
+                    for (int u = 0; u < kR; ++u) wp[u] = slot + (size_t)min(rr + u, rows - 1) * nvec;
+                    u64 cc[kR][NB];
+    #pragma unroll
+                    for (int u = 0; u < kR; ++u)
+    #pragma unroll
+                        for (int t = 0; t < NB; ++t) cc[u][t] = 0ull;
+    #pragma unroll
+                    for (int m = 0; m < kMaxVPT; ++m) {
+                        const int v = seg_lo + lane + 32 * m;
+                        if (v < seg_hi) {
+    #pragma unroll
+                            for (int u = 0; u < kR; ++u) {
+                                const uint4 w = wp[u][v];
+                                const u64 q0 = Arith<T>::widen2(w.x), q1 = Arith<T>::widen2(w.y);
+                                const u64 q2 = Arith<T>::widen2(w.z), q3 = Arith<T>::widen2(w.w);
+    #pragma unroll
+                                for (int t = 0; t < NB; ++t) {
+                                    ffma2(cc[u][t], q0, xg[m][0][t]); ffma2(cc[u][t], q1, xg[m][1][t]);
+                                    ffma2(cc[u][t], q2, xg[m][2][t]); ffma2(cc[u][t], q3, xg[m][3][t]);
+                                }
+                            }
                         }
                     }
+    #pragma unroll
+                    for (int u = 0; u < kR; ++u)
+    #pragma unroll
+                        for (int t = 0; t < NB; ++t) {
+                            const float2 e = upk(cc[u][t]);
+                            const float z = warp_sum(e.x + e.y);
+                            if (lane == 0 && rr + u < rows) S.red1[((rr + u) * kConsumerWarps + warp) * NB + t] = z;
+                        }
                 }
-#pragma unroll
-                for (int t = 0; t < NB; ++t) {
-                    const float2 e0 = upk(c0[t]), e1 = upk(c1[t]);
-                    const float z0 = warp_sum(e0.x + e0.y), z1 = warp_sum(e1.x + e1.y);
-                    if (lane == 0) {
-                        S.red1[(rr * kConsumerWarps + warp) * NB + t] = z0;
-                        if (two) S.red1[((rr + 1) * kConsumerWarps + warp) * NB + t] = z1;
+            } else {
+                for (int rr = 0; rr < rows; rr += 2) {
+                    const bool two = rr + 1 < rows;
+                    const uint4* w0p = slot + (size_t)rr * nvec;
+                    const uint4* w1p = slot + (size_t)(two ? rr + 1 : rr) * nvec;
+                    u64 c0[NB], c1[NB];
+    #pragma unroll
+                    for (int t = 0; t < NB; ++t) c0[t] = c1[t] = 0ull;
+    #pragma unroll
+                    for (int m = 0; m < kMaxVPT; ++m) {
+                        const int v = seg_lo + lane + 32 * m;
+                        if (v < seg_hi) {
+                            const uint4 w0 = w0p[v], w1 = w1p[v];
+                            const u64 p00 = Arith<T>::widen2(w0.x), p01 = Arith<T>::widen2(w0.y);
+                            const u64 p02 = Arith<T>::widen2(w0.z), p03 = Arith<T>::widen2(w0.w);
+                            const u64 p10 = Arith<T>::widen2(w1.x), p11 = Arith<T>::widen2(w1.y);
+                            const u64 p12 = Arith<T>::widen2(w1.z), p13 = Arith<T>::widen2(w1.w);
+    #pragma unroll
+                            for (int t = 0; t < NB; ++t) {
+                                ffma2(c0[t], p00, xg[m][0][t]); ffma2(c0[t], p01, xg[m][1][t]);
+                                ffma2(c0[t], p02, xg[m][2][t]); ffma2(c0[t], p03, xg[m][3][t]);
+                                ffma2(c1[t], p10, xg[m][0][t]); ffma2(c1[t], p11, xg[m][1][t]);
+                                ffma2(c1[t], p12, xg[m][2][t]); ffma2(c1[t], p13, xg[m][3][t]);
+                            }
+                        }
+                    }
+    #pragma unroll
+                    for (int t = 0; t < NB; ++t) {
+                        const float2 e0 = upk(c0[t]), e1 = upk(c1[t]);
+                        const float z0 = warp_sum(e0.x + e0.y), z1 = warp_sum(e1.x + e1.y);
+                        if (lane == 0) {
+                            S.red1[(rr * kConsumerWarps + warp) * NB + t] = z0;
+                            if (two) S.red1[((rr + 1) * kConsumerWarps + warp) * NB + t] = z1;
+                        }
                     }
                 }
             }
@@ -1018,7 +1059,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         return __float_as_int(S.misc[15]);
     };
 
-    if (p.tables) {
+    if constexpr (TAB) {
         // Per layer l: x_l, this CTA's slice of the caller's table, FFN -> partial | grid barrier
         //              y_l, u_l                                                      | grid barrier
         for (l = 0; l < p.L && ok; ++l) {
@@ -1165,14 +1206,15 @@ Geometry geometry(const spffn_config& c, int G, bool lookahead, bool tables = fa
     return g;
 }
 
-template <typename T, int NB, int HV, bool LA>
+template <typename T, int NB, int HV, bool LA, bool TAB = false>
 cudaError_t launch_t(spffn_ctx* const* layers, int L, const void* x_in, int B, void* x_out, float* y,
                      int32_t* counts, cudaStream_t st, const int32_t* const* tabs = nullptr,
                      const int32_t* const* tab_counts = nullptr)
 {
     const spffn_ctx& c0 = *layers[0];
     const int G = c0.lay.S;
-    const bool tables = tabs != nullptr;
+    const bool tables = TAB;
+    if (TAB != (tabs != nullptr)) return cudaErrorInvalidValue;
     Geometry g = geometry<T, NB>(c0.cfg, G, LA, tables);
     if (g.smem > 227 * 1024) return cudaErrorInvalidConfiguration;
     static Params p;   // host staging copy; the launch copies it into the kernel's parameter space
@@ -1195,7 +1237,7 @@ cudaError_t launch_t(spffn_ctx* const* layers, int L, const void* x_in, int B, v
                             tables ? tabs[l] : nullptr, tables ? tab_counts[l] : nullptr};
     }
     p.tables = tables ? 1 : 0;
-    cudaError_t e = cudaFuncSetAttribute(k_decode<T, NB, HV, LA>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem);
+    cudaError_t e = cudaFuncSetAttribute(k_decode<T, NB, HV, LA, TAB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem);
     if (e != cudaSuccess) return e;
     e = cudaMemsetAsync(&ctl->barrier[0], 0, 2 * sizeof(uint32_t), st);
     if (e != cudaSuccess) return e;
@@ -1209,7 +1251,7 @@ cudaError_t launch_t(spffn_ctx* const* layers, int L, const void* x_in, int B, v
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_decode<T, NB, HV, LA>, p);
+    return cudaLaunchKernelEx(&cfg, k_decode<T, NB, HV, LA, TAB>, p);
 }
 
 }  // namespace
@@ -1282,11 +1324,11 @@ cudaError_t launch_fused_tables(spffn_ctx* const* layers, int L, const void* x_i
     // the logits GEMV does not run: any hidden width fits (HV only sizes its registers)
     const bool bf = layers[0]->cfg.dtype == SPFFN_BF16;
     if (B == 1) {
-        return bf ? launch_t<__nv_bfloat16, 1, 1, false>(layers, L, x_in, B, x_out, y, counts, st, tabs, tab_counts)
-                  : launch_t<__half, 1, 1, false>(layers, L, x_in, B, x_out, y, counts, st, tabs, tab_counts);
+        return bf ? launch_t<__nv_bfloat16, 1, 1, false, true>(layers, L, x_in, B, x_out, y, counts, st, tabs, tab_counts)
+                  : launch_t<__half, 1, 1, false, true>(layers, L, x_in, B, x_out, y, counts, st, tabs, tab_counts);
     }
-    return bf ? launch_t<__nv_bfloat16, 2, 1, false>(layers, L, x_in, B, x_out, y, counts, st, tabs, tab_counts)
-              : launch_t<__half, 2, 1, false>(layers, L, x_in, B, x_out, y, counts, st, tabs, tab_counts);
+    return bf ? launch_t<__nv_bfloat16, 2, 1, false, true>(layers, L, x_in, B, x_out, y, counts, st, tabs, tab_counts)
+              : launch_t<__half, 2, 1, false, true>(layers, L, x_in, B, x_out, y, counts, st, tabs, tab_counts);
 }
 
 }  // namespace spffn

@@ -111,9 +111,9 @@ def step_bytes(cfg, counts_sum: int, layers: int) -> int:
 # captured on: any change to them and the bench reports null.
 DECODE_SOURCES = ("spffn_fused.cu", "spffn_fused.cuh", "spffn_internal.cuh")
 DECODE_TRAFFIC = {
-    "sha256": "c8d612a3911afc4fa903bbd7678236d3b50a76f446f701dcdba51a16cf9d809a",
+    "sha256": "1ab8b8f3c4695dd7a28f8ab8ebcd4a1c6d8f1a1e4c958cd03b9c30636800b1bd",
     "workload": "opt6.7b-d4096-n16384-L32", "batch": 1, "rate": 0.05,
-    "bytes_per_layer": (223.093504e6 + 4.497920e6) / 4,
+    "bytes_per_layer": (223.213824e6 + 5.454848e6) / 4,
     "summary": "profiles/k_decode_opt6.7b-d4096-n16384_b1.md",
 }
 

@@ -17,7 +17,8 @@ import numpy as np
 
 from . import build as _build
 
-__all__ = ["SpffnError", "Layer", "decode", "reorder", "permute_rows", "permute_vector",
+__all__ = ["SpffnError", "Layer", "decode", "decode_tables", "decode_kernel_launches", "forward_noalloc",
+           "reorder", "reorder_dealt", "permute_rows", "permute_vector", "set_trace", "trace_marks",
            "workspace_bytes", "library", "F16", "BF16"]
 
 F16, BF16 = 0, 1

@@ -63,7 +63,6 @@ struct Params {
     float* partial;       // [G][B][d]
     float* u;             // [B][d]
     int pred_slots, pred_slot_bytes, ffn_slots, R1, R2, max_rows;
-    int tables;                  // 1: no predictor, each layer's neuron table comes from the caller
     unsigned long long* trace;   // optional [G][L][kTraceMarks] globaltimer stamps
     LayerW layer[kMaxFusedLayers];
 };
@@ -203,9 +202,7 @@ __device__ __forceinline__ int split_lo(int total, int parts, int i) {
 // packed two-lane fp32 FMA.
 typedef unsigned long long u64;
 
-#ifndef SPFFN_WAIT_HINT_NS
-#define SPFFN_WAIT_HINT_NS 1000000
-#endif
+constexpr uint32_t kWaitHintNs = 1000000;        // suspend-time hint of a consumer's mbarrier wait
 
 __device__ __forceinline__ u64 pk(float a, float b) {
     u64 r;
@@ -267,7 +264,7 @@ __device__ __forceinline__ bool mbar_try_hint(uint64_t* b, uint32_t parity) {
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(sptr(b)), "r"(parity), "r"((uint32_t)SPFFN_WAIT_HINT_NS)
+        : "r"(sptr(b)), "r"(parity), "r"(kWaitHintNs)
         : "memory");
     return ok != 0;
 }
@@ -360,7 +357,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
                         S.flags[2] = k + 1;
                     }
                 }
-#ifndef SPFFN_NO_L2_PREFETCH
                 if (l + 1 < p.L) {
                     for (int part = 0; part < 2; ++part) {
                         const int r0 = part ? b0 : a0, r1 = part ? b1 : a1;
@@ -371,7 +367,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
                             bulk_prefetch_l2(base + (size_t)r0 * rb + off, (uint32_t)min((size_t)32768, total - off));
                     }
                 }
-#endif
             }
         pred_done:
             __threadfence_block();
@@ -1236,7 +1231,6 @@ cudaError_t launch_t(spffn_ctx* const* layers, int L, const void* x_in, int B, v
         p.layer[l] = LayerW{c.w.W1, c.w.b1, c.w.W2T, c.w.b2, c.w.Wp1, c.w.bp1, c.w.Wp2, c.w.bp2, c.idx(),
                             tables ? tabs[l] : nullptr, tables ? tab_counts[l] : nullptr};
     }
-    p.tables = tables ? 1 : 0;
     cudaError_t e = cudaFuncSetAttribute(k_decode<T, NB, HV, LA, TAB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem);
     if (e != cudaSuccess) return e;
     e = cudaMemsetAsync(&ctl->barrier[0], 0, 2 * sizeof(uint32_t), st);

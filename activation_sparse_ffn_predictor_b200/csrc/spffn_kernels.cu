@@ -1,7 +1,9 @@
 // Per-phase kernels of the sparse-FFN decode path (one launch per phase).
 //
-// These serve spffn_predict / spffn_forward / spffn_chain / the offline
-// profile and permutation calls.  Every weight row is read with 16-byte
+// These serve spffn_predict and spffn_forward at batches 3..15 (and for shapes
+// outside the persistent kernel's limits; batches of 16 and more run on the union
+// path, and spffn_forward at 1..2 on the persistent kernel), spffn_chain, and the
+// offline profile and permutation calls.  Every weight row is read with 16-byte
 // vector loads that bypass L1 (each row is touched once per call); fp32
 // accumulation throughout; every reduction has a fixed order.
 #include "spffn_internal.cuh"

@@ -1,27 +1,30 @@
-// Union-mask tensor-core path for batches of 16..32 tokens.
+// Union-mask tensor-core path for batches of 16..256 tokens.
 //
 // With B tokens the union of the per-token neuron sets is a dense contraction
 // over the gathered rows (each weight byte feeds B products), so every GEMM of
 // the layer runs on the 5th-generation tensor cores:
 //
-//   mode 0  predictor-1   D[H x B]   = Wp1[H x d]        . X[B x d]^T        split-K
-//   mode 1  predictor-2   D[n x 2B]  = Wp2[n x H]        . hsplit[2B x H]^T  -> mask words
-//   mode 2  FC1 (union)   D[U x B]   = W1[table][U x d]  . X[B x d]^T        split-K
-//   mode 3  FC2 (union)   D[d x 2B]  = W2T[table]^T      . asplit[2B x U]^T  split-K
+//   mode 0  predictor-1   D[H x B]    = Wp1[H x d]        . X[B x d]^T          split-K
+//   mode 1  predictor-2   D[n x 2Gt]  = Wp2[n x H]        . hsplit_g[2Gt x H]^T -> mask words
+//   mode 2  FC1 (union)   D[U x B]    = W1[table][U x d]  . X[B x d]^T          split-K
+//   mode 3  FC2 (union)   D[d x 2Gt]  = W2T[table]^T      . asplit_g[2Gt x U]^T split-K
 //
 // fp32 activations (h, a) enter the 16-bit MMA as a hi/lo pair of the storage
 // dtype (v ~= hi + lo, hi = round(v), lo = round(v - hi)); the epilogue adds the
-// two column halves of D.  X is already in the storage dtype (exact).
+// two column halves of D.  X is already in the storage dtype (exact).  Modes 1
+// and 3 run once per token group g of Gt <= 128 tokens (N = 2 Gt <= 256).
 //
-// One persistent CTA per SM; warp 0 issues TMA loads into a ring of 4..6 stages
-// (2-D tiles for the contiguous operands, tile::gather4 for FC2's table rows; never
-// multicast), warps 6..9 gather FC1's table rows with coalesced 16-byte cp.async
-// into the same 128-byte swizzled image (each thread fences its landed copies into
-// the async proxy before it arrives; twice the rate of gather4 for these 128-byte
-// row pieces, while FC2's 256-byte pieces go faster through gather4), warp 1
-// issues tcgen05.mma into a double buffered TMEM accumulator, warps 2..5 read TMEM
-// (tcgen05.ld) and run the epilogue.  Split-K partials are summed in fixed split order by the last CTA
-// to finish a tile (atomic ticket, no waiting), so results are deterministic.
+// One persistent CTA per SM:
+// - warp 0 issues TMA loads into a ring of 4..6 stages: 2-D tiles for the
+//   contiguous operands, tile::gather4 for FC2's table rows, never multicast;
+// - warps 6..9 gather FC1's table rows with coalesced 16-byte cp.async into the
+//   same 128-byte swizzled image.  Each thread fences its landed copies into the
+//   async proxy before it arrives.  This is twice the rate of gather4 for these
+//   128-byte row pieces, while FC2's 256-byte pieces go faster through gather4;
+// - warp 1 issues tcgen05.mma into a double-buffered TMEM accumulator;
+// - warps 2..5 read TMEM (tcgen05.ld), 16 columns at a time, and run the epilogue.
+// Split-K partials are summed in fixed split order by the last CTA to finish a
+// tile (atomic ticket, no waiting), so results are deterministic.
 #include <cuda.h>
 #include <algorithm>
 #include <cstring>

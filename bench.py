@@ -111,9 +111,9 @@ def step_bytes(cfg, counts_sum: int, layers: int) -> int:
 # captured on: any change to them and the bench reports null.
 DECODE_SOURCES = ("spffn_fused.cu", "spffn_fused.cuh", "spffn_internal.cuh")
 DECODE_TRAFFIC = {
-    "sha256": "1ab8b8f3c4695dd7a28f8ab8ebcd4a1c6d8f1a1e4c958cd03b9c30636800b1bd",
+    "sha256": "5f09df9818cc796c3d3a84b55a3f382c3dc1e04be6deb42743f4b9b4eeab11db",
     "workload": "opt6.7b-d4096-n16384-L32", "batch": 1, "rate": 0.05,
-    "bytes_per_layer": (223.213824e6 + 5.454848e6) / 4,
+    "bytes_per_layer": (223.219712e6 + 6.285056e6) / 4,
     "summary": "profiles/k_decode_opt6.7b-d4096-n16384_b1.md",
 }
 

@@ -14,6 +14,7 @@ under its own workload name.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1] [--lookahead] [--impl ours|reference]
     python bench.py --config 3 --rate 0.05 --true-mask     # sparse FFN on the true set, no predictor
+    python bench.py --dense                                # comparison: dense FFN with cuBLAS, same weights
 
 Under torchrun each rank runs its own replica on its own decode stream
 (independent requests: weak scaling, no data-path collective); the reported time
@@ -102,6 +103,10 @@ def ffn_bytes_per_neuron(cfg) -> int:
 
 def step_bytes(cfg, counts_sum: int, layers: int) -> int:
     return layers * predictor_bytes(cfg) + counts_sum * ffn_bytes_per_neuron(cfg)
+
+
+def dense_bytes_per_layer(cfg) -> int:
+    return 4 * cfg.n * cfg.d + 2 * cfg.n     # every W1 and W2T row + b1
 
 
 # DRAM traffic (ncu dram__bytes_read.sum + dram__bytes_write.sum) of the
@@ -449,6 +454,97 @@ def run_true_mask(args, cfg, world, rank, local):
     return res, (rank == 0)
 
 
+def dense_layer(dl, x):
+    """One layer's dense FFN with cuBLAS: y = W2T^T ReLU(W1 x + b1) (fp16 GEMM
+    outputs, fp32 accumulation inside cuBLAS), returned in fp32."""
+    import torch
+    a = torch.relu(torch.addmm(dl.b1, x, dl.W1.t()))
+    return torch.mm(a, dl.W2T).float()
+
+
+def dense_stack(dls, x, dt):
+    """x through every layer's dense FFN and the chaining x' = (x + y) / rms(x + y)."""
+    import torch
+    for dl in dls:
+        u = x.float() + dense_layer(dl, x)
+        x = (u * torch.rsqrt(u.square().mean(dim=-1, keepdim=True) + 1e-6)).to(dt)
+    return x
+
+
+def run_dense(args, cfg, world, rank, local):
+    """Comparison arm, not the product path: the dense FFN of every layer on the
+    same weights with cuBLAS GEMMs (dense_layer), ReLU and the same chaining in
+    plain torch ops, one CUDA graph per step.  It
+    shows what the predictor and the sparse FFN save over computing every
+    neuron."""
+    import torch
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist_init(world, "nccl")
+    L = cfg.layers
+    B, K, W = cfg.batch, args.steps, args.warmup
+    stack = build_stack(cfg, L, device, rate=args.rate, reorder=False)
+    dls = [s_[0] for s_ in stack]
+    dt = torch.bfloat16 if cfg.bf16 else torch.float16
+    seed = rank_seed(rank)
+    xs = torch.stack([wl.to_torch(wl.tokens(cfg, B, aux=s_, seed=seed), cfg, device) for s_ in range(K + W)])
+    x_in = torch.empty(B, cfg.d, dtype=dt, device=device)
+    out = {}
+    stream = torch.cuda.Stream(device)
+
+    def one_step():
+        out["x"] = dense_stack(dls, x_in, dt)
+
+    with torch.cuda.stream(stream):
+        x_in.copy_(xs[0])
+        one_step()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        one_step()
+    with torch.cuda.stream(stream):
+        for s_ in range(W):
+            x_in.copy_(xs[s_])
+            g.replay()
+    stream.synchronize()
+    barrier(world, device)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(local) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for k in range(K):
+                x_in.copy_(xs[W + k])
+                ev[k][0].record(stream)
+                g.replay()
+                ev[k][1].record(stream)
+            e1.record(stream)
+        stream.synchronize()
+    torch.cuda.synchronize()
+    barrier(world, device)
+    t_max = max_over_ranks(e0.elapsed_time(e1), world, device)
+    del g
+    mean_ms = sum(a_.elapsed_time(b_) for a_, b_ in ev) / K
+    achieved = L * dense_bytes_per_layer(cfg) / (mean_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+    res = {
+        "metric": METRIC, "value": world * B * K / (t_max * 1e-3), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": t_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": cfg.dtype, "data": "synthetic", "impl": "dense-cublas",
+        "config": {"workload": cfg.name + "-dense", "layers": L, "d": cfg.d, "n": cfg.n, "batch": B,
+                   "global_batch": B * world, "parallelism": "replicas%d" % world,
+                   "prediction": "none: every neuron computed (dense FFN, torch/cuBLAS)",
+                   "l2": "inputs larger than L2 (%.2f GB of FFN weights per step)" % (L * dense_bytes_per_layer(cfg) / 1e9)},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "kernel": "cuBLAS GEMMs + torch elementwise (one graph per step)",
+                     "peak_kind": peak_kind},
+        "gpu_launches": 0,
+        "clocks": clk.summary(),
+    }
+    return res, (rank == 0)
+
+
 # ---------------------------------------------------------------------------
 def cpu_threads() -> int:
     try:
@@ -538,6 +634,8 @@ def main(argv=None):
                     help="predict layer l+1's neuron set from layer l's input (DejaVu look-ahead)")
     ap.add_argument("--true-mask", action="store_true",
                     help="time the sparse FFN alone on each token's true activation set (no predictor)")
+    ap.add_argument("--dense", action="store_true",
+                    help="comparison arm: the dense FFN of every layer with cuBLAS on the same weights")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -551,6 +649,8 @@ def main(argv=None):
         res, show = run_reference(args, cfg, world, rank, local)
     elif args.true_mask:
         res, show = run_true_mask(args, cfg, world, rank, local)
+    elif args.dense:
+        res, show = run_dense(args, cfg, world, rank, local)
     else:
         res, show = run_ours(args, cfg, world, rank, local)
         if show and world == 1 and not args.no_cpu_baseline:

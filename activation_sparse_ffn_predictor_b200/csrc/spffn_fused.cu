@@ -1188,9 +1188,10 @@ Geometry geometry(const spffn_config& c, int G, bool lookahead, bool tables = fa
     fixed += (2 * 4 * 8 + 2 * 8 * 2 * NB) * 4 + 8 * NB * 4 + 32 * 8 * NB * 4 + 16 * 4 + 16;
     fixed += 8 * (2 * 8 + 2 * 8) + 8 * 8 + 128;                      // barriers + flags + slack
     const size_t fslot = 4 * (size_t)c.d + 128;
-    // look-ahead gathers a layer's FFN rows while the previous layer still runs, so
-    // it trades a predictor slot for more FFN slots
-    g.pred_slots = tables ? 1 : (lookahead ? 3 : 4);     // no predictor weights to stream with tables
+    // three predictor slots feed the logits GEMV as fast as four (its chunk rate is set
+    // inside the SM), so the rest of shared memory goes to FFN slots: more of a CTA's
+    // rows are resident when its list is final.  Caller tables stream no predictor.
+    g.pred_slots = tables ? 1 : 3;
     g.ffn_slots = (tables || lookahead) ? 10 : 8;
     auto total = [&]() { return fixed + (size_t)g.pred_slots * g.pred_slot_bytes + g.ffn_slots * fslot; };
     while (total() > (size_t)budget && g.ffn_slots > 3) --g.ffn_slots;

@@ -116,9 +116,9 @@ def dense_bytes_per_layer(cfg) -> int:
 # captured on: any change to them and the bench reports null.
 DECODE_SOURCES = ("spffn_fused.cu", "spffn_fused.cuh", "spffn_internal.cuh")
 DECODE_TRAFFIC = {
-    "sha256": "5f09df9818cc796c3d3a84b55a3f382c3dc1e04be6deb42743f4b9b4eeab11db",
+    "sha256": "6f268d5aef86e990c15ff3378f4bd60f66b74f64e42b4ac044f1d523b2d384b7",
     "workload": "opt6.7b-d4096-n16384-L32", "batch": 1, "rate": 0.05,
-    "bytes_per_layer": (223.219712e6 + 6.285056e6) / 4,
+    "bytes_per_layer": (223.223808e6 + 4.954112e6) / 4,
     "summary": "profiles/k_decode_opt6.7b-d4096-n16384_b1.md",
 }
 

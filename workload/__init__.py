@@ -39,6 +39,8 @@ SEED = 20241208
 
 # Stream ids: (layer << 32) | (tensor << 24) | aux.
 T_W1, T_W2T, T_WP1, T_WP2, T_X, T_XPROF, T_PERM, T_Y = 1, 2, 3, 4, 5, 6, 7, 8
+# attention layers: projections, output projection (head-major), head predictor, tokens
+T_WQ, T_WK, T_WV, T_WOT, T_WA1, T_WA2, T_XA = 9, 10, 11, 12, 13, 14, 15
 
 PMAX = 0.99
 RELU_MEAN = 1.0 / math.sqrt(2.0 * math.pi)
@@ -373,3 +375,112 @@ def to_torch(bits: np.ndarray, cfg: FFNConfig, device="cuda"):
     import torch
     t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(_torch_dtype(cfg))
     return t.to(device)
+
+
+# ---------------------------------------------------------------------------
+# attention layers with an attention-head predictor
+@dataclass(frozen=True)
+class AttnConfig:
+    """Shape of a synthetic attention stack: d model width, nh heads of width dh,
+    Ha predictor hidden units, per-head selection rate, tokens already in the
+    cache before timing (context) and cache capacity (tmax)."""
+    name: str
+    layers: int
+    d: int
+    nh: int
+    dh: int
+    Ha: int
+    dtype: str
+    rate: float
+    context: int
+    tmax: int
+
+    @property
+    def bf16(self) -> int:
+        return 1 if self.dtype == "bf16" else 0
+
+    def with_(self, **kw) -> "AttnConfig":
+        return replace(self, **kw)
+
+
+# A small block and the OPT-66B attention shape (72 heads of 128), with the head
+# rate of about 20% the DejaVu appendix reports.
+ATTN_CONFIGS = {
+    0: AttnConfig("attn-d1024-h16", 1, 1024, 16, 64, 256, "f16", 0.25, 24, 64),
+    1: AttnConfig("attn-opt66b-d9216-h72-L64", 64, 9216, 72, 128, 1024, "f16", 0.20, 1024, 1280),
+}
+
+
+@dataclass
+class HostAttn:
+    """One attention layer's weights as storage bits; biases of Q/K/V/O are zero."""
+    cfg: AttnConfig
+    layer: int
+    Wq: np.ndarray
+    Wk: np.ndarray
+    Wv: np.ndarray
+    WoT: np.ndarray
+    Wa1: np.ndarray
+    Wa2: np.ndarray
+    ba2: np.ndarray
+
+    def f64(self, name: str) -> np.ndarray:
+        return widen(getattr(self, name), self.cfg.bf16)
+
+
+def attn_head_bias(cfg: AttnConfig, Wa2: np.ndarray) -> np.ndarray:
+    """ba2 calibrated like the FFN predictor's so each head is selected at ``rate``."""
+    s1, s2 = row_stats(Wa2, cfg.bf16)
+    return predictor_bias(s1, s2, np.full(cfg.nh, cfg.rate), cfg.bf16)
+
+
+def host_attn(cfg: AttnConfig, layer: int = 0, seed: int = SEED) -> HostAttn:
+    bf, rows = cfg.bf16, cfg.nh * cfg.dh
+    sd = 1.0 / math.sqrt(cfg.d)
+    m = lambda t, r, c, sc: fill(stream_id(t, layer), r * c, sc, bf, seed=seed).reshape(r, c)
+    Wa2 = m(T_WA2, cfg.nh, cfg.Ha, 1.0 / math.sqrt(cfg.Ha))
+    return HostAttn(cfg, layer, m(T_WQ, rows, cfg.d, sd), m(T_WK, rows, cfg.d, sd), m(T_WV, rows, cfg.d, sd),
+                    m(T_WOT, rows, cfg.d, 1.0 / math.sqrt(rows)), m(T_WA1, cfg.Ha, cfg.d, sd), Wa2,
+                    attn_head_bias(cfg, Wa2))
+
+
+def attn_rows(cfg: AttnConfig, tensor: int, layer: int, rows, seed: int = SEED) -> np.ndarray:
+    """Storage bits of the given rows of one projection ([len(rows), d])."""
+    sc = 1.0 / math.sqrt(cfg.nh * cfg.dh) if tensor == T_WOT else 1.0 / math.sqrt(cfg.d)
+    return fill_rows(stream_id(tensor, layer), cfg.d, np.asarray(rows, dtype=np.int64), sc, cfg.bf16, seed)
+
+
+@dataclass
+class DeviceAttn:
+    Wq: object
+    Wk: object
+    Wv: object
+    WoT: object
+    Wa1: object
+    Wa2: object
+    ba2: object
+
+
+def device_attn(cfg: AttnConfig, layer: int, device="cuda", seed: int = SEED) -> DeviceAttn:
+    """Fill one attention layer directly in HBM with the same bits host_attn gives."""
+    import torch
+    dt = _torch_dtype(cfg)
+    bf, rows = cfg.bf16, cfg.nh * cfg.dh
+    sd = 1.0 / math.sqrt(cfg.d)
+    e = lambda r, c: torch.empty(r, c, dtype=dt, device=device)
+    out = DeviceAttn(e(rows, cfg.d), e(rows, cfg.d), e(rows, cfg.d), e(rows, cfg.d), e(cfg.Ha, cfg.d),
+                     e(cfg.nh, cfg.Ha), torch.empty(cfg.nh, dtype=dt, device=device))
+    device_fill(out.Wq, stream_id(T_WQ, layer), sd, bf, seed)
+    device_fill(out.Wk, stream_id(T_WK, layer), sd, bf, seed)
+    device_fill(out.Wv, stream_id(T_WV, layer), sd, bf, seed)
+    device_fill(out.WoT, stream_id(T_WOT, layer), 1.0 / math.sqrt(rows), bf, seed)
+    device_fill(out.Wa1, stream_id(T_WA1, layer), sd, bf, seed)
+    device_fill(out.Wa2, stream_id(T_WA2, layer), 1.0 / math.sqrt(cfg.Ha), bf, seed)
+    s1, s2 = device_row_stats(out.Wa2, bf)
+    out.ba2.copy_(torch.from_numpy(predictor_bias(s1, s2, np.full(cfg.nh, cfg.rate), bf).view(np.int16)).view(dt))
+    return out
+
+
+def attn_tokens(cfg: AttnConfig, T: int, aux: int, layer: int = 0, seed: int = SEED) -> np.ndarray:
+    """[T, d] storage bits of N(0,1) attention inputs."""
+    return fill(stream_id(T_XA, layer, aux), T * cfg.d, 1.0, cfg.bf16, seed=seed).reshape(T, cfg.d)

@@ -17,8 +17,9 @@ import numpy as np
 
 from . import build as _build
 
-__all__ = ["SpffnError", "Layer", "decode", "decode_tables", "decode_kernel_launches", "forward_noalloc",
+__all__ = ["SpffnError", "Layer", "AttnLayer", "attn_step_kernel_launches", "decode", "decode_tables", "decode_kernel_launches", "forward_noalloc",
            "reorder", "reorder_dealt", "permute_rows", "permute_vector", "set_trace", "trace_marks",
+           "set_l2_hot_rows", "l2_hot_rows", "set_union_stack", "union_stack",
            "workspace_bytes", "library", "F16", "BF16"]
 
 F16, BF16 = 0, 1
@@ -29,7 +30,10 @@ EXPORTS = ("spffn_workspace_bytes", "spffn_create", "spffn_destroy", "spffn_pred
            "spffn_permute_rows", "spffn_permute_vector", "spffn_last_device_error", "spffn_status_string",
            "spffn_num_partials", "spffn_decode_kernel_launches", "spffn_set_trace", "spffn_trace_marks",
            "spffn_last_cuda_error_string", "spffn_reorder_dealt", "spffn_forward_noalloc",
-           "spffn_decode_lookahead", "spffn_layer_table", "spffn_decode_tables")
+           "spffn_decode_lookahead", "spffn_layer_table", "spffn_decode_tables", "spffn_set_wait_test", "spffn_set_l2_hot_rows", "spffn_l2_hot_rows",
+           "spffn_set_union_stack", "spffn_union_stack",
+           "spffn_attn_workspace_bytes", "spffn_attn_create", "spffn_attn_destroy", "spffn_attn_reset",
+           "spffn_attn_step", "spffn_attn_cache", "spffn_attn_step_kernel_launches", "spffn_attn_last_device_error")
 
 
 class SpffnError(RuntimeError):
@@ -45,6 +49,21 @@ class Config(ctypes.Structure):
 
 class Weights(ctypes.Structure):
     _fields_ = [(k, ctypes.c_void_p) for k in ("W1", "b1", "W2T", "b2", "Wp1", "bp1", "Wp2", "bp2")]
+
+
+class AttnConfig(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("nh", ctypes.c_int32), ("dh", ctypes.c_int32), ("Ha", ctypes.c_int32),
+                ("tmax", ctypes.c_int32), ("dtype", ctypes.c_int32), ("flags", ctypes.c_uint32)]
+
+
+class AttnWeights(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_void_p) for k in ("Wq", "bq", "Wk", "bk", "Wv", "bv", "WoT", "bo", "Wa1", "ba1",
+                                                "Wa2", "ba2")]
+
+
+class AttnCacheView(ctypes.Structure):
+    _fields_ = [("K", ctypes.c_void_p), ("V", ctypes.c_void_p), ("filled", ctypes.c_void_p), ("Y", ctypes.c_void_p),
+                ("t", ctypes.c_void_p)]
 
 
 _lib = None
@@ -88,8 +107,21 @@ def library(path: Optional[str] = None):
         "spffn_num_partials": (i32, [vp]),
         "spffn_decode_kernel_launches": (i32, [ctypes.POINTER(vp), i32, i32]),
         "spffn_set_trace": (st, [vp, sz]),
+        "spffn_set_wait_test": (st, [ctypes.c_uint64, i32]),
+        "spffn_set_l2_hot_rows": (st, [i32]),
+        "spffn_set_union_stack": (st, [i32]),
+        "spffn_union_stack": (i32, []),
+        "spffn_l2_hot_rows": (i32, []),
         "spffn_trace_marks": (i32, []),
         "spffn_last_cuda_error_string": (ctypes.c_char_p, []),
+        "spffn_attn_workspace_bytes": (sz, [ctypes.POINTER(AttnConfig)]),
+        "spffn_attn_create": (st, [ctypes.POINTER(AttnConfig), ctypes.POINTER(AttnWeights), vp, sz, ctypes.POINTER(vp)]),
+        "spffn_attn_destroy": (st, [vp]),
+        "spffn_attn_reset": (st, [vp, vp]),
+        "spffn_attn_step": (st, [vp, vp, vp, vp, vp, vp]),
+        "spffn_attn_cache": (st, [vp, ctypes.POINTER(AttnCacheView)]),
+        "spffn_attn_step_kernel_launches": (i32, []),
+        "spffn_attn_last_device_error": (st, [vp, ctypes.POINTER(ctypes.c_uint32), vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -228,6 +260,83 @@ class Layer:
         return s, int(code.value)
 
 
+class AttnLayer:
+    """One attention layer with its head predictor (wraps an ``spffn_attn_ctx``).
+
+    Weight tensors (CUDA, row-major, float16 or bfloat16): ``Wq, Wk, Wv[nh*dh, d]``,
+    ``WoT[nh*dh, d]`` (output projection stored head-major), ``Wa1[Ha, d]``,
+    ``Wa2[nh, Ha]``; biases ``bq, bk, bv[nh*dh]``, ``bo[d]``, ``ba1[Ha]``,
+    ``ba2[nh]`` or None.  The workspace (cache included) is a zero-filled uint8
+    CUDA tensor, allocated here when not given.
+    """
+
+    def __init__(self, Wq, Wk, Wv, WoT, Wa1, Wa2, nh: int, tmax: int, bq=None, bk=None, bv=None, bo=None,
+                 ba1=None, ba2=None, workspace=None):
+        import torch
+        rows, d = Wq.shape
+        self.d, self.nh, self.dh, self.Ha, self.tmax = int(d), int(nh), int(rows) // int(nh), int(Wa1.shape[0]), int(tmax)
+        self.dtype = _dtype_code(Wq)
+        self.cfg = AttnConfig(self.d, self.nh, self.dh, self.Ha, self.tmax, self.dtype, 0)
+        self._keep = [Wq, bq, Wk, bk, Wv, bv, WoT, bo, Wa1, ba1, Wa2, ba2]
+        self.weights = AttnWeights(*[_p(t) for t in self._keep])
+        need = int(library().spffn_attn_workspace_bytes(ctypes.byref(self.cfg)))
+        if need == 0:
+            raise SpffnError(ERR_INVALID_ARG, "spffn_attn_workspace_bytes (bad shape)")
+        if workspace is None:
+            workspace = torch.zeros(need, dtype=torch.uint8, device=Wq.device)
+        self.workspace = workspace
+        ctx = ctypes.c_void_p()
+        _check(library().spffn_attn_create(ctypes.byref(self.cfg), ctypes.byref(self.weights), _p(workspace),
+                                           workspace.numel(), ctypes.byref(ctx)), "spffn_attn_create")
+        self.ctx = ctx
+
+    def close(self):
+        if getattr(self, "ctx", None):
+            library().spffn_attn_destroy(self.ctx)
+            self.ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def step(self, y, heads, count, out, stream=None):
+        """One decode step: y [d] -> out [d] (fp32); heads [nh], count [1] (int32)."""
+        _check(library().spffn_attn_step(self.ctx, _p(y), _p(heads), _p(count), _p(out), _stream(stream)),
+               "spffn_attn_step")
+
+    def reset(self, stream=None):
+        _check(library().spffn_attn_reset(self.ctx, _stream(stream)), "spffn_attn_reset")
+
+    def cache(self):
+        """(K, V, filled, Y, t) views of the cache as torch tensors on the workspace."""
+        import torch
+        v = AttnCacheView()
+        _check(library().spffn_attn_cache(self.ctx, ctypes.byref(v)), "spffn_attn_cache")
+        base = self.workspace.data_ptr()
+        dt = torch.bfloat16 if self.dtype == BF16 else torch.float16
+        def view(ptr, nbytes):
+            off = int(ptr) - base
+            return self.workspace[off:off + nbytes]
+        kv = self.nh * self.tmax * self.dh
+        K = view(v.K, 2 * kv).view(dt).view(self.nh, self.tmax, self.dh)
+        V = view(v.V, 2 * kv).view(dt).view(self.nh, self.tmax, self.dh)
+        filled = view(v.filled, self.nh * self.tmax).view(self.nh, self.tmax)
+        Y = view(v.Y, 2 * self.tmax * self.d).view(dt).view(self.tmax, self.d)
+        t = view(v.t, 4).view(torch.int32)
+        return K, V, filled, Y, t
+
+    def last_device_error(self, stream=None):
+        code = ctypes.c_uint32(0)
+        s = library().spffn_attn_last_device_error(self.ctx, ctypes.byref(code), _stream(stream))
+        return s, int(code.value)
+
+
+def attn_step_kernel_launches() -> int:
+    return int(library().spffn_attn_step_kernel_launches())
+
+
 def forward_noalloc(layer: Layer, x, idx, count, y, stream=None):
     """spffn_forward for `layer`'s weights without its context or workspace
     (scratch in the library's fixed device array; see include/spffn.h)."""
@@ -270,6 +379,27 @@ def set_trace(buf=None):
 
 def trace_marks() -> int:
     return int(library().spffn_trace_marks())
+
+
+def set_l2_hot_rows(rows_per_range: int):
+    """Keep the first ``rows_per_range`` slots of every dealt range (the hottest
+    neurons after the hot-first dealt placement) in L2 during small-batch decode
+    (spffn_set_l2_hot_rows; 0 turns the cache hints off)."""
+    _check(library().spffn_set_l2_hot_rows(int(rows_per_range)), "spffn_set_l2_hot_rows")
+
+
+def l2_hot_rows() -> int:
+    return int(library().spffn_l2_hot_rows())
+
+
+def set_union_stack(enable: bool):
+    """Whole-stack persistent launch (True, the default) or per-layer launches for
+    decode at 3 <= B <= 128 (spffn_set_union_stack)."""
+    _check(library().spffn_set_union_stack(1 if enable else 0), "spffn_set_union_stack")
+
+
+def union_stack() -> bool:
+    return bool(library().spffn_union_stack())
 
 
 def reorder(counts: np.ndarray) -> np.ndarray:

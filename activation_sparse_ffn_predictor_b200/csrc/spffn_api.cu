@@ -161,6 +161,8 @@ spffn_status decode_impl(spffn_ctx* const* layers, int32_t L, const void* x_in, 
     cudaStream_t st = (cudaStream_t)stream;
     if (fused_decode_supported(layers, L, B))
         return cuda_status(launch_fused_decode(layers, L, x_in, B, x_out, y, counts, lookahead, st));
+    if (!lookahead && ustack_supported(layers, L, B))
+        return cuda_status(launch_ustack(layers, L, x_in, B, x_out, y, counts, st));
     const void* xcur = x_in;
     cudaError_t e = cudaSuccess;
     if (lookahead) {
@@ -247,7 +249,7 @@ int32_t spffn_decode_kernel_launches(spffn_ctx* const* layers, int32_t L, int32_
     if (!layers || L < 1 || !layers[0] || B < 1 || B > layers[0]->cfg.max_batch) return 0;
     for (int l = 0; l < L; ++l)
         if (!layers[l]) return 0;
-    if (fused_decode_supported(layers, L, B)) return 1;
+    if (fused_decode_supported(layers, L, B) || ustack_supported(layers, L, B)) return 1;
     // per layer: predictor hidden, logits (per token group), compaction, FC1, FC2 (per group), chaining
     int n = 0;
     for (int l = 0; l < L; ++l) {
@@ -263,6 +265,26 @@ spffn_status spffn_set_trace(void* buf, size_t bytes) {
 }
 
 int32_t spffn_trace_marks(void) { return trace_marks(); }
+
+spffn_status spffn_set_union_stack(int32_t enable) {
+    set_ustack(enable != 0);
+    return SPFFN_OK;
+}
+
+int32_t spffn_union_stack(void) { return ustack_enabled() ? 1 : 0; }
+
+spffn_status spffn_set_l2_hot_rows(int32_t rows_per_range) {
+    if (rows_per_range < 0) return SPFFN_ERR_INVALID_ARG;
+    set_l2_hot_rows(rows_per_range);
+    return SPFFN_OK;
+}
+
+int32_t spffn_l2_hot_rows(void) { return l2_hot_rows(); }
+
+spffn_status spffn_set_wait_test(uint64_t limit_ns, int32_t unmeetable_barrier) {
+    set_wait_test((unsigned long long)limit_ns, unmeetable_barrier != 0);
+    return SPFFN_OK;
+}
 
 spffn_status spffn_profile_counts(spffn_ctx* ctx, const void* X, int32_t T, uint32_t* counts, void* stream) {
     if (!ctx || !X || !counts || T < 1 || !aligned16(X)) return SPFFN_ERR_INVALID_ARG;

@@ -1,0 +1,552 @@
+// Head-sparse attention decode with DejaVu's attention-head predictor (SP_A),
+// the attention half of equation (-1) in the DejaVu appendix of
+// "LLM模型之PowerInfer1.0": S_A <- SP_A(y), y~ <- MHA restricted to S_A, with
+// the page's handling of KV-cache misses (a head selected after being skipped
+// computes its missing K/V rows from the stored inputs of the past tokens).
+//
+// One step of one layer, one token, six launches on the caller's stream:
+//   1 SP_A hidden layer h = ReLU(Wa1 y + ba1)                 (the predictor GEMV kernel)
+//   2 head logits, threshold, ascending head list; y stored as Y[t]; for every
+//     selected head the list of positions p < t whose K/V rows are missing
+//   3 q, k, v rows of the selected heads for the new token, and the missing K/V
+//     rows from Y[p] (each weight row streamed once, reused from L1/L2 for the
+//     missing positions)
+//   4 attention per selected head over positions 0..t, split over CTAs with an
+//     online softmax in fixed position order, the splits combined in fixed
+//     order by the last CTA of the head (atomic ticket)
+//   5 output projection: each CTA accumulates o_k[i] WoT[k dh + i] over an equal
+//     share of the selected heads' rows into its own fp32 partial
+//   6 out = bo + the partials in fixed order; t = t + 1 (the position lives on
+//     the device, so a step replays in a CUDA graph)
+// Weight bytes dominate (Wa1, the selected heads' Wq/Wk/Wv/Wo rows, then the
+// cached K/V rows): every kernel streams rows with 16-byte loads.
+#include <cstring>
+#include <new>
+#include "spffn_internal.cuh"
+#include "spffn_kernels.cuh"
+#include "../../include/spffn_attn.h"
+
+namespace spffn {
+
+struct ALayout {
+    size_t ctl, h, q, miss, nmiss, opart, o, ypart, tickets, K, V, filled, Y, total;
+    int S, Sa;
+};
+
+inline ALayout attn_layout(const spffn_attn_config& c, int S) {
+    ALayout L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
+    L.S = S;
+    L.Sa = 8;                                                   // position splits per head
+    L.ctl = take(256);                                          // [0] error word, [1] t
+    L.h = take((size_t)c.Ha * sizeof(float));
+    L.q = take((size_t)c.nh * c.dh * sizeof(float));
+    L.miss = take((size_t)c.nh * c.tmax * sizeof(uint16_t));    // per head slot: missing positions
+    L.nmiss = take((size_t)c.nh * sizeof(int32_t));
+    L.opart = take((size_t)c.nh * L.Sa * (c.dh + 2) * sizeof(float));
+    L.o = take((size_t)c.nh * c.dh * sizeof(float));
+    L.ypart = take((size_t)S * c.d * sizeof(float));
+    L.tickets = take((size_t)c.nh * sizeof(uint32_t));
+    L.K = take((size_t)c.nh * c.tmax * c.dh * 2);
+    L.V = take((size_t)c.nh * c.tmax * c.dh * 2);
+    L.filled = take((size_t)c.nh * c.tmax);
+    L.Y = take((size_t)c.tmax * c.d * 2);
+    L.total = off;
+    return L;
+}
+
+struct AParams {
+    const void *Wq, *bq, *Wk, *bk, *Wv, *bv, *WoT, *bo, *Wa2, *ba2;
+    const void* y;
+    int d, nh, dh, Ha, tmax, Sa;
+    int32_t* tcur;
+    int32_t* heads;
+    int32_t* count;
+    uint32_t* err;
+    const float* h;
+    float* q;
+    uint16_t* miss;
+    int32_t* nmiss;
+    float* opart;
+    float* o;
+    float* ypart;
+    uint32_t* tickets;
+    void* K;
+    void* V;
+    uint8_t* filled;
+    void* Y;
+    float* out;
+};
+
+namespace {
+
+template <typename T>
+__device__ __forceinline__ float dot8(const uint4& w, const uint4& x) {
+    float a[8], b[8];
+    unpack8<T>(w, a);
+    unpack8<T>(x, b);
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s = fmaf(a[i], b[i], s);
+    return s;
+}
+
+// ---------------------------------------------------------------------------
+// 2: head logits l_k = Wa2[k] . h + ba2_k, selection l_k > 0, ascending list; Y[t] = y;
+// per selected head the positions p < t with no K/V row yet.  One CTA.
+template <typename T>
+__global__ void __launch_bounds__(256) k_attn_select(const AParams p)
+{
+    __shared__ unsigned char sel[1024];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t = *p.tcur;
+    const bool full = t >= p.tmax;
+    if (!full) {
+        const uint4* src = reinterpret_cast<const uint4*>(p.y);
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.Y) + (size_t)t * p.d);
+        for (int v = tid; v < p.d / 8; v += 256) dst[v] = src[v];
+    }
+    const int hv = p.Ha / 8;
+    for (int k = warp; k < p.nh; k += 8) {
+        const uint4* w = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.Wa2) + (size_t)k * p.Ha);
+        float acc = 0.f;
+        for (int v = lane; v < hv; v += 32) {
+            float wf[8];
+            unpack8<T>(ldg_stream(w + v), wf);
+            const float4 a = reinterpret_cast<const float4*>(p.h)[2 * v], b = reinterpret_cast<const float4*>(p.h)[2 * v + 1];
+            acc = fmaf(wf[0], a.x, acc); acc = fmaf(wf[1], a.y, acc); acc = fmaf(wf[2], a.z, acc); acc = fmaf(wf[3], a.w, acc);
+            acc = fmaf(wf[4], b.x, acc); acc = fmaf(wf[5], b.y, acc); acc = fmaf(wf[6], b.z, acc); acc = fmaf(wf[7], b.w, acc);
+        }
+        acc = warp_sum(acc);
+        const float bias = p.ba2 ? DT<T>::f(reinterpret_cast<const T*>(p.ba2)[k]) : 0.f;
+        if (lane == 0) sel[k] = !full && (acc + bias) > 0.f;
+    }
+    __syncthreads();
+    __shared__ int s_count;
+    if (warp == 0) {
+        int m = 0;
+        for (int k0 = 0; k0 < p.nh; k0 += 32) {
+            const bool on = k0 + lane < p.nh && sel[k0 + lane];
+            const uint32_t bal = __ballot_sync(0xffffffffu, on);
+            if (on) p.heads[m + __popc(bal & ((1u << lane) - 1u))] = k0 + lane;
+            m += __popc(bal);
+        }
+        if (lane == 0) {
+            *p.count = m;
+            s_count = m;
+            if (full) latch(p.err, ERR_CACHE_FULL);
+        }
+    }
+    __syncthreads();
+    // missing K/V rows of each selected head (one warp per head, ascending positions)
+    for (int s = warp; s < s_count; s += 8) {
+        const int h = p.heads[s];
+        const uint8_t* f = p.filled + (size_t)h * p.tmax;
+        uint16_t* ml = p.miss + (size_t)s * p.tmax;
+        int m = 0;
+        for (int p0 = 0; p0 < t; p0 += 32) {
+            const bool on = p0 + lane < t && !f[p0 + lane];
+            const uint32_t bal = __ballot_sync(0xffffffffu, on);
+            if (on) ml[m + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)(p0 + lane);
+            m += __popc(bal);
+        }
+        if (lane == 0) p.nmiss[s] = m;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 3: q, k, v rows of the selected heads for the new token; missing K/V rows from Y[p].
+// Work items: (head slot, block of 8 rows of the 3 dh rows q | k | v), one row per
+// warp; each CTA takes a contiguous range of items so consecutive items share a head.
+template <typename T>
+__global__ void __launch_bounds__(256) k_attn_qkv(const AParams p)
+{
+    extern __shared__ uint4 ys[];                      // the new token, d / 8 vectors
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t = *p.tcur, count = *p.count;
+    if (t >= p.tmax || count == 0) return;
+    const int nv = p.d / 8;
+    for (int v = tid; v < nv; v += 256) ys[v] = reinterpret_cast<const uint4*>(p.y)[v];
+    __syncthreads();
+    const int iph = (3 * p.dh + 7) / 8;
+    const int items = count * iph;
+    const int i0 = (int)((long long)items * blockIdx.x / gridDim.x), i1 = (int)((long long)items * (blockIdx.x + 1) / gridDim.x);
+    T* Kc = reinterpret_cast<T*>(p.K);
+    T* Vc = reinterpret_cast<T*>(p.V);
+    const T* Yh = reinterpret_cast<const T*>(p.Y);
+    for (int it = i0; it < i1; ++it) {
+        const int s = it / iph, r = (it % iph) * 8 + warp;
+        if (r >= 3 * p.dh) continue;
+        const int h = p.heads[s], type = r / p.dh, i = r % p.dh;
+        const T* W = reinterpret_cast<const T*>(type == 0 ? p.Wq : (type == 1 ? p.Wk : p.Wv));
+        const T* b = reinterpret_cast<const T*>(type == 0 ? p.bq : (type == 1 ? p.bk : p.bv));
+        const size_t row = (size_t)h * p.dh + i;
+        const uint4* w = reinterpret_cast<const uint4*>(W + row * p.d);
+        const float bias = b ? DT<T>::f(b[row]) : 0.f;
+        float acc = 0.f;
+        for (int v = lane; v < nv; v += 32) acc += dot8<T>(__ldg(w + v), ys[v]);
+        acc = warp_sum(acc) + bias;
+        if (lane == 0) {
+            if (type == 0) p.q[(size_t)s * p.dh + i] = acc;
+            else (type == 1 ? Kc : Vc)[((size_t)h * p.tmax + t) * p.dh + i] = DT<T>::r(acc);
+        }
+        if (type == 0) continue;
+        // the head's missing rows at earlier positions, eight at a time (the weight row
+        // comes back from L1/L2 after its first pass)
+        const int nm = p.nmiss[s];
+        const uint16_t* ml = p.miss + (size_t)s * p.tmax;
+        for (int g0 = 0; g0 < nm; g0 += 8) {
+            const int ng = min(8, nm - g0);
+            float a[8];
+#pragma unroll
+            for (int g = 0; g < 8; ++g) a[g] = 0.f;
+            for (int v = lane; v < nv; v += 32) {
+                const uint4 wv = __ldg(w + v);
+#pragma unroll
+                for (int g = 0; g < 8; ++g)
+                    if (g < ng) a[g] += dot8<T>(wv, __ldg(reinterpret_cast<const uint4*>(Yh + (size_t)ml[g0 + g] * p.d) + v));
+            }
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+                if (g < ng) {
+                    const float z = warp_sum(a[g]) + bias;
+                    if (lane == 0) (type == 1 ? Kc : Vc)[((size_t)h * p.tmax + ml[g0 + g]) * p.dh + i] = DT<T>::r(z);
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 4: o_k = softmax(q . K / sqrt(dh)) V over positions 0..t for every selected head.
+// Items (head slot, split of the positions); each warp walks its positions in order
+// with an online softmax (running max, sum and weighted V); the CTA's warps and then
+// the head's splits are combined in fixed order.  Marks the rows used as filled.
+template <typename T>
+__global__ void __launch_bounds__(256) k_attn_core(const AParams p)
+{
+    __shared__ float qs[256];
+    __shared__ float wm[8], wz[8];
+    __shared__ float wo[8][256];
+    __shared__ int s_last;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t = *p.tcur, count = *p.count;
+    if (t >= p.tmax || count == 0) return;
+    const int T_ = t + 1, dh = p.dh, Sa = p.Sa;
+    const int E = (dh + 31) / 32;                      // elements per lane (dh <= 256: E <= 8)
+    const float scale = 1.0f / sqrtf((float)dh);
+    const T* Kc = reinterpret_cast<const T*>(p.K);
+    const T* Vc = reinterpret_cast<const T*>(p.V);
+    for (int it = blockIdx.x; it < count * Sa; it += gridDim.x) {
+        const int s = it / Sa, sp = it % Sa, h = p.heads[s];
+        const int p0 = (int)((long long)T_ * sp / Sa), p1 = (int)((long long)T_ * (sp + 1) / Sa);
+        __syncthreads();
+        for (int e = tid; e < dh; e += 256) qs[e] = p.q[(size_t)s * dh + e];
+        __syncthreads();
+        float m = -INFINITY, z = 0.f, o[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = 0.f;
+        for (int pos = p0 + warp; pos < p1; pos += 8) {
+            const T* kr = Kc + ((size_t)h * p.tmax + pos) * dh;
+            const T* vr = Vc + ((size_t)h * p.tmax + pos) * dh;
+            float part = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int c = lane * E + e;
+                if (e < E && c < dh) part = fmaf(qs[c], DT<T>::f(kr[c]), part);
+            }
+            const float sc = warp_sum(part) * scale;
+            const float mn = fmaxf(m, sc);
+            const float cf = expf(m - mn), ef = expf(sc - mn);
+            z = z * cf + ef;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int c = lane * E + e;
+                if (e < E && c < dh) o[e] = o[e] * cf + ef * DT<T>::f(vr[c]);
+            }
+            m = mn;
+        }
+        if (lane == 0) { wm[warp] = m; wz[warp] = z; }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int c = lane * E + e;
+            if (e < E && c < dh) wo[warp][c] = o[e];
+        }
+        for (int pos = p0 + tid; pos < p1; pos += 256) p.filled[(size_t)h * p.tmax + pos] = 1;
+        __syncthreads();
+        // this split: combine the warps in order
+        float* part = p.opart + ((size_t)s * Sa + sp) * (dh + 2);
+        if (tid == 0) {
+            float M = -INFINITY;
+            for (int w = 0; w < 8; ++w) if (wz[w] > 0.f) M = fmaxf(M, wm[w]);
+            float Z = 0.f;
+            for (int w = 0; w < 8; ++w) if (wz[w] > 0.f) Z += wz[w] * expf(wm[w] - M);
+            part[0] = M;
+            part[1] = Z;
+        }
+        for (int c = tid; c < dh; c += 256) {
+            float M = -INFINITY;
+            for (int w = 0; w < 8; ++w) if (wz[w] > 0.f) M = fmaxf(M, wm[w]);
+            float O = 0.f;
+            for (int w = 0; w < 8; ++w) if (wz[w] > 0.f) O += wo[w][c] * expf(wm[w] - M);
+            part[2 + c] = O;
+        }
+        // the head's last split to finish combines all splits in order
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) s_last = atomicAdd(&p.tickets[s], 1u) == (uint32_t)(Sa - 1);
+        __syncthreads();
+        if (s_last) {
+            __threadfence();
+            const float* pa = p.opart + (size_t)s * Sa * (dh + 2);
+            float M = -INFINITY;
+            for (int q = 0; q < Sa; ++q) {
+                const float zq = __ldcg(pa + (size_t)q * (dh + 2) + 1);
+                if (zq > 0.f) M = fmaxf(M, __ldcg(pa + (size_t)q * (dh + 2)));
+            }
+            float Z = 0.f;
+            for (int q = 0; q < Sa; ++q) {
+                const float zq = __ldcg(pa + (size_t)q * (dh + 2) + 1);
+                if (zq > 0.f) Z += zq * expf(__ldcg(pa + (size_t)q * (dh + 2)) - M);
+            }
+            for (int c = tid; c < dh; c += 256) {
+                float O = 0.f;
+                for (int q = 0; q < Sa; ++q) {
+                    const float zq = __ldcg(pa + (size_t)q * (dh + 2) + 1);
+                    if (zq > 0.f) O += __ldcg(pa + (size_t)q * (dh + 2) + 2 + c) * expf(__ldcg(pa + (size_t)q * (dh + 2)) - M);
+                }
+                p.o[(size_t)s * dh + c] = O / Z;
+            }
+            if (tid == 0) p.tickets[s] = 0u;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 5: output projection over the selected heads' rows of WoT (head-major, each row
+// contiguous): CTA c accumulates o_k[i] WoT[k dh + i] over rows [c R / G, (c+1) R / G)
+// of the R = count dh rows into its fp32 partial.  Thread tid owns 8-column vectors
+// tid + 256 m (d <= 16384).
+template <typename T>
+__global__ void __launch_bounds__(256) k_attn_out(const AParams p)
+{
+    constexpr int kM = 8;
+    const int tid = threadIdx.x, nv = p.d / 8, G = gridDim.x, c = blockIdx.x;
+    const int t = *p.tcur;
+    const int count = t < p.tmax ? *p.count : 0;
+    const int R = count * p.dh;
+    const int r0 = (int)((long long)R * c / G), r1 = (int)((long long)R * (c + 1) / G);
+    float acc[kM][8];
+#pragma unroll
+    for (int m = 0; m < kM; ++m)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[m][e] = 0.f;
+    for (int r = r0; r < r1; ++r) {
+        const int s = r / p.dh, i = r % p.dh, h = p.heads[s];
+        const float a = p.o[(size_t)s * p.dh + i];
+        const uint4* w = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.WoT) + ((size_t)h * p.dh + i) * p.d);
+#pragma unroll
+        for (int m = 0; m < kM; ++m) {
+            const int v = tid + 256 * m;
+            if (v < nv) {
+                float wf[8];
+                unpack8<T>(ldg_stream(w + v), wf);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[m][e] = fmaf(a, wf[e], acc[m][e]);
+            }
+        }
+    }
+    float* dst = p.ypart + (size_t)c * p.d;
+#pragma unroll
+    for (int m = 0; m < kM; ++m) {
+        const int v = tid + 256 * m;
+        if (v < nv) {
+            __stcg(reinterpret_cast<float4*>(dst + v * 8), make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]));
+            __stcg(reinterpret_cast<float4*>(dst + v * 8) + 1, make_float4(acc[m][4], acc[m][5], acc[m][6], acc[m][7]));
+        }
+    }
+}
+
+// 6: out = bo + the G partials in fixed order; the position advances
+template <typename T>
+__global__ void __launch_bounds__(256) k_attn_reduce(const AParams p, int G)
+{
+    const int col = blockIdx.x * 256 + threadIdx.x;
+    if (col < p.d) {
+        float v = 0.f;
+        for (int g = 0; g < G; ++g) v += __ldcg(p.ypart + (size_t)g * p.d + col);
+        p.out[col] = v + (p.bo ? DT<T>::f(reinterpret_cast<const T*>(p.bo)[col]) : 0.f);
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        const int t = *p.tcur;
+        if (t < p.tmax) *p.tcur = t + 1;
+    }
+}
+
+bool aligned16(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; }
+
+bool valid(const spffn_attn_config* c) {
+    if (!c) return false;
+    if (c->d < 64 || c->d > 16384 || c->d % 64) return false;
+    if (c->nh < 1 || c->nh > 1024) return false;
+    if (c->dh < 8 || c->dh > 256 || c->dh % 8) return false;
+    if (c->Ha < 64 || c->Ha > 8192 || c->Ha % 64) return false;
+    if (c->tmax < 1 || c->tmax > 16384) return false;
+    if (c->dtype != SPFFN_F16 && c->dtype != SPFFN_BF16) return false;
+    return c->flags == 0;
+}
+
+int sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        n <= 0) {
+        cudaGetLastError();
+        return 148;
+    }
+    return n;
+}
+
+}  // namespace
+}  // namespace spffn
+
+struct spffn_attn_ctx {
+    spffn_attn_config cfg;
+    spffn_attn_weights w;
+    char* ws;
+    spffn::ALayout lay;
+};
+
+using namespace spffn;
+
+namespace {
+
+AParams attn_params(const spffn_attn_ctx& c, const void* y, int32_t* heads, int32_t* count, float* out) {
+    AParams p;
+    memset(&p, 0, sizeof(p));
+    const auto& w = c.w;
+    p.Wq = w.Wq; p.bq = w.bq; p.Wk = w.Wk; p.bk = w.bk; p.Wv = w.Wv; p.bv = w.bv; p.WoT = w.WoT; p.bo = w.bo;
+    p.Wa2 = w.Wa2; p.ba2 = w.ba2;
+    p.y = y;
+    p.d = c.cfg.d; p.nh = c.cfg.nh; p.dh = c.cfg.dh; p.Ha = c.cfg.Ha; p.tmax = c.cfg.tmax; p.Sa = c.lay.Sa;
+    uint32_t* ctl = reinterpret_cast<uint32_t*>(c.ws + c.lay.ctl);
+    p.err = ctl;
+    p.tcur = reinterpret_cast<int32_t*>(ctl + 1);
+    p.heads = heads;
+    p.count = count;
+    p.h = reinterpret_cast<const float*>(c.ws + c.lay.h);
+    p.q = reinterpret_cast<float*>(c.ws + c.lay.q);
+    p.miss = reinterpret_cast<uint16_t*>(c.ws + c.lay.miss);
+    p.nmiss = reinterpret_cast<int32_t*>(c.ws + c.lay.nmiss);
+    p.opart = reinterpret_cast<float*>(c.ws + c.lay.opart);
+    p.o = reinterpret_cast<float*>(c.ws + c.lay.o);
+    p.ypart = reinterpret_cast<float*>(c.ws + c.lay.ypart);
+    p.tickets = reinterpret_cast<uint32_t*>(c.ws + c.lay.tickets);
+    p.K = c.ws + c.lay.K;
+    p.V = c.ws + c.lay.V;
+    p.filled = reinterpret_cast<uint8_t*>(c.ws + c.lay.filled);
+    p.Y = c.ws + c.lay.Y;
+    p.out = out;
+    return p;
+}
+
+template <typename T>
+cudaError_t step_impl(const spffn_attn_ctx& c, const AParams& p, cudaStream_t st) {
+    const int G = c.lay.S;
+    cudaError_t e = launch_hidden(c.cfg.dtype, c.w.Wa1, c.w.ba1, p.y, 1, c.cfg.d, c.cfg.Ha,
+                                  reinterpret_cast<float*>(c.ws + c.lay.h), G, st);
+    if (e != cudaSuccess) return e;
+    k_attn_select<T><<<1, 256, 0, st>>>(p);
+    const size_t smem = (size_t)c.cfg.d * 2;
+    e = cudaFuncSetAttribute(k_attn_qkv<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k_attn_qkv<T><<<G, 256, smem, st>>>(p);
+    k_attn_core<T><<<G, 256, 0, st>>>(p);
+    k_attn_out<T><<<G, 256, 0, st>>>(p);
+    k_attn_reduce<T><<<(c.cfg.d + 255) / 256, 256, 0, st>>>(p, G);
+    return cudaGetLastError();
+}
+
+spffn_status status_of(cudaError_t e) { return e == cudaSuccess ? SPFFN_OK : SPFFN_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t spffn_attn_workspace_bytes(const spffn_attn_config* cfg) {
+    if (!valid(cfg)) return 0;
+    return attn_layout(*cfg, sms()).total;
+}
+
+spffn_status spffn_attn_create(const spffn_attn_config* cfg, const spffn_attn_weights* w, void* workspace,
+                               size_t workspace_bytes, spffn_attn_ctx** out) {
+    if (!out) return SPFFN_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!valid(cfg) || !w || !w->Wq || !w->Wk || !w->Wv || !w->WoT || !w->Wa1 || !w->Wa2) return SPFFN_ERR_INVALID_ARG;
+    const void* all[] = {w->Wq, w->bq, w->Wk, w->bk, w->Wv, w->bv, w->WoT, w->bo, w->Wa1, w->ba1, w->Wa2, w->ba2};
+    for (const void* q : all)
+        if (q && !aligned16(q)) return SPFFN_ERR_INVALID_ARG;
+    const ALayout lay = attn_layout(*cfg, sms());
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SPFFN_ERR_WORKSPACE;
+    if (workspace_bytes < lay.total) return SPFFN_ERR_WORKSPACE;
+    spffn_attn_ctx* c = new (std::nothrow) spffn_attn_ctx();
+    if (!c) return SPFFN_ERR_UNSUPPORTED;
+    c->cfg = *cfg;
+    c->w = *w;
+    c->ws = static_cast<char*>(workspace);
+    c->lay = lay;
+    *out = c;
+    return SPFFN_OK;
+}
+
+spffn_status spffn_attn_destroy(spffn_attn_ctx* ctx) {
+    delete ctx;
+    return SPFFN_OK;
+}
+
+spffn_status spffn_attn_reset(spffn_attn_ctx* ctx, void* stream) {
+    if (!ctx) return SPFFN_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaMemsetAsync(ctx->ws + ctx->lay.ctl + 4, 0, 4, st);                  // t = 0
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(ctx->ws + ctx->lay.filled, 0, (size_t)ctx->cfg.nh * ctx->cfg.tmax, st);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(ctx->ws + ctx->lay.tickets, 0, (size_t)ctx->cfg.nh * sizeof(uint32_t), st);
+    return status_of(e);
+}
+
+spffn_status spffn_attn_step(spffn_attn_ctx* ctx, const void* y, int32_t* heads, int32_t* count, float* out,
+                             void* stream) {
+    if (!ctx || !y || !heads || !count || !out) return SPFFN_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(out)) return SPFFN_ERR_INVALID_ARG;
+    const AParams p = attn_params(*ctx, y, heads, count, out);
+    cudaStream_t st = (cudaStream_t)stream;
+    return status_of(ctx->cfg.dtype == SPFFN_BF16 ? step_impl<__nv_bfloat16>(*ctx, p, st)
+                                                  : step_impl<__half>(*ctx, p, st));
+}
+
+spffn_status spffn_attn_cache(spffn_attn_ctx* ctx, spffn_attn_cache_view* view) {
+    if (!ctx || !view) return SPFFN_ERR_INVALID_ARG;
+    view->K = ctx->ws + ctx->lay.K;
+    view->V = ctx->ws + ctx->lay.V;
+    view->filled = reinterpret_cast<const uint8_t*>(ctx->ws + ctx->lay.filled);
+    view->Y = ctx->ws + ctx->lay.Y;
+    view->t = reinterpret_cast<const int32_t*>(ctx->ws + ctx->lay.ctl + 4);
+    return SPFFN_OK;
+}
+
+int32_t spffn_attn_step_kernel_launches(void) { return 6; }
+
+spffn_status spffn_attn_last_device_error(spffn_attn_ctx* ctx, uint32_t* code, void* stream) {
+    if (!ctx) return SPFFN_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t v = 0;
+    uint32_t* err = reinterpret_cast<uint32_t*>(ctx->ws + ctx->lay.ctl);
+    if (cudaMemcpyAsync(&v, err, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess) return SPFFN_ERR_CUDA;
+    if (cudaMemsetAsync(err, 0, sizeof(uint32_t), st) != cudaSuccess) return SPFFN_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SPFFN_ERR_CUDA;
+    if (code) *code = v;
+    return v ? SPFFN_ERR_DEVICE_CHECK : SPFFN_OK;
+}
+
+}  // extern "C"

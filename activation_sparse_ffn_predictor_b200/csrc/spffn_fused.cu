@@ -26,6 +26,7 @@
 // Every wait is bounded (globaltimer): on expiry the CTA latches an error,
 // raises a grid-wide abort flag, stops issuing copies, waits (bounded) for the
 // copies it already issued and returns.
+#include <cstring>
 #include "spffn_fused.cuh"
 
 namespace spffn {
@@ -38,7 +39,7 @@ constexpr int kThreads = kConsumers + 64;      // + predictor producer warp + FF
 constexpr int kMaxFusedLayers = 128;
 constexpr int kMaxVPT = 5;                      // 16-byte column vectors per consumer thread (d <= 10240)
 constexpr int kMaxG = 256;
-constexpr unsigned long long kWaitNs = 2000000000ull;   // 2 s per wait
+constexpr unsigned long long kWaitNs = 2000000000ull;   // 2 s per wait (grid barriers: p.wait_ns)
 constexpr int kTraceMarks = 16;                 // stamps per (CTA, layer), see TRACE() below
 constexpr int kMaxMaskWords = 2048;             // n <= 65536 on this path
 
@@ -63,6 +64,10 @@ struct Params {
     float* partial;       // [G][B][d]
     float* u;             // [B][d]
     int pred_slots, pred_slot_bytes, ffn_slots, R1, R2, max_rows;
+    unsigned long long wait_ns;  // limit of a grid-barrier wait (other waits: kWaitNs)
+    uint32_t bar_extra;          // arrivals a grid barrier expects beyond G (0; 1 only under the wait test)
+    int hot_rows;                // > 0: the first hot_rows slots of every dealt range stay in L2 (evict_last)
+                                 // and the predictor and the other FFN rows are copied evict_first
     unsigned long long* trace;   // optional [G][L][kTraceMarks] globaltimer stamps
     LayerW layer[kMaxFusedLayers];
 };
@@ -102,6 +107,32 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(sptr(dst)),
         "l"(src), "r"(bytes), "r"(sptr(bar))
         : "memory");
+}
+// the same with an L2 eviction-priority policy for the copied lines (createpolicy)
+__device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                              uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+        ::"r"(sptr(dst)), "l"(src), "r"(bytes), "r"(sptr(bar)), "l"(policy)
+        : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// offset of neuron slot j inside its dealt range (ranges c = [floor(n c / G), floor(n (c+1) / G)));
+// after the hot-first dealt placement, offset k holds the (k G + c)-th hottest neuron
+__device__ __forceinline__ int range_offset(int j, int n, int G) {
+    int c = (int)((long long)j * G / n);
+    while (c + 1 < G && (int)((long long)n * (c + 1) / G) <= j) ++c;
+    while (c > 0 && (int)((long long)n * c / G) > j) --c;
+    return j - (int)((long long)n * c / G);
 }
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
@@ -175,12 +206,12 @@ __device__ __forceinline__ bool grid_barrier(const Shared& S, const Params& p, u
     if (threadIdx.x == 0) {
         // the CTA barrier above orders every consumer's writes before this release
         red_release_add(p.bar, 1u);
-        const uint32_t target = epoch * (uint32_t)p.G;
+        const uint32_t target = epoch * ((uint32_t)p.G + p.bar_extra);
         if (ld_acquire(p.bar) < target) {
             const unsigned long long t0 = gtime();
             while (ld_acquire(p.bar) < target) {
                 if (*(volatile uint32_t*)p.abort) { S.flags[0] = 1; break; }
-                if (gtime() - t0 > kWaitNs) { raise_abort(S, p, ERR_BARRIER_TIMEOUT); break; }
+                if (gtime() - t0 > p.wait_ns) { raise_abort(S, p, ERR_BARRIER_TIMEOUT); break; }
             }
         }
     }
@@ -342,6 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
     // HBM keeps streaming while the consumers sit in latency-bound phases.
     if (warp == kConsumerWarps) {
         if (lane == 0) {
+            const uint64_t pol_first = policy_evict_first();
             int k = 0;
             for (int l = 0; l < p.L && !aborted(S, p) && !TAB; ++l) {
                 for (int part = 0; part < 2; ++part) {
@@ -353,7 +385,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
                         if (!wait_bounded(S, p, &S.pempty[s], ((k / p.pred_slots) & 1) ^ 1, true)) goto pred_done;
                         const uint32_t bytes = (uint32_t)(min(R, r1 - r) * rb);
                         mbar_expect_tx(&S.pfull[s], bytes);
-                        bulk_g2s(S.pring + (size_t)s * p.pred_slot_bytes, base + (size_t)r * rb, bytes, &S.pfull[s]);
+                        if (p.hot_rows > 0)
+                            bulk_g2s_hint(S.pring + (size_t)s * p.pred_slot_bytes, base + (size_t)r * rb, bytes,
+                                          &S.pfull[s], pol_first);
+                        else
+                            bulk_g2s(S.pring + (size_t)s * p.pred_slot_bytes, base + (size_t)r * rb, bytes, &S.pfull[s]);
                         S.flags[2] = k + 1;
                     }
                 }
@@ -379,6 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
     // consumers append to this CTA's list, as soon as it appears.
     if (warp == kConsumerWarps + 1) {
         if (lane == 0) {
+            const uint64_t pol_last = policy_evict_last(), pol_first = policy_evict_first();
             int k = 0;
             bool stop = false;
             for (int l = 0; l < p.L && !stop; ++l) {
@@ -397,8 +434,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
                         const int j = S.nl[(l & 1) * p.max_rows + issued];
                         char* dst = S.fring + (size_t)s * fslot_bytes;
                         mbar_expect_tx(&S.ffull[s], (uint32_t)(4 * d + 16));
-                        bulk_g2s(dst, w1 + (size_t)j * 2 * d, (uint32_t)(2 * d), &S.ffull[s]);
-                        bulk_g2s(dst + 2 * d, w2 + (size_t)j * 2 * d, (uint32_t)(2 * d), &S.ffull[s]);
+                        if (p.hot_rows > 0) {
+                            // hot rows ([PI1] §5.2: the most frequently active neurons) stay in L2
+                            const uint64_t pol = range_offset(j, n, G) < p.hot_rows ? pol_last : pol_first;
+                            bulk_g2s_hint(dst, w1 + (size_t)j * 2 * d, (uint32_t)(2 * d), &S.ffull[s], pol);
+                            bulk_g2s_hint(dst + 2 * d, w2 + (size_t)j * 2 * d, (uint32_t)(2 * d), &S.ffull[s], pol);
+                        } else {
+                            bulk_g2s(dst, w1 + (size_t)j * 2 * d, (uint32_t)(2 * d), &S.ffull[s]);
+                            bulk_g2s(dst + 2 * d, w2 + (size_t)j * 2 * d, (uint32_t)(2 * d), &S.ffull[s]);
+                        }
                         bulk_g2s(dst + 4 * d, bb0 + (size_t)(j & ~7) * 2, 16u, &S.ffull[s]);
                         S.flags[3] = ++k;
                         ++issued;
@@ -1155,6 +1199,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
 // ---------------------------------------------------------------------------
 unsigned long long* g_trace = nullptr;
 size_t g_trace_bytes = 0;
+unsigned long long g_wait_ns = kWaitNs;     // spffn_set_wait_test
+uint32_t g_bar_extra = 0;
+int g_hot_rows = 0;                        // spffn_set_l2_hot_rows
 
 int pow2_floor(int v) {
     int r = 1;
@@ -1213,7 +1260,9 @@ cudaError_t launch_t(spffn_ctx* const* layers, int L, const void* x_in, int B, v
     if (TAB != (tabs != nullptr)) return cudaErrorInvalidValue;
     Geometry g = geometry<T, NB>(c0.cfg, G, LA, tables);
     if (g.smem > 227 * 1024) return cudaErrorInvalidConfiguration;
-    static Params p;   // host staging copy; the launch copies it into the kernel's parameter space
+    Params p;          // host staging copy (per call: concurrent callers on other stacks stay independent);
+                       // the launch copies it into the kernel's parameter space
+    memset(&p, 0, sizeof(p));
     p.L = L; p.B = B; p.d = c0.cfg.d; p.n = c0.cfg.n; p.H = c0.cfg.H; p.G = G;
     p.x_in = x_in; p.x_out = x_out; p.y = y; p.counts = counts;
     Ctl* ctl = c0.ctl();
@@ -1227,6 +1276,9 @@ cudaError_t launch_t(spffn_ctx* const* layers, int L, const void* x_in, int B, v
     p.pred_slots = g.pred_slots; p.pred_slot_bytes = g.pred_slot_bytes; p.ffn_slots = g.ffn_slots;
     p.R1 = g.R1; p.R2 = g.R2; p.max_rows = g.max_rows;
     p.trace = (g_trace && g_trace_bytes >= (size_t)G * L * kTraceMarks * 8) ? g_trace : nullptr;
+    p.wait_ns = g_wait_ns;
+    p.bar_extra = g_bar_extra;
+    p.hot_rows = g_hot_rows;
     for (int l = 0; l < L; ++l) {
         const spffn_ctx& c = *layers[l];
         p.layer[l] = LayerW{c.w.W1, c.w.b1, c.w.W2T, c.w.b2, c.w.Wp1, c.w.bp1, c.w.Wp2, c.w.bp2, c.idx(),
@@ -1289,6 +1341,19 @@ void set_trace(void* buf, size_t bytes)
 }
 
 int trace_marks() { return kTraceMarks; }
+
+void set_wait_test(unsigned long long limit_ns, bool unmeetable_barrier)
+{
+    g_wait_ns = limit_ns ? limit_ns : kWaitNs;
+    g_bar_extra = unmeetable_barrier ? 1u : 0u;
+}
+
+void set_l2_hot_rows(int rows) { g_hot_rows = rows > 0 ? rows : 0; }
+int l2_hot_rows() { return g_hot_rows; }
+
+unsigned long long wait_test_ns() { return g_wait_ns; }
+uint32_t wait_test_bar_extra() { return g_bar_extra; }
+void* trace_buffer(size_t need) { return (g_trace && g_trace_bytes >= need) ? g_trace : nullptr; }
 
 cudaError_t launch_fused_decode(spffn_ctx* const* layers, int L, const void* x_in, int B, void* x_out, float* y,
                                 int32_t* counts, bool lookahead, cudaStream_t st)

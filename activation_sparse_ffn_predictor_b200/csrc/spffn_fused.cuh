@@ -14,4 +14,13 @@ cudaError_t launch_fused_tables(spffn_ctx* const* layers, int L, const void* x_i
                                 float* y, int32_t* counts, cudaStream_t st);
 void set_trace(void* buf, size_t bytes);
 int trace_marks();
+// testing aid for the bounded-wait failure path (process-wide): limit of the grid-barrier
+// waits of later persistent launches (0 = the default 2 s) and an unmeetable grid barrier
+void set_wait_test(unsigned long long limit_ns, bool unmeetable_barrier);
+unsigned long long wait_test_ns();        // current grid-barrier wait limit of the persistent kernels
+uint32_t wait_test_bar_extra();           // extra arrivals their grid barriers expect (0 or 1)
+void* trace_buffer(size_t need);          // the bound trace buffer if at least `need` bytes, else null
+// hot-neuron L2 residency (process-wide): rows per dealt range copied with evict_last (0 = off)
+void set_l2_hot_rows(int rows);
+int l2_hot_rows();
 }  // namespace spffn

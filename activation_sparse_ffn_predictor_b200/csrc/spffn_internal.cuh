@@ -14,9 +14,11 @@ enum : uint32_t {
     ERR_IDX_RANGE = 1u << 1,       // a neuron table entry outside [0, n) (skipped)
     ERR_BARRIER_TIMEOUT = 1u << 2, // a grid barrier wait hit its iteration limit
     ERR_PIPE_TIMEOUT = 1u << 3,    // a copy-completion wait hit its iteration limit
+    ERR_CACHE_FULL = 1u << 4,      // head-sparse attention: a step found the KV cache full
 };
 
 constexpr int kMaxBatch = 256;       // union tensor-core path (B >= 16, d % 128 == 0)
+constexpr int kUStackMinBatch = 3;   // whole-stack union kernel: 3 <= B <= 128 (smaller B: the small-batch kernel)
 constexpr int kMaxPhaseBatch = 32;   // per-phase kernels and the split-FFN partial buffer
 constexpr int kCtlBytes = 1024;    // control block at the head of the workspace
 constexpr int kMaxUnionCtas = 256;  // union path: split-K partial capacity in CTAs
@@ -27,11 +29,12 @@ struct Ctl {
     uint32_t err;          // latched error bits
     uint32_t ticket;       // reserved
     uint32_t pad0[14];
-    uint32_t barrier[64];  // grid-barrier counters (persistent kernels)
+    uint32_t barrier[64];  // persistent kernels: [0] grid barrier, [1] abort of the small-batch decode;
+                           // [2], [3] the same for the whole-stack union kernel
 };
 
 struct Layout {
-    size_t ctl, h, mask, partial, xbuf, ybuf, idx, count, ctacnt, hsplit, asplit, upartial, utickets, total;
+    size_t ctl, h, mask, partial, xbuf, ybuf, idx, count, ctacnt, hsplit, asplit, upartial, utickets, uss, total;
     int S;  // number of FFN partial sums
 };
 
@@ -56,12 +59,14 @@ inline Layout make_layout(const spffn_config& c, int S) {
     const int srows = 2 * (c.max_batch <= 128 ? (c.max_batch + 15) / 16 * 16 : (c.max_batch + 127) / 128 * 128);
     L.hsplit = take((size_t)srows * c.H * 2);
     L.asplit = take((size_t)srows * c.n * 2);
-    if (c.max_batch >= 16) {
+    if (c.max_batch >= kUStackMinBatch) {
         const int nmax = c.max_batch > 32 ? 256 : 64;    // widest MMA N of a union launch
         L.upartial = take((size_t)kMaxUnionCtas * 128 * nmax * sizeof(float));
         L.utickets = take((size_t)kUnionTickets * sizeof(uint32_t));
+        // whole-stack union kernel: per 128-column tile, per token sums of squares of x + y
+        L.uss = take((size_t)((c.d + 127) / 128) * c.max_batch * sizeof(float));
     } else {
-        L.upartial = L.utickets = 0;
+        L.upartial = L.utickets = L.uss = 0;
     }
     L.total = off;
     return L;
@@ -91,6 +96,7 @@ struct spffn_ctx {
     void* asplit() const { return ws + lay.asplit; }
     float* upartial() const { return reinterpret_cast<float*>(ws + lay.upartial); }
     uint32_t* utickets() const { return reinterpret_cast<uint32_t*>(ws + lay.utickets); }
+    float* uss() const { return reinterpret_cast<float*>(ws + lay.uss); }
 };
 
 namespace spffn {

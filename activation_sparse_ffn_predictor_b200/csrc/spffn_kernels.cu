@@ -451,6 +451,18 @@ static cudaError_t profile_impl(const spffn_ctx& c, const void* X, int T_, uint3
     return cudaGetLastError();
 }
 
+cudaError_t launch_hidden(int dtype, const void* W, const void* b, const void* x, int B, int d, int H, float* h,
+                          int num_sms, cudaStream_t st)
+{
+    const int hb = min((H + 7) / 8, num_sms * 8);
+    if (dtype == SPFFN_BF16)
+        k_hidden<__nv_bfloat16><<<hb, 256, 0, st>>>((const __nv_bfloat16*)W, (const __nv_bfloat16*)b,
+                                                    (const __nv_bfloat16*)x, B, d, H, h);
+    else
+        k_hidden<__half><<<hb, 256, 0, st>>>((const __half*)W, (const __half*)b, (const __half*)x, B, d, H, h);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_compact(const spffn_ctx& c, int32_t* idx, int32_t* count, int32_t* count2, cudaStream_t st)
 {
     k_compact<<<1, 1024, 0, st>>>(c.mask(), c.cfg.n / 32, idx, count, count2);

@@ -13,6 +13,9 @@ cudaError_t launch_permute_rows(const void* src, void* dst, int rows, int row_by
                                 cudaStream_t st);
 cudaError_t launch_permute_vec(const void* src, void* dst, int count, const int32_t* perm, cudaStream_t st);
 int ffn_token_group(const spffn_ctx& c);
+// h[t][r] = ReLU(W[r] . x_t + b[r]) for an H x d weight (the predictor hidden layer; b may be null)
+cudaError_t launch_hidden(int dtype, const void* W, const void* b, const void* x, int B, int d, int H, float* h,
+                          int num_sms, cudaStream_t st);
 cudaError_t launch_forward_scratch(const spffn_config& g, const spffn_weights& w, const void* x, int B,
                                    const int32_t* idx, const int32_t* count, float* y, float* partial, int S,
                                    uint32_t* err, cudaStream_t st);

@@ -2,17 +2,19 @@
 """Sparse-FFN decode benchmark: tokens/s per layer stack and achieved HBM GB/s
 over the bytes the path touches, on seeded synthetic power-law-sparse inputs.
 
-Default workload: the OPT-6.7B-shaped stack (32 layers, d=4096, n=16384,
-predictor H=1024, fp16 weights, batch 1, mean activation rate 5%, alpha=1.2),
-weights generated in HBM, hot-first reordered offline (untimed), then K decode
-steps timed with CUDA events.  One step = spffn_decode over all layers:
-predictor (two GEMVs + threshold + compaction), sparse FC1/FC2 with the
-deterministic split reduction, and the chaining into the next layer.
+Default workload: the largest single-GPU configuration, the OPT-66B-shaped
+stack (64 layers, d=9216, n=36864, predictor H=2048, fp16 weights, ~87 GB,
+batch 32 on the union-mask tensor-core path, mean activation rate 1%,
+alpha=1.0); ``--config 1`` is the OPT-6.7B-shaped stack at batch 1.  Weights
+are generated in HBM, hot-first reordered offline (untimed), then K decode steps
+are timed with CUDA events.  One step = spffn_decode over all layers: predictor
+(two GEMVs + threshold + compaction), sparse FC1/FC2 with the deterministic
+split reduction, and the chaining into the next layer.
 With --lookahead the step is spffn_decode_lookahead instead (layer l+1's set
 predicted from layer l's input, DejaVu's asynchronous predictor), reported
 under its own workload name.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1] [--lookahead] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 4] [--lookahead] [--impl ours|reference]
     python bench.py --config 3 --rate 0.05 --true-mask     # sparse FFN on the true set, no predictor
     python bench.py --dense                                # comparison: dense FFN with cuBLAS, same weights
 
@@ -47,7 +49,39 @@ PREDICTION = {False: "each layer's set predicted from its own input",
 
 
 def workload_name(cfg, args) -> str:
-    return cfg.name + ("-lookahead" if args.lookahead else "")
+    hot = "-l2hot%d" % args.l2_hot_rows if getattr(args, "l2_hot_rows", 0) else ""
+    per = "-perlayer" if getattr(args, "per_layer_launches", False) else ""
+    return cfg.name + ("-lookahead" if args.lookahead else "") + hot + per
+
+
+def config_dict(cfg, args, world: int) -> dict:
+    """The workload as both arms print it (same keys and values in each), so a
+    line of this implementation and a line of the reference arm name one config."""
+    rate = args.rate or cfg.rate
+    return {"workload": workload_name(cfg, args), "layers": cfg.layers, "d": cfg.d, "n": cfg.n, "H": cfg.H,
+            "batch": cfg.batch, "dtype": cfg.dtype, "prediction": PREDICTION[args.lookahead],
+            "activation_rate": rate, "alpha": cfg.alpha, "global_batch": cfg.batch * world,
+            "parallelism": "replicas%d" % world,
+            "placement": "hot-first dealt over the SM count of CTA ranges (offline profile of %d tokens)"
+                         % PROFILE_TOKENS,
+            "l2": l2_statement(cfg, args),
+            "l2_hot_rows_per_range": getattr(args, "l2_hot_rows", 0)}
+
+
+L2_BYTES = 126 * 2 ** 20
+
+
+def l2_statement(cfg, args) -> str:
+    weights = cfg.layers * (predictor_bytes(cfg) + dense_bytes_per_layer(cfg))
+    if weights > 2 * L2_BYTES:
+        return "inputs larger than L2: every layer's weights (%.1f GB in all) stream from HBM each step" % (weights / 1e9)
+    if getattr(args, "flush_l2", False):
+        return "weights (%.1f MB) fit in L2; L2 flushed (%d MB written) before every timed step" % (
+            weights / 1e6, FLUSH_BYTES // 2 ** 20)
+    return "weights (%.1f MB) fit in L2 and stay resident between steps (no flush)" % (weights / 1e6)
+
+
+FLUSH_BYTES = 512 * 2 ** 20
 
 
 # ---------------------------------------------------------------------------
@@ -119,7 +153,6 @@ DECODE_TRAFFIC = {
     "sha256": "6f268d5aef86e990c15ff3378f4bd60f66b74f64e42b4ac044f1d523b2d384b7",
     "workload": "opt6.7b-d4096-n16384-L32", "batch": 1, "rate": 0.05,
     "bytes_per_layer": (223.223808e6 + 4.954112e6) / 4,
-    "summary": "profiles/k_decode_opt6.7b-d4096-n16384_b1.md",
 }
 
 
@@ -251,6 +284,9 @@ def run_ours(args, cfg, world, rank, local):
     hist = torch.zeros(K + W, L, dtype=torch.int32, device=device)
     stream = torch.cuda.Stream(device)
 
+    sp.set_l2_hot_rows(args.l2_hot_rows)
+    sp.set_union_stack(not args.per_layer_launches)
+
     def one_step():
         sp.decode(layers, x_in, x_out, y, counts, stream=stream, lookahead=args.lookahead)
 
@@ -273,11 +309,14 @@ def run_ours(args, cfg, world, rank, local):
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=device) if args.flush_l2 else None
     with Clocks(local) as clk:
         with torch.cuda.stream(stream):
             e0.record(stream)
             for s in range(K):
                 x_in.copy_(xs[W + s])
+                if flush is not None:
+                    flush.fill_(float(s))           # evicts the weights from L2 (outside the step's events)
                 ev[s][0].record(stream)
                 g.replay()
                 ev[s][1].record(stream)
@@ -288,17 +327,22 @@ def run_ours(args, cfg, world, rank, local):
     barrier(world, device)
     total_ms = e0.elapsed_time(e1)
     kernel_ms = [a.elapsed_time(b) for a, b in ev]
-    t_max = max_over_ranks(total_ms, world, device)
+    # with a flush between steps the time is the steps' own (the flushes are not decode work)
+    t_max = max_over_ranks(sum(kernel_ms) if flush is not None else total_ms, world, device)
+    del flush
     ks = hist[W:].cpu().numpy()
     bytes_per_step = [step_bytes(cfg, int(ks[s].sum()), L) for s in range(K)]
     peak, peak_kind = measured_peaks()
     mean_launch_ms = sum(kernel_ms) / K
     achieved = (sum(bytes_per_step) / K) / (mean_launch_ms * 1e-3) / 1e9
 
-    # end to end through the public API: pinned host x in, y back, each step
+    # end to end through the public API: each step copies x in from pinned host memory,
+    # calls spffn_decode through the binding (argument checks, parameter staging and
+    # every launch included) and copies y back to pinned host memory
     xh = torch.empty(K, B, cfg.d, dtype=dt).pin_memory()
     xh.copy_(xs[W:].cpu())
     yh = torch.empty(K, B, cfg.d, dtype=torch.float32).pin_memory()
+    del g
     barrier(world, device)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
@@ -306,30 +350,30 @@ def run_ours(args, cfg, world, rank, local):
         f0.record(stream)
         for s in range(K):
             x_in.copy_(xh[s], non_blocking=True)
-            g.replay()
+            one_step()
             yh[s].copy_(y, non_blocking=True)
         f1.record(stream)
     stream.synchronize()
     e2e_ms = max_over_ranks(f0.elapsed_time(f1), world, device)
-    del g
 
     value = world * B * K / (t_max * 1e-3)
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": t_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": cfg.dtype, "data": "synthetic",
-        "config": {"workload": workload_name(cfg, args), "layers": L, "d": cfg.d, "n": cfg.n, "H": cfg.H, "batch": B,
-                   "prediction": PREDICTION[args.lookahead],
-                   "activation_rate": args.rate or cfg.rate, "alpha": cfg.alpha, "global_batch": B * world,
-                   "mean_active_neurons": float(ks.mean()), "parallelism": "replicas%d" % world,
-                   "placement": "hot-first dealt over %d CTA ranges (offline profile of %d tokens)" % (layers[0].num_partials, PROFILE_TOKENS), "l2": "inputs larger than L2 (%.2f GB touched per step)"
-                   % (sum(bytes_per_step) / K / 1e9)},
+        "config": config_dict(cfg, args, world),
+        "workload_stats": {"mean_active_neurons": float(ks.mean()),
+                           "touched_gb_per_step": sum(bytes_per_step) / K / 1e9,
+                           "placement_ranges": layers[0].num_partials},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak,
                      "traffic": decode_traffic(cfg, L, B, args.rate, args.lookahead) if launches_per_step == 1 else None,
-                     "kernel": "spffn decode step (one replay per step)", "peak_kind": peak_kind},
+                     "kernel": "spffn decode step (one graph replay per step, %d launch%s)"
+                               % (launches_per_step, "" if launches_per_step == 1 else "es"),
+                     "peak_kind": peak_kind},
         "e2e": {"value": world * B * K / (e2e_ms * 1e-3), "unit": UNIT,
-                "h2d_bytes_per_step": B * cfg.d * 2, "d2h_bytes_per_step": B * cfg.d * 4},
+                "h2d_bytes_per_step": B * cfg.d * 2, "d2h_bytes_per_step": B * cfg.d * 4,
+                "path": "spffn_decode through the Python binding each step, pinned host copies in the timed region"},
         "gpu_launches": launches_per_step * K,
         "clocks": clk.summary(),
     }
@@ -546,6 +590,131 @@ def run_dense(args, cfg, world, rank, local):
 
 
 # ---------------------------------------------------------------------------
+# head-sparse attention with the attention-head predictor (DejaVu's SP_A)
+ATTN_METRIC = "head-sparse attention decode tokens/s per layer-stack"
+
+
+def attn_step_bytes(acfg, count: int, t: int) -> int:
+    """Bytes one layer's step touches: the head predictor, the selected heads'
+    Wq/Wk/Wv/Wo rows, their cached K/V rows at positions 0..t, and the stored token."""
+    pred = 2 * (acfg.Ha * acfg.d + acfg.nh * acfg.Ha) + 2 * acfg.nh
+    per_head = 4 * acfg.dh * acfg.d * 2 + 2 * (t + 1) * acfg.dh * 2
+    return pred + count * per_head + acfg.d * 2
+
+
+def run_attn(args, world, rank, local):
+    """Each step runs every layer's head-sparse attention on the step's token (the
+    layers are independent here: the FFN between them is the other benchmark).
+    Every layer's cache is first filled with ``context`` tokens by the same kernels
+    (untimed), so the timed steps see the lazily filled caches decode reaches."""
+    import torch
+    import activation_sparse_ffn_predictor_b200 as sp
+    acfg = wl.ATTN_CONFIGS[args.attn_config]
+    if args.layers:
+        acfg = acfg.with_(layers=args.layers)
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist_init(world, "nccl")
+    L, K, W = acfg.layers, args.steps, args.warmup
+    dt = torch.bfloat16 if acfg.bf16 else torch.float16
+    assert acfg.context + 1 + W + 2 * K <= acfg.tmax, "cache too small for the run"
+    layers = []
+    for l in range(L):
+        da = wl.device_attn(acfg, l, device=device)
+        layers.append((da, sp.AttnLayer(da.Wq, da.Wk, da.Wv, da.WoT, da.Wa1, da.Wa2, nh=acfg.nh, tmax=acfg.tmax,
+                                        ba2=da.ba2)))
+    steps_total = acfg.context + 1 + W + 2 * K
+    toks = torch.empty(steps_total, acfg.d, dtype=dt, device=device)
+    wl.device_fill(toks, wl.stream_id(wl.T_XA, 0, 1000 + rank), 1.0, acfg.bf16)
+    y_in = torch.empty(acfg.d, dtype=dt, device=device)
+    heads = torch.zeros(L, acfg.nh, dtype=torch.int32, device=device)
+    count = torch.zeros(L, 1, dtype=torch.int32, device=device)
+    out = torch.empty(L, acfg.d, dtype=torch.float32, device=device)
+    stream = torch.cuda.Stream(device)
+
+    def one_step():
+        for l, (_, A) in enumerate(layers):
+            A.step(y_in, heads[l], count[l], out[l], stream=stream)
+
+    pos = 0
+    with torch.cuda.stream(stream):
+        y_in.copy_(toks[pos]); pos += 1
+        one_step()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        one_step()
+    with torch.cuda.stream(stream):
+        for _ in range(acfg.context - 1 + W):           # fill the caches, then warm up
+            y_in.copy_(toks[pos]); pos += 1
+            g.replay()
+    stream.synchronize()
+    barrier(world, device)
+    torch.cuda.synchronize()
+    t0 = pos
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    hist = torch.zeros(K, L, dtype=torch.int32, device=device)
+    with Clocks(local) as clk:
+        with torch.cuda.stream(stream):
+            e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for k in range(K):
+                y_in.copy_(toks[pos]); pos += 1
+                ev[k][0].record(stream)
+                g.replay()
+                ev[k][1].record(stream)
+                hist[k].copy_(count[:, 0])
+            e1.record(stream)
+        stream.synchronize()
+    torch.cuda.synchronize()
+    barrier(world, device)
+    t_max = max_over_ranks(e0.elapsed_time(e1), world, device)
+    kernel_ms = sum(a.elapsed_time(b) for a, b in ev) / K
+    cnt = hist.cpu().numpy()
+    bytes_per_step = [sum(attn_step_bytes(acfg, int(cnt[k, l]), t0 + k) for l in range(L)) for k in range(K)]
+    achieved = (sum(bytes_per_step) / K) / (kernel_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+    dense = L * (2 * (4 * acfg.nh * acfg.dh * acfg.d) + 2 * 2 * (t0 + K) * acfg.nh * acfg.dh)
+    # end to end: token in from pinned host memory, every layer through the binding, out back
+    del g
+    yh = torch.empty(K, acfg.d, dtype=dt).pin_memory()
+    yh.copy_(toks[pos:pos + K].cpu())
+    oh = torch.empty(K, acfg.d, dtype=torch.float32).pin_memory()
+    barrier(world, device)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for k in range(K):
+            y_in.copy_(yh[k], non_blocking=True)
+            one_step()
+            oh[k].copy_(out[L - 1], non_blocking=True)
+        f1.record(stream)
+    stream.synchronize()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world, device)
+    res = {
+        "metric": ATTN_METRIC, "value": world * K / (t_max * 1e-3), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": t_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": acfg.dtype, "data": "synthetic", "impl": "head-sparse-attention",
+        "config": {"workload": acfg.name, "layers": L, "d": acfg.d, "heads": acfg.nh, "head_dim": acfg.dh,
+                   "predictor_hidden": acfg.Ha, "head_rate": acfg.rate, "context_tokens": t0,
+                   "batch": 1, "parallelism": "replicas%d" % world,
+                   "l2": "inputs larger than L2 (%.2f GB touched per step)" % (sum(bytes_per_step) / K / 1e9)},
+        "workload_stats": {"mean_selected_heads": float(cnt.mean()),
+                           "dense_attention_gb_per_step": dense / 1e9},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "kernel": "spffn_attn_step x %d layers (one graph replay per step, %d launches)"
+                     % (L, L * sp.attn_step_kernel_launches()), "peak_kind": peak_kind},
+        "e2e": {"value": world * K / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": acfg.d * 2,
+                "d2h_bytes_per_step": acfg.d * 4,
+                "path": "spffn_attn_step through the binding for every layer, pinned host copies in the timed region"},
+        "gpu_launches": L * sp.attn_step_kernel_launches() * K,
+        "clocks": clk.summary(),
+    }
+    return res, (rank == 0)
+
+
+# ---------------------------------------------------------------------------
 def cpu_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -557,32 +726,62 @@ def cpu_threads() -> int:
     return len(os.sched_getaffinity(0))
 
 
-def oracle_sample(cfg, budget_s: float, rate=None, seed=1):
-    """Time the CPU oracle on (layer, step) samples of the same workload until
-    `budget_s` of oracle compute is spent; returns tokens/s per layer stack."""
-    import oracle as O
-    prepared = []
-    for l in range(min(2, cfg.layers)):
-        p, Wp1, bp1, Wp2, bp2 = wl.host_predictor(cfg, l, rate=rate)
-        prepared.append((l, p, wl.widen(Wp1, cfg.bf16), wl.widen(bp1, cfg.bf16), wl.widen(Wp2, cfg.bf16),
-                         wl.widen(bp2, cfg.bf16), wl.widen(wl.fc1_bias(p, cfg.bf16), cfg.bf16)))
-    spent, samples, s = 0.0, 0, 0
-    while spent < budget_s and samples < 10000:
-        l, p, Wp1, bp1, Wp2, bp2, b1 = prepared[samples % len(prepared)]
-        x64 = wl.widen(wl.tokens(cfg, cfg.batch, aux=s, seed=seed), cfg.bf16)
-        idx, k, _ = O.predict(Wp1, Wp2, bp2, x64, bp1)
-        sc = 1.0 / math.sqrt(cfg.d)
-        W1 = wl.widen(wl.fill_rows(wl.stream_id(wl.T_W1, l), cfg.d, idx, sc, cfg.bf16), cfg.bf16)
-        W2T = wl.widen(wl.fill_rows(wl.stream_id(wl.T_W2T, l), cfg.d, idx, sc, cfg.bf16), cfg.bf16)
-        t0 = time.perf_counter()
-        idx, k, _ = O.predict(Wp1, Wp2, bp2, x64, bp1)
-        O.sparse_ffn(W1, b1, W2T, None, x64, idx, row_ids=idx)
-        spent += time.perf_counter() - t0
-        samples += 1
-        s += 1
-    per_layer = spent / samples
-    tok_s = cfg.batch / (per_layer * cfg.layers)
-    return tok_s, samples, spent
+class OracleSampler:
+    """Times the CPU oracle on (layer, step) samples of the workload: the first
+    two layers' predictors are generated once and kept, then each sample draws a
+    fresh batch of tokens, regenerates the FFN rows its table names (untimed) and
+    times the oracle's predict + sparse FFN.  The rate is extrapolated to the
+    whole stack (tokens/s per layer stack)."""
+
+    def __init__(self, cfg, rate=None, seed=1):
+        self.cfg, self.seed, self.s = cfg, seed, 0
+        bf = cfg.bf16
+        self.prepared = []
+        for l in range(min(2, cfg.layers)):
+            p, Wp1, bp1, Wp2, bp2 = wl.host_predictor(cfg, l, rate=rate)
+            self.prepared.append((l, wl.widen(Wp1, bf), wl.widen(bp1, bf), wl.widen(Wp2, bf), wl.widen(bp2, bf),
+                                  wl.widen(wl.fc1_bias(p, bf), bf)))
+
+    def run(self, budget_s: float, threads=None):
+        """Samples until `budget_s` of oracle compute is spent (at least one);
+        `threads` caps the BLAS thread pool (None: all it has)."""
+        import contextlib
+        import oracle as O
+        cfg = self.cfg
+        ctx = contextlib.nullcontext()
+        if threads is not None:
+            from threadpoolctl import threadpool_limits
+            ctx = threadpool_limits(limits=threads, user_api="blas")
+        spent, samples = 0.0, 0
+        with ctx:
+            while (spent < budget_s or samples == 0) and samples < 10000:
+                l, Wp1, bp1, Wp2, bp2, b1 = self.prepared[self.s % len(self.prepared)]
+                x64 = wl.widen(wl.tokens(cfg, cfg.batch, aux=self.s, seed=self.seed), cfg.bf16)
+                idx, k, _ = O.predict(Wp1, Wp2, bp2, x64, bp1)
+                sc = 1.0 / math.sqrt(cfg.d)
+                W1 = wl.widen(wl.fill_rows(wl.stream_id(wl.T_W1, l), cfg.d, idx, sc, cfg.bf16), cfg.bf16)
+                W2T = wl.widen(wl.fill_rows(wl.stream_id(wl.T_W2T, l), cfg.d, idx, sc, cfg.bf16), cfg.bf16)
+                t0 = time.perf_counter()
+                idx, k, _ = O.predict(Wp1, Wp2, bp2, x64, bp1)
+                O.sparse_ffn(W1, b1, W2T, None, x64, idx, row_ids=idx)
+                spent += time.perf_counter() - t0
+                samples += 1
+                self.s += 1
+        tok_s = cfg.batch / (spent / samples * cfg.layers)
+        return tok_s, samples, spent
+
+
+def cpu_baseline(cfg, budget_s: float, rate=None):
+    """The oracle timed on all host cores (BLAS threads) and on one thread, on
+    bounded samples of the workload; returns the JSON object."""
+    sampler = OracleSampler(cfg, rate=rate)
+    v_all, n_all, t_all = sampler.run(budget_s)
+    v_one, n_one, t_one = sampler.run(budget_s, threads=1)
+    return {"value": v_all, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": "%d (layer, step) samples of the first 2 layers, %.1f s of oracle compute, extrapolated "
+                      "to %d layers" % (n_all, t_all, cfg.layers),
+            "single_thread": {"value": v_one, "unit": UNIT, "cores": 1,
+                              "sample": "%d samples, %.1f s of oracle compute" % (n_one, t_one)}}
 
 
 def run_reference(args, cfg, world, rank, local):
@@ -591,27 +790,29 @@ def run_reference(args, cfg, world, rank, local):
         return None, False
     K, W = args.steps, args.warmup
     per_step_budget = max(0.5, min(10.0, args.ref_budget / max(1, K + W)))
+    sampler = OracleSampler(cfg, rate=args.rate)
     for _ in range(W):
-        oracle_sample(cfg, per_step_budget * 0.2, rate=args.rate)
+        sampler.run(per_step_budget * 0.2)
     vals, spent, samples = [], 0.0, 0
     for _ in range(K):
-        v, n_s, sp_ = oracle_sample(cfg, per_step_budget, rate=args.rate)
+        v, n_s, sp_ = sampler.run(per_step_budget)
         vals.append(v)
         spent += sp_
         samples += n_s
     value = statistics.mean(vals)
+    v_one, n_one, t_one = sampler.run(per_step_budget, threads=1)
     cores = cpu_threads()
     ms = cfg.batch / value * 1e3
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": workload_name(cfg, args), "layers": cfg.layers, "d": cfg.d, "n": cfg.n, "H": cfg.H,
-                   "batch": cfg.batch, "activation_rate": args.rate or cfg.rate, "alpha": cfg.alpha,
-                   "prediction": PREDICTION[args.lookahead]},
+        "config": config_dict(cfg, args, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": "%d (layer, step) samples of the first 2 layers, %.1f s of oracle compute, "
-                                   "extrapolated to %d layers" % (samples, spent, cfg.layers)},
+                                   "extrapolated to %d layers" % (samples, spent, cfg.layers),
+                         "single_thread": {"value": v_one, "unit": UNIT, "cores": 1,
+                                           "sample": "%d samples, %.1f s of oracle compute" % (n_one, t_one)}},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     return res, True
@@ -622,18 +823,28 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--config", type=int, default=4)
     ap.add_argument("--rate", type=float, default=None)
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--layers", type=int, default=None)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle compute for cpu_baseline")
+    ap.add_argument("--cpu-budget", type=float, default=10.0,
+                    help="seconds of oracle compute for each cpu_baseline leg (all cores, one thread)")
     ap.add_argument("--ref-budget", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--l2-hot-rows", type=int, default=0,
+                    help="keep this many of the hottest slots of every dealt range in L2 (B <= 2 decode)")
+    ap.add_argument("--per-layer-launches", action="store_true",
+                    help="decode 3 <= B <= 128 as per-layer launches instead of one whole-stack launch")
+    ap.add_argument("--flush-l2", action="store_true",
+                    help="write a buffer larger than L2 before every timed step (for workloads that fit in L2)")
     ap.add_argument("--lookahead", action="store_true",
                     help="predict layer l+1's neuron set from layer l's input (DejaVu look-ahead)")
     ap.add_argument("--true-mask", action="store_true",
                     help="time the sparse FFN alone on each token's true activation set (no predictor)")
+    ap.add_argument("--attn", action="store_true",
+                    help="head-sparse attention decode with the attention-head predictor (its own metric)")
+    ap.add_argument("--attn-config", type=int, default=1)
     ap.add_argument("--dense", action="store_true",
                     help="comparison arm: the dense FFN of every layer with cuBLAS on the same weights")
     args = ap.parse_args(argv)
@@ -647,6 +858,8 @@ def main(argv=None):
     world, rank, local = dist_env()
     if args.impl == "reference":
         res, show = run_reference(args, cfg, world, rank, local)
+    elif args.attn:
+        res, show = run_attn(args, world, rank, local)
     elif args.true_mask:
         res, show = run_true_mask(args, cfg, world, rank, local)
     elif args.dense:
@@ -654,10 +867,7 @@ def main(argv=None):
     else:
         res, show = run_ours(args, cfg, world, rank, local)
         if show and world == 1 and not args.no_cpu_baseline:
-            v, n_s, spent = oracle_sample(cfg, args.cpu_budget, rate=args.rate)
-            res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-                                   "sample": "%d (layer, step) samples of the first 2 layers, %.1f s of oracle "
-                                             "compute, extrapolated to %d layers" % (n_s, spent, cfg.layers)}
+            res["cpu_baseline"] = cpu_baseline(cfg, args.cpu_budget, rate=args.rate)
     if show and res is not None:
         print(json.dumps(res), flush=True)
     if world > 1:

@@ -231,23 +231,79 @@ spffn_status spffn_permute_vector(const void* src, void* dst, int32_t count, con
 spffn_status spffn_set_trace(void* buf, size_t bytes);
 int32_t spffn_trace_marks(void);
 
-/* Allocation-free variant of spffn_forward (no counterpart on the pages; it
- * exists for callers that cannot allocate device memory, e.g. code running in
- * another allocator's arena or under a fixed device-memory budget, and so
- * cannot provide an spffn_ctx workspace).  Computes exactly what spffn_forward
- * computes for the layer described by `cfg`/`w` (same kernels, same
- * deterministic split reduction; cfg->H and cfg->max_batch are not used) and
- * needs no context: the fp32 partial sums live in a fixed 1 MiB __device__
- * array that every GPU loading this library reserves until the process exits.
- *   Limit: B * cfg->d * 4 bytes <= 1 MiB (e.g. B = 32 needs d <= 8192), else
- *   SPFFN_ERR_UNSUPPORTED, checked on the host before anything is enqueued;
- *   the number of partial sums is the largest count (<= the SM count) that
- *   fits, so results agree with spffn_forward to rounding, not bitwise.
+/* Selects how spffn_decode runs 3 <= B <= 128 (B <= max_batch, d % 128 == 0,
+ * every layer of one shape, at most 64 layers, no look-ahead): enable != 0
+ * (the default) runs the whole stack as one persistent launch on the union
+ * tensor-core path, with the weights of the next phase streaming across its
+ * grid barriers; 0 runs it as per-layer launches (the predictor kernels, the
+ * compaction, FC1/FC2 and the chaining for every layer; at B >= 16 the
+ * tensor-core kernels of spffn_predict / spffn_forward).  Both compute the same
+ * function; their fp32 reductions run in different orders, so results agree to
+ * rounding.  Process-wide; applies to calls made afterwards. */
+spffn_status spffn_set_union_stack(int32_t enable);
+int32_t spffn_union_stack(void);
+
+/* Hot-neuron L2 residency ([PI1] §5.2 equation (1): a neuron's impact is its
+ * activation frequency; §5.3 places the most impactful neurons in the faster
+ * memory).  On one GPU the faster tier is the L2 cache.  After the hot-first
+ * placement dealt over the SM count of ranges (spffn_reorder_dealt with parts =
+ * spffn_num_partials), slot k of every range holds the (k G + c)-th hottest
+ * neuron, so the first `rows_per_range` slots of all ranges are the
+ * rows_per_range x G hottest neurons of the layer.  With rows_per_range > 0 the
+ * persistent decode kernel at B <= 2 (spffn_decode, spffn_decode_lookahead,
+ * spffn_decode_tables and spffn_forward there) copies those neurons' W1 and W2T
+ * rows with an L2 evict_last policy and every other weight byte (predictor and
+ * cold rows) with evict_first, per instruction: no device-wide L2 setting is
+ * changed.  The hot rows of all layers should fit in L2 together:
+ * rows_per_range x G x L x 4d bytes (about 77 MB for 32 layers at d = 4096 and
+ * one row per range).  0 (the default) issues no hints.  Results are the same
+ * bits either way.  Process-wide; applies to launches enqueued afterwards;
+ * INVALID_ARG for a negative value. */
+spffn_status spffn_set_l2_hot_rows(int32_t rows_per_range);
+int32_t spffn_l2_hot_rows(void);
+
+/* Testing aid for the failure path of the persistent whole-stack kernels (the
+ * single launch of spffn_decode, spffn_decode_lookahead and spffn_decode_tables
+ * at B <= 2, and of spffn_decode at 16 <= B <= 128 on the union path).  Every
+ * wait in those kernels is bounded; on expiry the kernel latches
+ * SPFFN_ERR_TIMEOUT in the error word, raises a grid-wide abort, stops issuing
+ * copies, waits (bounded) for the copies it already issued and returns,
+ * leaving the context usable.  This call sets, for launches enqueued after it:
+ *   limit_ns            limit of each grid-barrier wait in nanoseconds (0
+ *                       restores the default of 2 s; the other waits keep 2 s);
+ *   unmeetable_barrier  nonzero: each grid barrier expects one arrival more
+ *                       than there are CTAs, so the first one cannot complete
+ *                       and its wait runs out after limit_ns.
+ * A test sets a short limit and an unmeetable barrier, runs one decode, checks
+ * that spffn_last_device_error reports SPFFN_ERR_TIMEOUT, then calls
+ * spffn_set_wait_test(0, 0) and checks that the next decode is clean.
+ * Process-wide; not thread-safe. */
+spffn_status spffn_set_wait_test(uint64_t limit_ns, int32_t unmeetable_barrier);
+
+/* Allocation-free variant of spffn_forward (the pages have no counterpart).
+ * It is for callers that cannot allocate device memory, and so cannot provide
+ * the workspace an spffn_ctx needs: code that runs inside another allocator's
+ * arena (a cudaMalloc of its own would bypass that allocator's accounting), or
+ * code under a fixed device-memory budget that is already spent on its own
+ * buffers.  The caller passes only inputs and outputs; the
+ * fp32 partial sums live in a fixed 1 MiB __device__ array that every GPU
+ * loading this library reserves until the process exits.
+ * It computes the same function as spffn_forward for the layer described by
+ * `cfg`/`w` (cfg->H and cfg->max_batch are not used), always with the
+ * per-phase split kernels: a fixed split of the table into partial sums, then
+ * a fixed-order reduction.  spffn_forward runs other kernels at some batches
+ * (the persistent kernel at B <= 2, the tensor-core union path at B >= 16), so
+ * the two agree to fp32 rounding at every B, not bitwise.
+ *   Limit: 1 <= B <= 32 and B * cfg->d * 4 bytes <= 1 MiB (B = 32 needs
+ *   d <= 8192), else SPFFN_ERR_INVALID_ARG / SPFFN_ERR_UNSUPPORTED, checked on
+ *   the host before anything is enqueued; the number of partial sums is the
+ *   largest count (<= the SM count) that fits.
  *   Set-up: the first call on a device looks up the array's device address
  *   with that device current; make that first call before any stream capture.
- *   Every call shares the array: calls that overlap on the GPU (different
- *   streams, or different host threads without ordering) race and must not be
- *   issued; calls on one stream are ordered and safe.
+ *   Every call shares the array and the array keeps the last call's contents
+ *   (each call overwrites what it reads): calls that overlap on the GPU
+ *   (different streams, or different host threads without ordering) race and
+ *   must not be issued; calls on one stream are ordered and safe.
  *   Device-side checks still clamp the count and skip out-of-range entries,
  *   but this entry point does not report them.
  *   Calls no cudaMalloc, cudaFree or allocating library routine. */

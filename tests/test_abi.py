@@ -32,10 +32,12 @@ def test_library_exports_every_declared_symbol():
     assert set(sp.EXPORTS) <= set(syms)
 
 
-def test_library_is_sm100a_build():
-    so = sp.library()._name
-    data = open(so, "rb").read()
-    assert b"sm_100a" in data
+def test_library_is_built_for_sm100a_only():
+    """The build compiles every source for sm_100a and nothing else."""
+    from activation_sparse_ffn_predictor_b200 import build
+    flags = " ".join(build.FLAGS)
+    assert "-gencode arch=compute_100a,code=sm_100a" in flags
+    assert flags.count("-gencode") == 1 and "-arch" not in build.FLAGS
 
 
 def test_status_strings():

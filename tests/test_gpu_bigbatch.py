@@ -8,7 +8,7 @@ import pytest
 import activation_sparse_ffn_predictor_b200 as sp
 import oracle as O
 import workload as wl
-from _gpu import REL_L2_BAR, check_table, oracle_layer, rel_l2, torch_layer, x_tokens
+from _gpu import check_table, check_y, oracle_layer, torch_layer, x_tokens
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -44,7 +44,7 @@ def test_bigbatch_step_parity(name, B):
     diff = check_table(idx.cpu().numpy(), k, idx_or, logits)
     sel = idx.cpu().numpy()[:k] if diff else idx_or
     y_or = O.sparse_ffn(OL["W1"], OL["b1"], OL["W2T"], OL["b2"], x64, sel)
-    assert rel_l2(y.cpu().numpy(), y_or) <= REL_L2_BAR
+    check_y(y.cpu().numpy(), y_or)
     assert L.last_device_error() == (sp.OK, 0)
 
 
@@ -60,13 +60,13 @@ def test_bigbatch_forward_caller_tables(B):
         y = torch.empty(B, cfg.d, dtype=torch.float32, device="cuda")
         L.forward(x, idx, cnt, y)
         y_or = O.sparse_ffn(OL["W1"], OL["b1"], OL["W2T"], OL["b2"], x64, tab)
-        assert rel_l2(y.cpu().numpy(), y_or) <= REL_L2_BAR, len(tab)
+        check_y(y.cpu().numpy(), y_or)
     # the full table is the dense FFN
     y_dense = O.dense_ffn(OL["W1"], OL["b1"], OL["W2T"], OL["b2"], x64)
     idx = torch.arange(cfg.n, dtype=torch.int32, device="cuda")
     y = torch.empty(B, cfg.d, dtype=torch.float32, device="cuda")
     L.forward(x, idx, torch.tensor([cfg.n], dtype=torch.int32, device="cuda"), y)
-    assert rel_l2(y.cpu().numpy(), y_dense) <= REL_L2_BAR
+    check_y(y.cpu().numpy(), y_dense)
     assert L.last_device_error() == (sp.OK, 0)
 
 
@@ -127,5 +127,5 @@ def test_union_forward_dense_and_sparse_blocks(B):
         cnt = torch.tensor([len(t)], dtype=torch.int32, device="cuda")
         y = torch.empty(B, cfg.d, dtype=torch.float32, device="cuda")
         L.forward(x, idx, cnt, y)
-        assert rel_l2(y.cpu().numpy(), y_or) <= REL_L2_BAR
+        check_y(y.cpu().numpy(), y_or)
     assert L.last_device_error() == (sp.OK, 0)

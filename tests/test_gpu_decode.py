@@ -1,12 +1,12 @@
 """Whole-stack decode (spffn_decode, the launch the bench times) vs the oracle
-chaining its own layer inputs: per-layer counts, last layer y, final x."""
-import numpy as np
+chaining its layer inputs: every layer's neuron table and count, the last
+layer's y and the final x (the oracle continues on the GPU's table where the two
+differ only inside the near-threshold band)."""
 import pytest
 
 import activation_sparse_ffn_predictor_b200 as sp
-import oracle as O
 import workload as wl
-from _gpu import REL_L2_BAR, ambiguous, oracle_layer, rel_l2, torch_layer, x_tokens
+from _gpu import HostOracle, check_stack, prefix_runner, torch_layer, x_tokens
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -29,41 +29,28 @@ def run_case(cfg, Lc, B, aux):
     x_out = torch.empty(B, cfg.d, dtype=dt, device="cuda")
     y = torch.empty(B, cfg.d, dtype=torch.float32, device="cuda")
     counts = torch.full((Lc,), -1, dtype=torch.int32, device="cuda")
-    sp.decode(layers, wl.to_torch(xb, cfg), x_out, y, counts)
+    x_in = wl.to_torch(xb, cfg)
+    sp.decode(layers, x_in, x_out, y, counts)
     torch.cuda.synchronize()
-    return hs, layers, x64, x_out, y, counts
+    return hs, layers, x64, x_in, x_out, y, counts
 
 
 @pytest.mark.parametrize("B", [1, 2, 3])
 @pytest.mark.parametrize("name", list(CASES))
 def test_decode_matches_oracle_chain(name, B):
     cfg, Lc = CASES[name]
-    hs, layers, x64, x_out, y, counts = run_case(cfg, Lc, B, aux=300 + B)
-    xo = x64
-    exact = True
-    for l, h in enumerate(hs):
-        OL = oracle_layer(h)
-        idx, k, logits = O.predict(OL["Wp1"], OL["Wp2"], OL["bp2"], xo, OL["bp1"])
-        amb = ambiguous(logits)
-        if exact:
-            assert abs(int(counts[l].item()) - k) <= len(amb), (l, int(counts[l].item()), k)
-        exact = exact and not amb
-        y_or = O.sparse_ffn(OL["W1"], OL["b1"], OL["W2T"], OL["b2"], xo, idx)
-        if l == Lc - 1 and exact:
-            assert rel_l2(y.cpu().numpy(), y_or) <= REL_L2_BAR
-        xo = wl.widen(wl.round_to(O.chain(xo, y_or), cfg.bf16), cfg.bf16)
-    if exact:
-        got = wl.widen(x_out.cpu().view(torch.int16).numpy().view(np.uint16), cfg.bf16)
-        assert rel_l2(got, xo) <= REL_L2_BAR
+    hs, layers, x64, x_in, x_out, y, counts = run_case(cfg, Lc, B, aux=300 + B)
     for L in layers:
         assert L.last_device_error() == (sp.OK, 0)
+    check_stack(layers, [HostOracle(h) for h in hs], cfg, x64, y, x_out, counts,
+                run_prefix=prefix_runner(layers, x_in, cfg))
 
 
 def test_decode_is_deterministic_and_repeatable():
     cfg, Lc = CASES["block-d1024-n4096-L4"]
     outs = []
     for _ in range(2):
-        hs, layers, x64, x_out, y, counts = run_case(cfg, Lc, 1, aux=77)
+        hs, layers, x64, x_in, x_out, y, counts = run_case(cfg, Lc, 1, aux=77)
         outs.append((x_out.cpu(), y.cpu(), counts.cpu()))
     assert all(torch.equal(a, b) for a, b in zip(outs[0], outs[1]))
 

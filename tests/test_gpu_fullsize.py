@@ -10,7 +10,7 @@ import pytest
 import activation_sparse_ffn_predictor_b200 as sp
 import oracle as O
 import workload as wl
-from _gpu import REL_L2_BAR, ambiguous, check_table, rel_l2, x_tokens
+from _gpu import check_table, check_y, x_tokens
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -66,7 +66,7 @@ def test_fullsize_layer_step(cfg_id, B, rate):
     diff = check_table(idx.cpu().numpy(), k, idx_or, logits)
     sel = idx.cpu().numpy()[:k] if diff else idx_or
     y_or = _rows_y(cfg, layer, p, x64, sel)
-    assert rel_l2(y.cpu().numpy(), y_or) <= REL_L2_BAR
+    check_y(y.cpu().numpy(), y_or)
     assert L.last_device_error() == (sp.OK, 0)
     L.close()
     del dl, L
@@ -89,38 +89,7 @@ def test_fullsize_true_mask_forward():
     L.forward(wl.to_torch(xb, cfg), torch.from_numpy(truth).cuda(),
               torch.tensor([truth.size], dtype=torch.int32, device="cuda"), y)
     yd = O.dense_ffn(h.f64("W1"), h.f64("b1"), h.f64("W2T"), None, x64)
-    assert rel_l2(y.cpu().numpy(), yd) <= REL_L2_BAR
+    check_y(y.cpu().numpy(), yd)
     L.close()
     del dl, L, h
     torch.cuda.empty_cache()
-
-
-def test_fullsize_stack_decode_bench_shape():
-    """The bench's workload shape (d4096 n16384 H1024, batch 1) through
-    spffn_decode over 3 layers, checked layer by layer against the oracle's own
-    chained inputs."""
-    cfg = wl.CONFIGS[1]
-    Lc = 3
-    dls = [wl.device_layer(cfg, l) for l in range(Lc)]
-    layers = [sp.Layer.from_device_layer(d, max_batch=1) for d in dls]
-    xb, x64 = x_tokens(cfg, 1, aux=5)
-    x_out = torch.empty(1, cfg.d, dtype=torch.float16, device="cuda")
-    y = torch.empty(1, cfg.d, dtype=torch.float32, device="cuda")
-    counts = torch.zeros(Lc, dtype=torch.int32, device="cuda")
-    sp.decode(layers, wl.to_torch(xb, cfg), x_out, y, counts)
-    torch.cuda.synchronize()
-    xo = x64
-    for l in range(Lc):
-        p, idx_or, logits = _oracle_layer_rows(cfg, l, xo)
-        amb = ambiguous(logits)
-        k = int(counts[l].item())
-        assert abs(k - idx_or.size) <= len(amb), (l, k, idx_or.size)
-        y_or = _rows_y(cfg, l, p, xo, idx_or)
-        if l == Lc - 1 and not amb:
-            assert rel_l2(y.cpu().numpy(), y_or) <= REL_L2_BAR
-        xo = wl.widen(wl.round_to(O.chain(xo, y_or), 0), 0)
-    got = wl.widen(x_out.cpu().view(torch.int16).numpy().view(np.uint16), 0)
-    assert rel_l2(got, xo) <= REL_L2_BAR
-    for L in layers:
-        assert L.last_device_error() == (sp.OK, 0)
-        L.close()

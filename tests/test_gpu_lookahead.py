@@ -2,15 +2,15 @@
 (spffn_decode_lookahead, DejaVu appendix equation (-2) of "LLM模型之PowerInfer1.0"),
 against the oracle chaining its own layer inputs: every layer's neuron table
 (bit-exact outside the near-threshold band) and count, the last layer's y and
-the final x.  Covers the persistent kernel (B <= 2), the per-layer path (B = 3)
-and the union tensor-core path (B = 16, 64 and 200)."""
-import numpy as np
+the final x.  Where a table differs from the oracle's only inside that band the
+oracle continues on the GPU's table, so every layer is compared on every seed.
+Covers the persistent kernel (B <= 2), the per-layer path (B = 3) and the union
+tensor-core path (B = 16, 64 and 200)."""
 import pytest
 
 import activation_sparse_ffn_predictor_b200 as sp
-import oracle as O
 import workload as wl
-from _gpu import REL_L2_BAR, ambiguous, check_table, oracle_layer, rel_l2, torch_layer, x_tokens
+from _gpu import HostOracle, check_stack, prefix_runner, torch_layer, x_tokens
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -24,17 +24,6 @@ CASES = {
 }
 
 
-def oracle_chain(cfg, hs, x64, lookahead):
-    """Oracle per layer on its own chained (rounded) inputs: (idx, k, logits, y) and x_0..x_L."""
-    xs, out = [x64], []
-    for l, h in enumerate(hs):
-        xp = xs[max(l - 1, 0)] if lookahead else xs[l]
-        r = O.step_lookahead(oracle_layer(h), xp, xs[l])
-        out.append(r)
-        xs.append(wl.widen(wl.round_to(O.chain(xs[l], r[3]), cfg.bf16), cfg.bf16))
-    return out, xs
-
-
 def run_and_check(cfg, Lc, B, aux, lookahead, max_batch=None):
     hs = [wl.host_layer(cfg, l) for l in range(Lc)]
     layers = [sp.Layer(**torch_layer(h), max_batch=max_batch or B) for h in hs]
@@ -43,29 +32,15 @@ def run_and_check(cfg, Lc, B, aux, lookahead, max_batch=None):
     x_out = torch.empty(B, cfg.d, dtype=dt, device="cuda")
     y = torch.empty(B, cfg.d, dtype=torch.float32, device="cuda")
     counts = torch.full((Lc,), -1, dtype=torch.int32, device="cuda")
-    sp.decode(layers, wl.to_torch(xb, cfg), x_out, y, counts, lookahead=lookahead)
+    x_in = wl.to_torch(xb, cfg)
+    sp.decode(layers, x_in, x_out, y, counts, lookahead=lookahead)
     torch.cuda.synchronize()
     for L in layers:
         assert L.last_device_error() == (sp.OK, 0)
-    want, xs = oracle_chain(cfg, hs, x64, lookahead)
     kc = counts.cpu().numpy()
-    exact, checked = True, 0
-    for l in range(Lc):
-        idx_or, k_or, logits, y_or = want[l]
-        if not exact:
-            break
-        tab = layers[l].table(int(kc[l])).cpu().numpy()
-        diff = check_table(tab, int(kc[l]), idx_or, logits)
-        assert abs(int(kc[l]) - k_or) <= len(diff)
-        checked += 1
-        # a near-threshold neuron taken differently changes y and every later input
-        exact = not diff
-    if exact:
-        assert rel_l2(y.cpu().numpy(), want[-1][3]) <= REL_L2_BAR
-        got = wl.widen(x_out.cpu().view(torch.int16).numpy().view(np.uint16), cfg.bf16)
-        assert rel_l2(got, xs[-1]) <= REL_L2_BAR
-    assert checked >= 1
-    return kc, want
+    check_stack(layers, [HostOracle(h) for h in hs], cfg, x64, y, x_out, counts, lookahead=lookahead,
+                run_prefix=prefix_runner(layers, x_in, cfg, lookahead))
+    return kc
 
 
 @pytest.mark.parametrize("lookahead", [False, True])
@@ -85,8 +60,8 @@ def test_union_decode_tables_match_oracle(lookahead, B):
 def test_lookahead_changes_the_sets():
     # the two modes agree on layer 0 and (for this seed) differ on a later layer
     cfg, Lc = CASES["block-d1024-n4096-L4"]
-    k_std, _ = run_and_check(cfg, Lc, 1, aux=9, lookahead=False)
-    k_la, want = run_and_check(cfg, Lc, 1, aux=9, lookahead=True)
+    k_std = run_and_check(cfg, Lc, 1, aux=9, lookahead=False)
+    k_la = run_and_check(cfg, Lc, 1, aux=9, lookahead=True)
     assert k_std[0] == k_la[0]
     assert any(k_std[l] != k_la[l] for l in range(1, Lc))
 

@@ -8,7 +8,7 @@ import pytest
 import activation_sparse_ffn_predictor_b200 as sp
 import oracle as O
 import workload as wl
-from _gpu import REL_L2_BAR, check_table, oracle_layer, rel_l2, torch_layer, x_tokens
+from _gpu import REL_L2_BAR, check_table, check_y, oracle_layer, rel_l2, torch_layer, x_tokens
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -52,8 +52,7 @@ def test_predict_and_step_parity(name, B):
     # the GPU's table is a valid answer; the oracle computes y for it
     sel = np.asarray(idx.cpu().numpy()[:k]) if diff else idx_or
     y_or = O.sparse_ffn(OL["W1"], OL["b1"], OL["W2T"], OL["b2"], x64, sel)
-    err = rel_l2(y.cpu().numpy(), y_or)
-    assert err <= REL_L2_BAR, err
+    check_y(y.cpu().numpy(), y_or)
     assert L.last_device_error() == (sp.OK, 0)
 
 
@@ -76,11 +75,10 @@ def test_forward_given_table(name, B):
         y = torch.empty(B, cfg.d, dtype=torch.float32, device="cuda")
         L.forward(x, idx, cnt, y)
         y_or = O.sparse_ffn(OL["W1"], OL["b1"], OL["W2T"], OL["b2"], x64, tab)
-        err = rel_l2(y.cpu().numpy(), y_or)
-        assert err <= REL_L2_BAR, (tag, err)
+        check_y(y.cpu().numpy(), y_or)
         if tag in ("true-mask", "all"):
             yd = O.dense_ffn(OL["W1"], OL["b1"], OL["W2T"], OL["b2"], x64)
-            assert rel_l2(y.cpu().numpy(), yd) <= REL_L2_BAR
+            check_y(y.cpu().numpy(), yd)
 
 
 def test_forward_is_deterministic():
@@ -115,7 +113,7 @@ def test_edge_cases_empty_clamped_and_out_of_range():
     # count > n: clamped to n (the dense FFN), latched
     L.forward(x, idx, torch.tensor([cfg.n + 9], dtype=torch.int32, device="cuda"), y)
     yd = O.dense_ffn(OL["W1"], OL["b1"], OL["W2T"], OL["b2"], x64)
-    assert rel_l2(y.cpu().numpy(), yd) <= REL_L2_BAR
+    check_y(y.cpu().numpy(), yd)
     s, code = L.last_device_error()
     assert s == sp.ERR_DEVICE_CHECK and code & 1
     # negative count: clamped to 0
@@ -126,7 +124,7 @@ def test_edge_cases_empty_clamped_and_out_of_range():
     bad = torch.tensor([3, 40, 7, -1, 9], dtype=torch.int32, device="cuda")
     L.forward(x, bad, torch.tensor([5], dtype=torch.int32, device="cuda"), y)
     y_or = O.sparse_ffn(OL["W1"], OL["b1"], OL["W2T"], OL["b2"], x64, [3, 7, 9])
-    assert rel_l2(y.cpu().numpy(), y_or) <= REL_L2_BAR
+    check_y(y.cpu().numpy(), y_or)
     s, code = L.last_device_error()
     assert s == sp.ERR_DEVICE_CHECK and code & 2
     assert L.last_device_error() == (sp.OK, 0)      # reading clears it

@@ -9,7 +9,7 @@ import pytest
 import activation_sparse_ffn_predictor_b200 as sp
 import oracle as O
 import workload as wl
-from _gpu import REL_L2_BAR, oracle_layer, rel_l2, torch_layer, x_tokens
+from _gpu import STACK_Y_INTERNAL_BAR, STACK_Y_INTERNAL_BAR_BF16, bits_of, check_x, check_y, oracle_layer, torch_layer, x_tokens
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -56,9 +56,8 @@ def test_decode_tables_true_sets_match_oracle(name, B):
     tabs, ys, xs = oracle_true_chain(cfg, hs, x64)
     x_out, y, counts = run_tables(cfg, layers, xb, tabs, B)
     assert counts.cpu().numpy().tolist() == [len(t) for t in tabs]
-    assert rel_l2(y.cpu().numpy(), ys[-1]) <= REL_L2_BAR
-    got = wl.widen(x_out.cpu().view(torch.int16).numpy().view(np.uint16), cfg.bf16)
-    assert rel_l2(got, xs[-1]) <= REL_L2_BAR
+    check_y(y.cpu().numpy(), ys[-1], internal=STACK_Y_INTERNAL_BAR_BF16 if cfg.bf16 else STACK_Y_INTERNAL_BAR)
+    check_x(bits_of(x_out), xs[-1], cfg.bf16, stack=True)
     for L in layers:
         assert L.last_device_error() == (sp.OK, 0)
 
@@ -73,12 +72,12 @@ def test_decode_tables_order_and_bad_entries(B):
     r = np.random.default_rng(B)
     shuffled = [r.permutation(t).astype(np.int32) for t in tabs]
     x_out, y, counts = run_tables(cfg, layers, xb, shuffled, B)
-    assert rel_l2(y.cpu().numpy(), ys[-1]) <= REL_L2_BAR
+    check_y(y.cpu().numpy(), ys[-1], internal=STACK_Y_INTERNAL_BAR_BF16 if cfg.bf16 else STACK_Y_INTERNAL_BAR)
     for L in layers:
         assert L.last_device_error() == (sp.OK, 0)
     # out-of-range entries in layer 0's table: skipped (the result is unchanged) and latched
     bad = [np.concatenate([[cfg.n + 3], tabs[0], [-7]]).astype(np.int32), tabs[1]]
     x_out, y, counts = run_tables(cfg, layers, xb, bad, B)
-    assert rel_l2(y.cpu().numpy(), ys[-1]) <= REL_L2_BAR
+    check_y(y.cpu().numpy(), ys[-1], internal=STACK_Y_INTERNAL_BAR_BF16 if cfg.bf16 else STACK_Y_INTERNAL_BAR)
     s, code = layers[0].last_device_error()
     assert s == sp.ERR_DEVICE_CHECK and code & 2

@@ -392,14 +392,18 @@ def l2_hot_rows() -> int:
     return int(library().spffn_l2_hot_rows())
 
 
-def set_union_stack(enable: bool):
-    """Whole-stack persistent launch (True, the default) or per-layer launches for
-    decode at 3 <= B <= 128 (spffn_set_union_stack)."""
-    _check(library().spffn_set_union_stack(1 if enable else 0), "spffn_set_union_stack")
+UNION_PER_LAYER, UNION_STACK, UNION_AUTO = 0, 1, 2
 
 
-def union_stack() -> bool:
-    return bool(library().spffn_union_stack())
+def set_union_stack(mode: int):
+    """How decode runs 3 <= B <= 128 (spffn_set_union_stack): UNION_STACK (one
+    persistent launch), UNION_PER_LAYER, or UNION_AUTO (the default: the whole
+    stack below 16 tokens, per-layer launches from 16 up)."""
+    _check(library().spffn_set_union_stack(int(mode)), "spffn_set_union_stack")
+
+
+def union_stack() -> int:
+    return int(library().spffn_union_stack())
 
 
 def reorder(counts: np.ndarray) -> np.ndarray:

@@ -266,12 +266,13 @@ spffn_status spffn_set_trace(void* buf, size_t bytes) {
 
 int32_t spffn_trace_marks(void) { return trace_marks(); }
 
-spffn_status spffn_set_union_stack(int32_t enable) {
-    set_ustack(enable != 0);
+spffn_status spffn_set_union_stack(int32_t mode) {
+    if (mode < 0 || mode > 2) return SPFFN_ERR_INVALID_ARG;
+    set_ustack_mode(mode);
     return SPFFN_OK;
 }
 
-int32_t spffn_union_stack(void) { return ustack_enabled() ? 1 : 0; }
+int32_t spffn_union_stack(void) { return ustack_mode(); }
 
 spffn_status spffn_set_l2_hot_rows(int32_t rows_per_range) {
     if (rows_per_range < 0) return SPFFN_ERR_INVALID_ARG;

@@ -81,6 +81,25 @@ struct AParams {
 
 namespace {
 
+// w . x over a d-length row (nv 16-byte vectors): lane-strided, four independent loads in
+// flight per lane, the four partial sums added in a fixed order (then a warp sum by the caller)
+template <typename T>
+__device__ __forceinline__ float dot8(const uint4& w, const uint4& x);
+template <typename T>
+__device__ __forceinline__ float row_dot(const uint4* w, const uint4* x, int nv, int lane) {
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    int v = lane;
+    for (; v + 96 < nv; v += 128) {
+        const uint4 w0 = __ldg(w + v), w1 = __ldg(w + v + 32), w2 = __ldg(w + v + 64), w3 = __ldg(w + v + 96);
+        a0 += dot8<T>(w0, x[v]);
+        a1 += dot8<T>(w1, x[v + 32]);
+        a2 += dot8<T>(w2, x[v + 64]);
+        a3 += dot8<T>(w3, x[v + 96]);
+    }
+    for (; v < nv; v += 32) a0 += dot8<T>(__ldg(w + v), x[v]);
+    return (a0 + a1) + (a2 + a3);
+}
+
 template <typename T>
 __device__ __forceinline__ float dot8(const uint4& w, const uint4& x) {
     float a[8], b[8];
@@ -184,9 +203,7 @@ __global__ void __launch_bounds__(256) k_attn_qkv(const AParams p)
         const size_t row = (size_t)h * p.dh + i;
         const uint4* w = reinterpret_cast<const uint4*>(W + row * p.d);
         const float bias = b ? DT<T>::f(b[row]) : 0.f;
-        float acc = 0.f;
-        for (int v = lane; v < nv; v += 32) acc += dot8<T>(__ldg(w + v), ys[v]);
-        acc = warp_sum(acc) + bias;
+        float acc = warp_sum(row_dot<T>(w, ys, nv, lane)) + bias;
         if (lane == 0) {
             if (type == 0) p.q[(size_t)s * p.dh + i] = acc;
             else (type == 1 ? Kc : Vc)[((size_t)h * p.tmax + t) * p.dh + i] = DT<T>::r(acc);
@@ -201,11 +218,17 @@ __global__ void __launch_bounds__(256) k_attn_qkv(const AParams p)
             float a[8];
 #pragma unroll
             for (int g = 0; g < 8; ++g) a[g] = 0.f;
+            const uint4* yr[8];
+#pragma unroll
+            for (int g = 0; g < 8; ++g) yr[g] = reinterpret_cast<const uint4*>(Yh + (size_t)ml[g0 + min(g, ng - 1)] * p.d);
             for (int v = lane; v < nv; v += 32) {
                 const uint4 wv = __ldg(w + v);
+                uint4 yv[8];
+#pragma unroll
+                for (int g = 0; g < 8; ++g) yv[g] = g < ng ? __ldg(yr[g] + v) : make_uint4(0, 0, 0, 0);
 #pragma unroll
                 for (int g = 0; g < 8; ++g)
-                    if (g < ng) a[g] += dot8<T>(wv, __ldg(reinterpret_cast<const uint4*>(Yh + (size_t)ml[g0 + g] * p.d) + v));
+                    if (g < ng) a[g] += dot8<T>(wv, yv[g]);
             }
 #pragma unroll
             for (int g = 0; g < 8; ++g) {
@@ -247,25 +270,48 @@ __global__ void __launch_bounds__(256) k_attn_core(const AParams p)
         float m = -INFINITY, z = 0.f, o[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) o[e] = 0.f;
-        for (int pos = p0 + warp; pos < p1; pos += 8) {
-            const T* kr = Kc + ((size_t)h * p.tmax + pos) * dh;
-            const T* vr = Vc + ((size_t)h * p.tmax + pos) * dh;
-            float part = 0.f;
+        // lane's elements c = lane E .. lane E + E - 1 of each K/V row; two positions per step
+        // (independent loads), folded into the running softmax in position order
+        auto kv = [&](const T* row, float* f) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const int c = lane * E + e;
-                if (e < E && c < dh) part = fmaf(qs[c], DT<T>::f(kr[c]), part);
+                f[e] = (e < E && c < dh) ? DT<T>::f(row[c]) : 0.f;
             }
-            const float sc = warp_sum(part) * scale;
-            const float mn = fmaxf(m, sc);
-            const float cf = expf(m - mn), ef = expf(sc - mn);
-            z = z * cf + ef;
+        };
+        for (int pos = p0 + warp; pos < p1; pos += 16) {
+            const int pos2 = pos + 8;
+            const bool two = pos2 < p1;
+            float k0[8], v0[8], k1[8], v1[8];
+            kv(Kc + ((size_t)h * p.tmax + pos) * dh, k0);
+            kv(Vc + ((size_t)h * p.tmax + pos) * dh, v0);
+            kv(Kc + ((size_t)h * p.tmax + (two ? pos2 : pos)) * dh, k1);
+            kv(Vc + ((size_t)h * p.tmax + (two ? pos2 : pos)) * dh, v1);
+            float part0 = 0.f, part1 = 0.f;
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const int c = lane * E + e;
-                if (e < E && c < dh) o[e] = o[e] * cf + ef * DT<T>::f(vr[c]);
+                const float qc = (e < E && c < dh) ? qs[c] : 0.f;
+                part0 = fmaf(qc, k0[e], part0);
+                part1 = fmaf(qc, k1[e], part1);
             }
-            m = mn;
+            const float sc0 = warp_sum(part0) * scale, sc1 = warp_sum(part1) * scale;
+            {
+                const float mn = fmaxf(m, sc0);
+                const float cf = expf(m - mn), ef = expf(sc0 - mn);
+                z = z * cf + ef;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[e] = o[e] * cf + ef * v0[e];
+                m = mn;
+            }
+            if (two) {
+                const float mn = fmaxf(m, sc1);
+                const float cf = expf(m - mn), ef = expf(sc1 - mn);
+                z = z * cf + ef;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[e] = o[e] * cf + ef * v1[e];
+                m = mn;
+            }
         }
         if (lane == 0) { wm[warp] = m; wz[warp] = z; }
 #pragma unroll
@@ -460,7 +506,7 @@ cudaError_t step_impl(const spffn_attn_ctx& c, const AParams& p, cudaStream_t st
     const size_t smem = (size_t)c.cfg.d * 2;
     e = cudaFuncSetAttribute(k_attn_qkv<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_attn_qkv<T><<<G, 256, smem, st>>>(p);
+    k_attn_qkv<T><<<2 * G, 256, smem, st>>>(p);      // two CTAs per SM: more loads in flight
     k_attn_core<T><<<G, 256, 0, st>>>(p);
     k_attn_out<T><<<G, 256, 0, st>>>(p);
     k_attn_reduce<T><<<(c.cfg.d + 255) / 256, 256, 0, st>>>(p, G);

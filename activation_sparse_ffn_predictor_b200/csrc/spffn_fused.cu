@@ -60,7 +60,7 @@ struct Params {
     uint32_t* err;
     uint32_t* abort;
     int32_t* cta_count;   // [2][G + 1] list lengths per CTA, by list parity
-    float* h;             // [B][H]
+    float* h;             // [2][NB][H]: h of predictor layer q in buffer q & 1
     float* partial;       // [G][B][d]
     float* u;             // [B][d]
     int pred_slots, pred_slot_bytes, ffn_slots, R1, R2, max_rows;
@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         S.fring = q; q += (size_t)p.ffn_slots * fslot_bytes;
         S.xs = q; q += ((size_t)NB * d * sizeof(T) + 127) / 128 * 128;
         S.hs = reinterpret_cast<float*>(q); q += ((size_t)NB * H * 4 + 127) / 128 * 128;
-        S.sel = reinterpret_cast<unsigned char*>(q); q += (p.max_rows + 127) / 128 * 128;
+        S.sel = reinterpret_cast<unsigned char*>(q); q += (p.max_rows + 127) / 128 * 128;   // >= 2 x 32 flags
         S.nl = reinterpret_cast<int32_t*>(q); q += ((size_t)2 * p.max_rows * 4 + 127) / 128 * 128;
         S.bias1 = reinterpret_cast<float*>(q); q += ((size_t)(H / G + 2) * 4 + 127) / 128 * 128;
         S.bias2 = reinterpret_cast<float*>(q); q += ((size_t)p.max_rows * 4 + 127) / 128 * 128;
@@ -583,7 +583,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
     // [w nvec/8, (w+1) nvec/8) of every row; its lanes keep that segment of x in
     // registers as fp32 pairs, and the eight warps' partial dots of a row are added
     // in fixed order through shared memory.
-    auto gemv1 = [&]() -> bool {
+    auto gemv1 = [&](int q) -> bool {
+        float* hq = p.h + (size_t)(q & 1) * NB * H;
         const int seg_lo = split_lo(nvec, kConsumerWarps, warp), seg_hi = split_lo(nvec, kConsumerWarps, warp + 1);
         u64 xg[kMaxVPT][4][NB];
 #pragma unroll
@@ -690,7 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
                 float zz = 0.f;
 #pragma unroll
                 for (int q = 0; q < kConsumerWarps; ++q) zz += S.red1[(rr * kConsumerWarps + q) * NB + t];
-                if (t < B) p.h[(size_t)t * H + r + rr] = fmaxf(zz + S.bias1[r + rr - a0], 0.f);
+                if (t < B) hq[(size_t)t * H + r + rr] = fmaxf(zz + S.bias1[r + rr - a0], 0.f);
             }
             consumer_sync();
         }
@@ -710,7 +711,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         constexpr int kHV = HV;                // H <= 256 * HV
         // one L2 read of h per CTA (every CTA reads the same few lines: keep that traffic small)
         for (int i = tid; i < (NB * H) >> 2; i += kConsumers)
-            reinterpret_cast<float4*>(S.hs)[i] = __ldcg(reinterpret_cast<const float4*>(p.h) + i);
+            reinterpret_cast<float4*>(S.hs)[i] = __ldcg(reinterpret_cast<const float4*>(p.h + (size_t)(q & 1) * NB * H) + i);
         consumer_sync();
         u64 hr[kHV][4][NB];
 #pragma unroll
@@ -731,6 +732,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         TRACE(4);
         for (int r = b0; r < b1; r += R2, ++pk_) {
             const int s = pk_ % p.pred_slots;
+            // the chunk's selection flags, double-buffered by chunk: warp 0 still reads the
+            // previous chunk's flags for its append while the other warps write this one's
+            unsigned char* sel = S.sel + (pk_ & 1) * 32;
             if (!cwait(S, p, &S.pfull[s], (pk_ / p.pred_slots) & 1)) return -1;
             if (r == b0) TRACE(5);
             const uint4* slot = reinterpret_cast<const uint4*>(S.pring + (size_t)s * p.pred_slot_bytes);
@@ -775,8 +779,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
                     }
                 }
                 if (lane == 0) {
-                    S.sel[rr] = any0;
-                    if (two) S.sel[rr2] = any1;
+                    sel[rr] = any0;
+                    if (two) sel[rr2] = any1;
                 }
             }
             __syncwarp();
@@ -785,7 +789,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
             // append this chunk's selected rows in ascending order and publish the count
             if (warp == 0) {
                 for (int q0 = 0; q0 < rows; q0 += 32) {
-                    const bool on = q0 + lane < rows && S.sel[q0 + lane];
+                    const bool on = q0 + lane < rows && sel[q0 + lane];
                     const uint32_t bal = __ballot_sync(0xffffffffu, on);
                     if (on) nl[m + __popc(bal & ((1u << lane) - 1u))] = r + q0 + lane;
                     m += __popc(bal);
@@ -1125,7 +1129,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
             form_x(l);
             consumer_sync();
             TRACE(0);
-            if (!gemv1()) { ok = false; break; }
+            if (!gemv1(l)) { ok = false; break; }
             TRACE(2);
             if (!grid_barrier(S, p, epoch)) { ok = false; break; }
             TRACE(3);
@@ -1150,7 +1154,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         load_biases(0, -1);
         form_x(0);
         consumer_sync();
-        if (!gemv1() || !grid_barrier(S, p, epoch)) ok = false;
+        if (!gemv1(0) || !grid_barrier(S, p, epoch)) ok = false;
         if (ok) {
             m = gemv2(0);
             if (m < 0) ok = false;
@@ -1161,7 +1165,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
             if (l > 0) form_x(l);
             consumer_sync();
             TRACE(0);
-            if (next && !gemv1()) { ok = false; break; }
+            if (next && !gemv1(l + 1)) { ok = false; break; }
             TRACE(2);
             if (!ffn(l, m)) { ok = false; break; }
             if (!grid_barrier(S, p, epoch)) { ok = false; break; }

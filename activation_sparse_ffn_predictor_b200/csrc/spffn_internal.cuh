@@ -1,5 +1,6 @@
 // Internal definitions shared by the spffn kernels and the C-ABI glue.
 #pragma once
+#include <algorithm>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
@@ -34,7 +35,7 @@ struct Ctl {
 };
 
 struct Layout {
-    size_t ctl, h, mask, partial, xbuf, ybuf, idx, count, ctacnt, hsplit, asplit, upartial, utickets, uss, total;
+    size_t ctl, h, mask, partial, xbuf, ybuf, idx, count, ctacnt, hsplit, asplit, upartial, utickets, uss, utab, total;
     int S;  // number of FFN partial sums
 };
 
@@ -46,7 +47,9 @@ inline Layout make_layout(const spffn_config& c, int S) {
     auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
     L.S = S;
     L.ctl = take(kCtlBytes);
-    L.h = take((size_t)c.max_batch * c.H * sizeof(float));
+    // two buffers: the small-batch decode alternates them by predictor layer, so a CTA can
+    // write the next layer's h while slower CTAs still read this one (look-ahead prologue)
+    L.h = take((size_t)2 * std::max(c.max_batch, 2) * c.H * sizeof(float));
     L.mask = take((size_t)(c.n / 32) * sizeof(uint32_t));
     const int pb = c.max_batch < kMaxPhaseBatch ? c.max_batch : kMaxPhaseBatch;
     L.partial = take((size_t)S * pb * c.d * sizeof(float));
@@ -65,8 +68,10 @@ inline Layout make_layout(const spffn_config& c, int S) {
         L.utickets = take((size_t)kUnionTickets * sizeof(uint32_t));
         // whole-stack union kernel: per 128-column tile, per token sums of squares of x + y
         L.uss = take((size_t)((c.d + 127) / 128) * c.max_batch * sizeof(float));
+        // and every CTA's private copy of the neuron table (no grid barrier before the gathers)
+        L.utab = take((size_t)S * c.n * sizeof(int32_t));
     } else {
-        L.upartial = L.utickets = L.uss = 0;
+        L.upartial = L.utickets = L.uss = L.utab = 0;
     }
     L.total = off;
     return L;
@@ -97,6 +102,7 @@ struct spffn_ctx {
     float* upartial() const { return reinterpret_cast<float*>(ws + lay.upartial); }
     uint32_t* utickets() const { return reinterpret_cast<uint32_t*>(ws + lay.utickets); }
     float* uss() const { return reinterpret_cast<float*>(ws + lay.uss); }
+    int32_t* utab() const { return reinterpret_cast<int32_t*>(ws + lay.utab); }
 };
 
 namespace spffn {

@@ -12,6 +12,22 @@
 
 namespace spffn {
 
+// programmatic dependent launch (no-ops when the launch has no programmatic dependency)
+__device__ __forceinline__ void pdl_trigger_k() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_k() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+static cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, cudaStream_t st, cudaLaunchAttribute* attr) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.stream = st;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cfg;
+}
+
 // ---------------------------------------------------------------------------
 // S1  predictor hidden layer: h[t][r] = ReLU(Wp1[r] . x_t + bp1[r])
 // One warp per predictor row; tokens in groups of 8 held in registers.
@@ -32,9 +48,9 @@ __global__ void __launch_bounds__(256) k_hidden(const T* __restrict__ Wp1, const
             float acc[8];
 #pragma unroll
             for (int t = 0; t < 8; ++t) acc[t] = 0.f;
-            for (int v = lane; v < nv; v += 32) {
+            auto fold = [&](const uint4& wv, int v) {
                 float w[8];
-                unpack8<T>(ldg_stream(wrow + v), w);
+                unpack8<T>(wv, w);
 #pragma unroll
                 for (int t = 0; t < 8; ++t) {
                     if (t < nt) {
@@ -44,7 +60,16 @@ __global__ void __launch_bounds__(256) k_hidden(const T* __restrict__ Wp1, const
                         for (int k = 0; k < 8; ++k) acc[t] = fmaf(w[k], xv[k], acc[t]);
                     }
                 }
+            };
+            // four weight vectors per lane in flight before they are used (the loads are
+            // volatile asm, which the compiler does not move across each other)
+            int v = lane;
+            for (; v + 96 < nv; v += 128) {
+                const uint4 w0 = ldg_stream(wrow + v), w1 = ldg_stream(wrow + v + 32);
+                const uint4 w2 = ldg_stream(wrow + v + 64), w3 = ldg_stream(wrow + v + 96);
+                fold(w0, v); fold(w1, v + 32); fold(w2, v + 64); fold(w3, v + 96);
             }
+            for (; v < nv; v += 32) fold(ldg_stream(wrow + v), v);
 #pragma unroll
             for (int t = 0; t < 8; ++t) {
                 if (t < nt) {
@@ -116,6 +141,8 @@ __global__ void __launch_bounds__(1024) k_compact(const uint32_t* __restrict__ m
                                                   int32_t* __restrict__ count2)
 {
     __shared__ uint32_t wsum[32];
+    pdl_trigger_k();
+    pdl_wait_k();                                  // the mask words come from the previous kernel
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int per = (words + 1023) / 1024;
     const int w0 = min(words, tid * per), w1 = min(words, w0 + per);
@@ -266,6 +293,8 @@ __global__ void __launch_bounds__(1024) k_chain(const T* __restrict__ x, const f
 {
     constexpr int kV = 2;                         // 8-column vectors per thread (d <= 16384)
     __shared__ float ws[32];
+    pdl_trigger_k();
+    pdl_wait_k();                                 // y comes from the previous kernel
     const int t = blockIdx.x, tid = threadIdx.x;
     const int nv = d >> 3;
     const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * d);
@@ -438,8 +467,9 @@ cudaError_t launch_forward_scratch(const spffn_config& g, const spffn_weights& w
 template <typename T>
 static cudaError_t chain_impl(const spffn_ctx& c, const void* x, const float* y, int B, void* xn, cudaStream_t st)
 {
-    k_chain<T><<<B, 1024, 0, st>>>((const T*)x, y, c.cfg.d, (T*)xn);
-    return cudaGetLastError();
+    cudaLaunchAttribute attr[1];
+    const cudaLaunchConfig_t cfg = pdl_config(dim3(B), dim3(1024), st, attr);
+    return cudaLaunchKernelEx(&cfg, k_chain<T>, (const T*)x, y, c.cfg.d, (T*)xn);
 }
 
 template <typename T>
@@ -465,8 +495,9 @@ cudaError_t launch_hidden(int dtype, const void* W, const void* b, const void* x
 
 cudaError_t launch_compact(const spffn_ctx& c, int32_t* idx, int32_t* count, int32_t* count2, cudaStream_t st)
 {
-    k_compact<<<1, 1024, 0, st>>>(c.mask(), c.cfg.n / 32, idx, count, count2);
-    return cudaGetLastError();
+    cudaLaunchAttribute attr[1];
+    const cudaLaunchConfig_t cfg = pdl_config(dim3(1), dim3(1024), st, attr);
+    return cudaLaunchKernelEx(&cfg, k_compact, (const uint32_t*)c.mask(), c.cfg.n / 32, idx, count, count2);
 }
 
 cudaError_t launch_predict(const spffn_ctx& c, const void* x, int B, int32_t* idx, int32_t* count,

@@ -95,6 +95,10 @@ static __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
 }
 static __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 static __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+// programmatic dependent launch: let the next kernel of the stream start launching, and wait
+// until the previous one has completed and its writes are visible (no-ops without the attribute)
+static __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+static __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // host side: tensor maps through the driver entry point (no link-time libcuda dependency)

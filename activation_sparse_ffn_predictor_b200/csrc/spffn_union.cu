@@ -194,6 +194,12 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Programmatic dependent launch: the next kernel may launch now (its CTAs take an SM as
+    // this kernel's CTA there retires).  Everything read from the previous kernel's outputs
+    // waits for it: the table length and rows (modes 2, 3) from the start; in modes 0 and 1
+    // the TMA lane first issues weight tiles, which do not depend on it.
+    pdl_trigger();
+    if (p.mode >= 2 || (warp != 0 && warp != 1)) pdl_wait();
     const Plan q = make_plan(p);
     if (p.mode == 2 && blockIdx.x == 0 && threadIdx.x == 0) {
         const int U = *p.count;
@@ -209,12 +215,26 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
         // the A rows of the neuron table)
         int st = 0, ph = 0;
         uint32_t issued = 0, last_ph = 0;    // stages ever filled, parity of each one's last fill
+        // modes 0, 1: the first ring's worth of weight tiles goes out before the wait for the
+        // previous kernel; their activation tiles follow it
+        bool waited = p.mode >= 2;
+        int pend_st[kMaxStages], pend_kb[kMaxStages], npend = 0;
+        auto release = [&]() {
+            if (lane == 0) pdl_wait();
+            __syncwarp();
+            waited = true;
+            for (int i = 0; i < npend; ++i)
+                if (lane == 0) tma_2d(base + pend_st[i] * kStageBytes + 16384, &p.tmB, pend_kb[i] * kBK, p.b_row0,
+                                      &full[pend_st[i]]);
+            npend = 0;
+        };
         for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
             const int tile = u / q.splits, sp = u % q.splits;
             const int kb0 = (int)((long long)sp * q.kblocks / q.splits);
             const int kb1 = (int)((long long)(sp + 1) * q.kblocks / q.splits);
             bool okw = true;
             for (int kb = kb0; kb < kb1; ++kb) {
+                if (!waited && npend == kStages) release();     // every stage holds a pending tile
                 if (lane == 0) okw = ub_wait(&empty[st], ph ^ 1, abort_flag, p.err);
                 okw = __shfl_sync(0xffffffffu, okw, 0);
                 if (!okw) break;
@@ -225,13 +245,20 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
                 if (p.mode <= 1) {
                     if (lane == 0) tma_2d(sa, &p.tmA, kb * kBK, tile * kBM, &full[st]);
                 }
-                if (lane == 0) tma_2d(sb, &p.tmB, kb * kBK, p.b_row0, &full[st]);
+                if (!waited) {
+                    pend_st[npend] = st;
+                    pend_kb[npend] = kb;
+                    ++npend;
+                } else if (lane == 0) {
+                    tma_2d(sb, &p.tmB, kb * kBK, p.b_row0, &full[st]);
+                }
                 issued |= 1u << st;
                 last_ph = (last_ph & ~(1u << st)) | ((uint32_t)ph << st);
                 if (++st == kStages) { st = 0; ph ^= 1; }
             }
             if (!okw) break;
         }
+        if (!waited) release();
         // on abort, wait (bounded) until the last fill of every stage has landed, so no copy
         // this warp issued can arrive after the CTA retires; a short sleep stays as the margin
         // for a mode-2/3 stage whose row gathers were never issued (its barrier cannot complete,
@@ -500,17 +527,21 @@ cudaError_t launch(UParams& p, int grid, cudaStream_t st) {
     size_launch(p);
     if (p.N > kMaxN || p.stages < 2) return cudaErrorInvalidValue;
     const size_t smem = (size_t)p.stages * p.stage_bytes + 1024 + 256;
-    cudaError_t e;
-    if (p.dtype == SPFFN_BF16) {
-        e = cudaFuncSetAttribute(k_umma<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        k_umma<__nv_bfloat16><<<grid, kUThreads, smem, st>>>(p);
-    } else {
-        e = cudaFuncSetAttribute(k_umma<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        k_umma<__half><<<grid, kUThreads, smem, st>>>(p);
-    }
-    return cudaGetLastError();
+    auto kern = p.dtype == SPFFN_BF16 ? k_umma<__nv_bfloat16> : k_umma<__half>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    // programmatic dependent launch: the kernel may start while the previous one drains
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kUThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 UParams base_params(const spffn_ctx& c, int B) {

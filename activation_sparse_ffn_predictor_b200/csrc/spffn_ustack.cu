@@ -7,12 +7,13 @@
 //
 //   P0  h = ReLU(Wp1 x_l + bp1)          D[H x N1]   split-K, -> hsplit (hi/lo) | grid barrier 0
 //   P1  l = Wp2 h + bp2, l > 0 -> mask   D[n x N2]                             | grid barrier 1
-//   C   neuron table (ascending) from the mask words; every CTA writes its
-//       slice of words and knows the length U                               | grid barrier 2
-//   P2  a = ReLU(W1[table] x_l + b1)     D[U x N1]   split-K, -> asplit (hi/lo) | grid barrier 3
+//   C   neuron table (ascending) from the mask words: every CTA expands all of
+//       it into its own copy (L2-resident) and writes its slice of the table
+//       the caller reads; no barrier: a CTA's gathers read only its own copy
+//   P2  a = ReLU(W1[table] x_l + b1)     D[U x N1]   split-K, -> asplit (hi/lo) | grid barrier 2
 //   P3  y = W2T[table]^T a + b2          D[d x N2]   split-K, u = x_l + y and
-//       the per-tile sums of squares of u                                     | grid barrier 4
-//   X   x_{l+1} = round(u / sqrt(mean(u^2) + 1e-6)), every CTA its slice      | grid barrier 5
+//       the per-tile sums of squares of u                                     | grid barrier 3
+//   X   x_{l+1} = round(u / sqrt(mean(u^2) + 1e-6)), every CTA its slice      | grid barrier 4
 //
 // N1 = round16(B) columns (tokens); N2 = 2 N1: fp32 activations (h, a) enter the
 // 16-bit MMA as a hi/lo pair of the storage dtype, whose two column halves the
@@ -53,8 +54,8 @@ constexpr int kSMaxLayers = 64;       // per launch (kernel parameter space)
 constexpr int kSBM = 128;
 constexpr int kSBK = 64;
 constexpr int kSMaxStages = 8;
-constexpr int kSLag = 4;              // fewest ring stages (the gathers keep up to stages - 1 groups in flight)
-constexpr int kSBarriers = 6;         // grid barriers per layer
+constexpr int kSLag = 4;              // gather groups per thread: up to kSLag - 1 in flight (stages >= kSLag)
+constexpr int kSBarriers = 5;         // grid barriers per layer
 constexpr int kSTraceMarks = 16;
 constexpr unsigned long long kSDrainNs = 20000000ull;
 
@@ -84,6 +85,7 @@ struct alignas(64) SParams {
     uint32_t* tickets;     // [tiles]
     float* u;              // [B][d]
     float* ss;             // [d / 128][B]
+    int32_t* ptab;         // [G][n]: each CTA's own copy of the layer's neuron table
     uint32_t* bar;
     uint32_t* abort;
     uint32_t* err;
@@ -257,9 +259,9 @@ __global__ void __launch_bounds__(kSThreads, 1) k_ustack(const __grid_constant__
                     const CUtensorMap* amap = mode == 0 ? &p.tmWp1[l] : &p.tmWp2[l];
                     // (P2 waits for x_l too: a CTA with no P0 tile has not waited for it yet)
                     uint32_t dep = 0;
-                    if ((mode == 0 || mode == 2) && l > 0) dep = gb_target(p, l - 1, 5);
+                    if ((mode == 0 || mode == 2) && l > 0) dep = gb_target(p, l - 1, kSBarriers - 1);
                     if (mode == 1) dep = gb_target(p, l, 0);
-                    if (mode == 3) dep = gb_target(p, l, 3);
+                    if (mode == 3) dep = gb_target(p, l, 2);
                     bool met = dep == 0 || ld_acq(p.bar) >= dep;
                     if (met && dep) fence_async_global();
                     int npend = 0;
@@ -329,12 +331,13 @@ __global__ void __launch_bounds__(kSThreads, 1) k_ustack(const __grid_constant__
         // P3: K block kb = table rows kb*64..+63 of W2T, 256 bytes of each (this tile's 128
         //     output columns: two 64-column blocks 8 KB apart, row r at r*128, swizzled:
         //     the MN-major image).  Sixteen lanes per row.
-        // Each thread commits one cp.async group per stage and keeps up to stages - 1 groups in
-        // flight (the ring's depth: bytes in flight set the gather rate); once the oldest has
-        // landed it fences it into the async proxy, and after a group barrier one thread gives
-        // the group's arrival on that stage's full barrier.
+        // Each thread commits one cp.async group per stage and keeps up to kSLag - 1 groups in
+        // flight; once the oldest has landed it fences it into the async proxy, and after a
+        // group barrier one thread gives the group's arrival on that stage's full barrier.
         const int t = threadIdx.x - 6 * 32;
-        const int lag = NS;                  // a stage's arrival comes lag - 1 fills after its copies
+        // a stage's arrival comes lag - 1 fills after its copies; more groups in flight measured
+        // slower for these scattered row pieces (the rate falls as requests queue up)
+        const int lag = kSLag;
         int st = 0, ph = 0, nlag = 0, nb = 0;
         int lag_st[kSMaxStages];
         bool ok = true;
@@ -354,21 +357,19 @@ __global__ void __launch_bounds__(kSThreads, 1) k_ustack(const __grid_constant__
                 for (int i = 0; i < nlag; ++i) ub_arrive(&S->full[lag_st[i]]);
             nlag = 0;
         };
+        const int32_t* tab = p.ptab + (size_t)c * p.n;       // this CTA's copy of the table
         for (int l = 0; l < p.L && ok; ++l) {
-            const int32_t* tab = p.layer[l].idx;
             const char* W1 = reinterpret_cast<const char*>(p.layer[l].W1);
             const char* W2 = reinterpret_cast<const char*>(p.layer[l].W2T);
             for (int mode = 0; mode < 4 && ok; ++mode) {
                 int U = 0;
-                if (mode == 2) {
-                    // the table is complete once every CTA has written its slice
-                    bool g = true;
-                    if (t == 0) g = gb_wait(p, S, gb_target(p, l, 2));
-                    if (!group_ok(g)) { ok = false; break; }
-                }
                 if (mode >= 2) {
+                    // U is published once this CTA's copy of the table is written
                     bool g = true;
-                    if (t == 0) g = wait_U(p, S, l) >= 0;   // published before barrier 2
+                    if (t == 0) {
+                        g = wait_U(p, S, l) >= 0;
+                        __threadfence_block();
+                    }
                     if (!group_ok(g)) { ok = false; break; }
                     U = *(volatile int*)&S->U[l & 1];
                 }
@@ -542,15 +543,16 @@ __global__ void __launch_bounds__(kSThreads, 1) k_ustack(const __grid_constant__
         for (int l = 0; l < p.L && ok; ++l) {
             if (et == 0) STRACE(0);
             // x_l complete (written by every CTA's chaining of layer l - 1)
-            if (l > 0 && !group_gb(gb_target(p, l - 1, 5))) { ok = false; break; }
+            if (l > 0 && !group_gb(gb_target(p, l - 1, kSBarriers - 1))) { ok = false; break; }
             const T* xl = reinterpret_cast<const T*>(x_ptr(p, l));
             const SLayer& Ly = p.layer[l];
             const bool last_layer = l == p.L - 1;
             int U = 0;
             for (int mode = 0; mode < 4 && ok; ++mode) {
                 if (mode == 2) {
-                    // ---- C: the neuron table from the mask words (every CTA computes the prefix;
-                    //      it writes the entries of its own slice of words)
+                    // ---- C: the neuron table from the mask words: every CTA computes the prefix,
+                    //      expands the whole table into its own copy and writes its slice of
+                    //      words into the layer's table (the caller's copy)
                     if (!group_gb(gb_target(p, l, 1))) { ok = false; break; }
                     const int W = p.n >> 5;
                     const int per = (W + 127) / 128;
@@ -566,29 +568,28 @@ __global__ void __launch_bounds__(kSThreads, 1) k_ustack(const __grid_constant__
                     }
                     epi_sync();
                     U = S->U[l & 1];
-                    if (et == 0) {
-                        if (c == 0 && p.counts) p.counts[l] = U;
-                        __threadfence_block();
-                        *(volatile int*)&S->flagU = l + 1;     // TMA, MMA and gathers may plan P2, P3
-                    }
                     const int sw0 = (int)((long long)W * c / G), sw1 = (int)((long long)W * (c + 1) / G);
+                    int32_t* own = p.ptab + (size_t)c * p.n;
                     int pos = S->scan[et];
                     for (int w = w0; w < w1; ++w) {
                         uint32_t bits = __ldcg(p.mask + w);
-                        if (w >= sw0 && w < sw1) {
-                            int k = pos;
-                            while (bits) {
-                                const int b = __ffs(bits) - 1;
-                                bits &= bits - 1;
-                                Ly.idx[k++] = w * 32 + b;
-                            }
+                        const bool mine = w >= sw0 && w < sw1;
+                        while (bits) {
+                            const int b = __ffs(bits) - 1;
+                            bits &= bits - 1;
+                            own[pos] = w * 32 + b;
+                            if (mine) Ly.idx[pos] = w * 32 + b;
+                            ++pos;
                         }
-                        pos += __popc(__ldcg(p.mask + w));
                     }
-                    if (!arrive(l, 2)) { ok = false; break; }
-                    if (et == 0) STRACE(3);
-                    // every CTA's slice written before this CTA's P2 epilogue reads the table
-                    if (!group_gb(gb_target(p, l, 2))) { ok = false; break; }
+                    __threadfence_block();
+                    epi_sync();
+                    if (et == 0) {
+                        if (c == 0 && p.counts) p.counts[l] = U;
+                        __threadfence_block();
+                        *(volatile int*)&S->flagU = l + 1;     // TMA, MMA and gathers may run P2, P3
+                        STRACE(3);
+                    }
                 }
                 const SPlan q = splan(p, mode, U);
                 const bool pair = mode == 1 || mode == 3;
@@ -628,7 +629,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_ustack(const __grid_constant__
                             }
                         } else if (mode == 2) {
                             if (r < q.tiles * kSBM && r < p.n) {
-                                const int j = r < U ? __ldcg(Ly.idx + r) : -1;
+                                const int j = r < U ? __ldcg(p.ptab + (size_t)c * p.n + r) : -1;
                                 const bool live = (unsigned)j < (unsigned)p.n;
                                 const float bias = live ? ldf<T>(Ly.b1, j) : 0.f;
                                 T* as = reinterpret_cast<T*>(p.asplit);
@@ -747,13 +748,13 @@ __global__ void __launch_bounds__(kSThreads, 1) k_ustack(const __grid_constant__
                     epi_sync();
                 }
                 if (!ok) break;
-                // P0 -> barrier 0, P1 -> 1, P2 -> 3, P3 -> 4
-                if (!arrive(l, mode <= 1 ? mode : mode + 1)) { ok = false; break; }
+                // P0 -> barrier 0, P1 -> 1, P2 -> 2, P3 -> 3
+                if (!arrive(l, mode)) { ok = false; break; }
                 if (et == 0) STRACE(mode == 0 ? 1 : (mode == 1 ? 2 : (mode == 2 ? 4 : 5)));
             }
             if (!ok) break;
             // ---- X: x_{l+1} = round(u / sqrt(mean(u^2) + 1e-6)) for this CTA's slice
-            if (!group_gb(gb_target(p, l, 4))) { ok = false; break; }
+            if (!group_gb(gb_target(p, l, 3))) { ok = false; break; }
             const int T_ = p.d / kSBM;
             if (et < p.B) {
                 float s = 0.f;
@@ -775,7 +776,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_ustack(const __grid_constant__
                 for (int k = 0; k < 8; ++k) o[k] = DT<T>::r(f[k] * rs);
                 *reinterpret_cast<uint4*>(xo + e) = *reinterpret_cast<const uint4*>(o);
             }
-            if (!arrive(l, 5)) { ok = false; break; }
+            if (!arrive(l, 4)) { ok = false; break; }
             if (et == 0) STRACE(6);
         }
     }
@@ -803,20 +804,26 @@ void ustack_geometry(int B, int& N1, int& N2, int& stages, int& stage_bytes, int
     while (tmem_cols < 2 * N2) tmem_cols *= 2;
 }
 
-bool g_ustack_on = true;     // spffn_set_union_stack
+// spffn_set_union_stack: 0 per-layer launches, 1 whole stack for 3 <= B <= 128, 2 (default)
+// whole stack below 16 tokens only: from 16 up the per-layer tensor-core kernels, chained by
+// programmatic dependent launch, measured faster (OPT-13B shape at B = 16: 3.1 vs 4.0 ms per
+// step; OPT-66B shape at B = 32: 7.7 vs 9.8 ms), and below 16 slower (B = 4: 6.8 vs 3.5 ms)
+int g_ustack_mode = 2;
 
 }  // namespace
 
-void set_ustack(bool on) { g_ustack_on = on; }
-bool ustack_enabled() { return g_ustack_on; }
+void set_ustack_mode(int mode) { g_ustack_mode = mode; }
+int ustack_mode() { return g_ustack_mode; }
 
 bool ustack_supported(spffn_ctx* const* layers, int L, int B)
 {
-    if (!g_ustack_on) return false;
+    if (g_ustack_mode == 0 || (g_ustack_mode == 2 && B >= 16)) return false;
     // batches below 16 pad the MMA's N to 16 columns: idle tensor-core lanes, the same bytes
     if (L < 1 || L > kSMaxLayers || B < kUStackMinBatch || B > 128) return false;
     const spffn_ctx& c0 = *layers[0];
-    if (c0.lay.uss == 0 || c0.num_sms > kMaxUnionCtas || c0.lay.S != c0.num_sms || encoder() == nullptr) return false;
+    if (c0.lay.uss == 0 || c0.lay.utab == 0 || c0.num_sms > kMaxUnionCtas || c0.lay.S != c0.num_sms ||
+        encoder() == nullptr)
+        return false;
     for (int l = 0; l < L; ++l) {
         const spffn_ctx& c = *layers[l];
         if (B > c.cfg.max_batch || c.cfg.d % 128 != 0 || c.lay.upartial == 0 || c.lay.uss == 0) return false;
@@ -851,6 +858,7 @@ cudaError_t launch_ustack(spffn_ctx* const* layers, int L, const void* x_in, int
     p->tickets = c0.utickets();
     p->u = c0.ybuf();
     p->ss = c0.uss();
+    p->ptab = c0.utab();
     Ctl* ctl = c0.ctl();
     p->bar = &ctl->barrier[2];
     p->abort = &ctl->barrier[3];

@@ -50,7 +50,7 @@ PREDICTION = {False: "each layer's set predicted from its own input",
 
 def workload_name(cfg, args) -> str:
     hot = "-l2hot%d" % args.l2_hot_rows if getattr(args, "l2_hot_rows", 0) else ""
-    per = "-perlayer" if getattr(args, "per_layer_launches", False) else ""
+    per = {0: "-perlayer", 1: "-wholestack"}.get(getattr(args, "union_stack", 2), "")
     return cfg.name + ("-lookahead" if args.lookahead else "") + hot + per
 
 
@@ -285,7 +285,7 @@ def run_ours(args, cfg, world, rank, local):
     stream = torch.cuda.Stream(device)
 
     sp.set_l2_hot_rows(args.l2_hot_rows)
-    sp.set_union_stack(not args.per_layer_launches)
+    sp.set_union_stack(args.union_stack)
 
     def one_step():
         sp.decode(layers, x_in, x_out, y, counts, stream=stream, lookahead=args.lookahead)
@@ -834,8 +834,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--l2-hot-rows", type=int, default=0,
                     help="keep this many of the hottest slots of every dealt range in L2 (B <= 2 decode)")
-    ap.add_argument("--per-layer-launches", action="store_true",
-                    help="decode 3 <= B <= 128 as per-layer launches instead of one whole-stack launch")
+    ap.add_argument("--union-stack", type=int, choices=[0, 1, 2], default=2,
+                    help="decode 3 <= B <= 128: 0 per-layer launches, 1 one whole-stack launch, 2 (default) "
+                         "whole stack below 16 tokens")
     ap.add_argument("--flush-l2", action="store_true",
                     help="write a buffer larger than L2 before every timed step (for workloads that fit in L2)")
     ap.add_argument("--lookahead", action="store_true",

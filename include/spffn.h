@@ -232,15 +232,18 @@ spffn_status spffn_set_trace(void* buf, size_t bytes);
 int32_t spffn_trace_marks(void);
 
 /* Selects how spffn_decode runs 3 <= B <= 128 (B <= max_batch, d % 128 == 0,
- * every layer of one shape, at most 64 layers, no look-ahead): enable != 0
- * (the default) runs the whole stack as one persistent launch on the union
- * tensor-core path, with the weights of the next phase streaming across its
- * grid barriers; 0 runs it as per-layer launches (the predictor kernels, the
- * compaction, FC1/FC2 and the chaining for every layer; at B >= 16 the
- * tensor-core kernels of spffn_predict / spffn_forward).  Both compute the same
- * function; their fp32 reductions run in different orders, so results agree to
- * rounding.  Process-wide; applies to calls made afterwards. */
-spffn_status spffn_set_union_stack(int32_t enable);
+ * every layer of one shape, at most 64 layers, no look-ahead):
+ *   1  the whole stack as one persistent launch on the union tensor-core path,
+ *      with the weights of the next phase streaming across its grid barriers;
+ *   0  per-layer launches (the predictor kernels, the compaction, FC1/FC2 and
+ *      the chaining for every layer; at B >= 16 the tensor-core kernels of
+ *      spffn_predict / spffn_forward, chained by programmatic dependent launch);
+ *   2  (the default) 1 below 16 tokens, 0 from 16 up: the faster of the two on
+ *      the measured shapes.
+ * Both compute the same function; their fp32 reductions run in different
+ * orders, so results agree to rounding.  Process-wide; applies to calls made
+ * afterwards; INVALID_ARG outside 0..2.  spffn_union_stack returns the mode. */
+spffn_status spffn_set_union_stack(int32_t mode);
 int32_t spffn_union_stack(void);
 
 /* Hot-neuron L2 residency ([PI1] §5.2 equation (1): a neuron's impact is its

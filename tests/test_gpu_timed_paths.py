@@ -49,8 +49,9 @@ def test_timed_path_matches_oracle(name):
     cfg = wl.CONFIGS[cid]
     dls = [wl.device_layer(cfg, l, rate=rate) for l in range(Lc)]
     layers = [sp.Layer.from_device_layer(d, max_batch=B) for d in dls]
-    # B <= 2 and 16 <= B <= 128: the whole stack is one persistent launch, as in the benchmark
-    want_launches = 1 if B <= 128 else Lc * (4 + 2 * ((B + 127) // 128))
+    # B < 16: the whole stack is one persistent launch, as in the benchmark
+    # (the default dispatch: one launch below 16 tokens, per-layer tensor-core kernels from 16)
+    want_launches = 1 if B < 16 else Lc * (4 + 2 * ((B + 127) // 128))
     assert sp.decode_kernel_launches(layers, B) == want_launches
     xb, x64 = x_tokens(cfg, B, aux=4000 + 17 * cid + B)
     dt = torch.bfloat16 if cfg.bf16 else torch.float16
@@ -65,6 +66,36 @@ def test_timed_path_matches_oracle(name):
     oracles = [RowsOracle(cfg, l, rate=rate) for l in range(Lc)]
     check_stack(layers, oracles, cfg, x64, y, x_out, counts, lookahead=lookahead,
                 run_prefix=prefix_runner(layers, x_in, cfg, lookahead))
+    for L in layers:
+        L.close()
+    del dls, layers
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("cid,Lc,B,mode", [(4, 2, 32, 1), (2, 2, 16, 1), (2, 2, 4, 0)])
+def test_other_union_dispatch_matches_oracle(cid, Lc, B, mode):
+    """The dispatch the default does not pick at this batch: the whole-stack
+    kernel at B >= 16 (mode 1), per-layer launches below 16 (mode 0)."""
+    cfg = wl.CONFIGS[cid]
+    dls = [wl.device_layer(cfg, l) for l in range(Lc)]
+    layers = [sp.Layer.from_device_layer(d, max_batch=B) for d in dls]
+    try:
+        sp.set_union_stack(mode)
+        assert sp.decode_kernel_launches(layers, B) == (1 if mode == 1 else Lc * 6)
+        xb, x64 = x_tokens(cfg, B, aux=4100 + cid)
+        dt = torch.bfloat16 if cfg.bf16 else torch.float16
+        x_out = torch.empty(B, cfg.d, dtype=dt, device="cuda")
+        y = torch.empty(B, cfg.d, dtype=torch.float32, device="cuda")
+        counts = torch.full((Lc,), -1, dtype=torch.int32, device="cuda")
+        x_in = wl.to_torch(xb, cfg)
+        sp.decode(layers, x_in, x_out, y, counts)
+        torch.cuda.synchronize()
+        for L in layers:
+            assert L.last_device_error() == (sp.OK, 0)
+        oracles = [RowsOracle(cfg, l) for l in range(Lc)]
+        check_stack(layers, oracles, cfg, x64, y, x_out, counts, run_prefix=prefix_runner(layers, x_in, cfg))
+    finally:
+        sp.set_union_stack(sp.UNION_AUTO)
     for L in layers:
         L.close()
     del dls, layers

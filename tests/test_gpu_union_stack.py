@@ -15,6 +15,15 @@ from _gpu import HostOracle, bits_of, check_stack, prefix_runner, torch_layer, x
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
+@pytest.fixture(autouse=True)
+def whole_stack_mode():
+    """These tests run the whole-stack kernel at every batch it serves (the
+    default picks it below 16 tokens only)."""
+    sp.set_union_stack(sp.UNION_STACK)
+    yield
+    sp.set_union_stack(sp.UNION_AUTO)
+
+
 CASES = {
     "block-d1024-n4096-H256-L3": (wl.CONFIGS[0], 3),
     "ragged-bf16-d1152-n4128-H320-L3": (wl.FFNConfig("uragged", 1, 1152, 4128, 320, "bf16", 1.0, 0.1), 3),

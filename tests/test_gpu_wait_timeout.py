@@ -23,6 +23,7 @@ def test_unmeetable_grid_barrier_times_out_and_context_recovers(B, lookahead):
     Lc = 2
     hs = [wl.host_layer(cfg, l) for l in range(Lc)]
     layers = [sp.Layer(**torch_layer(h), max_batch=B) for h in hs]
+    sp.set_union_stack(sp.UNION_STACK)          # B = 16: the whole-stack union kernel
     assert sp.decode_kernel_launches(layers, B) == 1
     xb, x64 = x_tokens(cfg, B, aux=91)
     x_in = wl.to_torch(xb, cfg)
@@ -36,6 +37,7 @@ def test_unmeetable_grid_barrier_times_out_and_context_recovers(B, lookahead):
         torch.cuda.synchronize()
     finally:
         assert lib.spffn_set_wait_test(0, 0) == sp.OK
+        sp.set_union_stack(sp.UNION_STACK)
     s, code = layers[0].last_device_error()
     assert s == sp.ERR_TIMEOUT, (s, code)
     assert code & ERR_BARRIER_TIMEOUT, code
@@ -47,3 +49,4 @@ def test_unmeetable_grid_barrier_times_out_and_context_recovers(B, lookahead):
         assert L.last_device_error() == (sp.OK, 0)
     check_stack(layers, [HostOracle(h) for h in hs], cfg, x64, y, x_out, counts, lookahead=lookahead,
                 run_prefix=prefix_runner(layers, x_in, cfg, lookahead))
+    sp.set_union_stack(sp.UNION_AUTO)

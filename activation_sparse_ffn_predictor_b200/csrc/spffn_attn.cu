@@ -20,6 +20,7 @@
 //     the device, so a step replays in a CUDA graph)
 // Weight bytes dominate (Wa1, the selected heads' Wq/Wk/Wv/Wo rows, then the
 // cached K/V rows): every kernel streams rows with 16-byte loads.
+#include <algorithm>
 #include <cstring>
 #include <new>
 #include "spffn_internal.cuh"
@@ -29,7 +30,7 @@
 namespace spffn {
 
 struct ALayout {
-    size_t ctl, h, q, miss, nmiss, opart, o, ypart, tickets, K, V, filled, Y, total;
+    size_t ctl, h, q, miss, nmiss, upref, opart, o, ypart, tickets, K, V, filled, Y, total;
     int S, Sa;
 };
 
@@ -44,6 +45,7 @@ inline ALayout attn_layout(const spffn_attn_config& c, int S) {
     L.q = take((size_t)c.nh * c.dh * sizeof(float));
     L.miss = take((size_t)c.nh * c.tmax * sizeof(uint16_t));    // per head slot: missing positions
     L.nmiss = take((size_t)c.nh * sizeof(int32_t));
+    L.upref = take((size_t)(c.nh + 1) * sizeof(int32_t));     // work units before each head slot
     L.opart = take((size_t)c.nh * L.Sa * (c.dh + 2) * sizeof(float));
     L.o = take((size_t)c.nh * c.dh * sizeof(float));
     L.ypart = take((size_t)S * c.d * sizeof(float));
@@ -68,6 +70,7 @@ struct AParams {
     float* q;
     uint16_t* miss;
     int32_t* nmiss;
+    int32_t* upref;
     float* opart;
     float* o;
     float* ypart;
@@ -81,24 +84,7 @@ struct AParams {
 
 namespace {
 
-// w . x over a d-length row (nv 16-byte vectors): lane-strided, four independent loads in
-// flight per lane, the four partial sums added in a fixed order (then a warp sum by the caller)
-template <typename T>
-__device__ __forceinline__ float dot8(const uint4& w, const uint4& x);
-template <typename T>
-__device__ __forceinline__ float row_dot(const uint4* w, const uint4* x, int nv, int lane) {
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    int v = lane;
-    for (; v + 96 < nv; v += 128) {
-        const uint4 w0 = __ldg(w + v), w1 = __ldg(w + v + 32), w2 = __ldg(w + v + 64), w3 = __ldg(w + v + 96);
-        a0 += dot8<T>(w0, x[v]);
-        a1 += dot8<T>(w1, x[v + 32]);
-        a2 += dot8<T>(w2, x[v + 64]);
-        a3 += dot8<T>(w3, x[v + 96]);
-    }
-    for (; v < nv; v += 32) a0 += dot8<T>(__ldg(w + v), x[v]);
-    return (a0 + a1) + (a2 + a3);
-}
+constexpr int kPos = 4;                                 // positions per k/v work unit
 
 template <typename T>
 __device__ __forceinline__ float dot8(const uint4& w, const uint4& x) {
@@ -172,71 +158,126 @@ __global__ void __launch_bounds__(256) k_attn_select(const AParams p)
         }
         if (lane == 0) p.nmiss[s] = m;
     }
+    __syncthreads();
+    // the q/k/v kernel's work units per head slot (dh q rows, then the k and v rows once per
+    // group of kPos positions: the new token and the missing ones) and their exclusive prefix
+    if (warp == 0) {
+        int run = 0;
+        for (int s0 = 0; s0 < s_count; s0 += 32) {
+            const int s = s0 + lane;
+            const int u = s < s_count ? p.dh * (1 + 2 * ((p.nmiss[s] + kPos) / kPos)) : 0;
+            int x = u;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            if (s < s_count) p.upref[s] = run + x - u;
+            run += __shfl_sync(0xffffffffu, x, 31);
+        }
+        if (lane == 0) p.upref[s_count] = run;
+    }
 }
 
 // ---------------------------------------------------------------------------
 // 3: q, k, v rows of the selected heads for the new token; missing K/V rows from Y[p].
-// Work items: (head slot, block of 8 rows of the 3 dh rows q | k | v), one row per
-// warp; each CTA takes a contiguous range of items so consecutive items share a head.
+// Work units, balanced over every warp of the grid (unit u goes to warp u mod W): per
+// head slot, its dh q rows (the new token), then for each k and each v row one unit per
+// group of kPos positions (the new token first, then the missing positions in order).
+// Consecutive units of one row go to neighbouring warps of one CTA, so the weight row
+// they share is read from HBM once.  The y rows come from the stored inputs Y (the new
+// token was stored by the select kernel).
+
+// NP dot products w . y_j over a d-length row, U rows of 16-byte loads in flight per lane;
+// each position accumulates lane-strided in ascending vector order, then a warp sum.
+template <typename T, int NP, int U>
+__device__ __forceinline__ void rows_dot(const uint4* w, const uint4* const* y, int nv, int lane, float* z) {
+    float a[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) a[j] = 0.f;
+    int v = lane;
+    for (; v + 32 * (U - 1) < nv; v += 32 * U) {
+        uint4 wv[U], yv[U][NP];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            wv[u] = __ldg(w + v + 32 * u);
+#pragma unroll
+            for (int j = 0; j < NP; ++j) yv[u][j] = __ldg(y[j] + v + 32 * u);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int j = 0; j < NP; ++j) a[j] += dot8<T>(wv[u], yv[u][j]);
+    }
+    for (; v < nv; v += 32) {
+        const uint4 wv = __ldg(w + v);
+#pragma unroll
+        for (int j = 0; j < NP; ++j) a[j] += dot8<T>(wv, __ldg(y[j] + v));
+    }
+#pragma unroll
+    for (int j = 0; j < NP; ++j) z[j] = warp_sum(a[j]);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) k_attn_qkv(const AParams p)
 {
-    extern __shared__ uint4 ys[];                      // the new token, d / 8 vectors
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ int up[1025];
+    const int lane = threadIdx.x & 31;
     const int t = *p.tcur, count = *p.count;
     if (t >= p.tmax || count == 0) return;
-    const int nv = p.d / 8;
-    for (int v = tid; v < nv; v += 256) ys[v] = reinterpret_cast<const uint4*>(p.y)[v];
+    for (int s = threadIdx.x; s <= count; s += 256) up[s] = p.upref[s];
     __syncthreads();
-    const int iph = (3 * p.dh + 7) / 8;
-    const int items = count * iph;
-    const int i0 = (int)((long long)items * blockIdx.x / gridDim.x), i1 = (int)((long long)items * (blockIdx.x + 1) / gridDim.x);
-    T* Kc = reinterpret_cast<T*>(p.K);
-    T* Vc = reinterpret_cast<T*>(p.V);
+    const int nv = p.d / 8, dh = p.dh, total = up[count], W = gridDim.x * 8;
     const T* Yh = reinterpret_cast<const T*>(p.Y);
-    for (int it = i0; it < i1; ++it) {
-        const int s = it / iph, r = (it % iph) * 8 + warp;
-        if (r >= 3 * p.dh) continue;
-        const int h = p.heads[s], type = r / p.dh, i = r % p.dh;
-        const T* W = reinterpret_cast<const T*>(type == 0 ? p.Wq : (type == 1 ? p.Wk : p.Wv));
-        const T* b = reinterpret_cast<const T*>(type == 0 ? p.bq : (type == 1 ? p.bk : p.bv));
-        const size_t row = (size_t)h * p.dh + i;
-        const uint4* w = reinterpret_cast<const uint4*>(W + row * p.d);
-        const float bias = b ? DT<T>::f(b[row]) : 0.f;
-        float acc = warp_sum(row_dot<T>(w, ys, nv, lane)) + bias;
-        if (lane == 0) {
-            if (type == 0) p.q[(size_t)s * p.dh + i] = acc;
-            else (type == 1 ? Kc : Vc)[((size_t)h * p.tmax + t) * p.dh + i] = DT<T>::r(acc);
+    const uint4* yt = reinterpret_cast<const uint4*>(Yh + (size_t)t * p.d);
+    for (int u = blockIdx.x * 8 + (threadIdx.x >> 5); u < total; u += W) {
+        int lo = 0, hi = count - 1;                     // the slot: last s with up[s] <= u
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (up[mid] <= u) lo = mid; else hi = mid - 1;
         }
-        if (type == 0) continue;
-        // the head's missing rows at earlier positions, eight at a time (the weight row
-        // comes back from L1/L2 after its first pass)
-        const int nm = p.nmiss[s];
+        const int s = lo, h = p.heads[s];
+        int w = u - up[s];
+        if (w < dh) {
+            const size_t row = (size_t)h * dh + w;
+            const uint4* wr = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.Wq) + row * p.d);
+            const float bias = p.bq ? DT<T>::f(reinterpret_cast<const T*>(p.bq)[row]) : 0.f;
+            float z;
+            rows_dot<T, 1, 4>(wr, &yt, nv, lane, &z);
+            if (lane == 0) p.q[(size_t)s * dh + w] = z + bias;
+            continue;
+        }
+        w -= dh;
+        const int nm = p.nmiss[s], ng = (nm + kPos) / kPos;
+        const int type = w / (dh * ng);                 // 0: k row, 1: v row
+        const int rem = w - type * dh * ng, i = rem / ng, g = rem - i * ng;
+        const size_t row = (size_t)h * dh + i;
+        const T* Wr = reinterpret_cast<const T*>(type == 0 ? p.Wk : p.Wv);
+        const T* br = reinterpret_cast<const T*>(type == 0 ? p.bk : p.bv);
+        const float bias = br ? DT<T>::f(br[row]) : 0.f;
+        const uint4* wr = reinterpret_cast<const uint4*>(Wr + row * p.d);
         const uint16_t* ml = p.miss + (size_t)s * p.tmax;
-        for (int g0 = 0; g0 < nm; g0 += 8) {
-            const int ng = min(8, nm - g0);
-            float a[8];
+        const int j0 = g * kPos, np = min(kPos, nm + 1 - j0);
+        int pos[kPos];
+        const uint4* yr[kPos];
 #pragma unroll
-            for (int g = 0; g < 8; ++g) a[g] = 0.f;
-            const uint4* yr[8];
+        for (int j = 0; j < kPos; ++j) {
+            const int jj = j0 + min(j, np - 1);
+            pos[j] = jj == 0 ? t : (int)ml[jj - 1];
+            yr[j] = reinterpret_cast<const uint4*>(Yh + (size_t)pos[j] * p.d);
+        }
+        float z[kPos];
+        switch (np) {
+            case 1: rows_dot<T, 1, 4>(wr, yr, nv, lane, z); break;
+            case 2: rows_dot<T, 2, 2>(wr, yr, nv, lane, z); break;
+            case 3: rows_dot<T, 3, 2>(wr, yr, nv, lane, z); break;
+            default: rows_dot<T, 4, 2>(wr, yr, nv, lane, z); break;
+        }
+        if (lane == 0) {
+            T* C = reinterpret_cast<T*>(type == 0 ? p.K : p.V);
 #pragma unroll
-            for (int g = 0; g < 8; ++g) yr[g] = reinterpret_cast<const uint4*>(Yh + (size_t)ml[g0 + min(g, ng - 1)] * p.d);
-            for (int v = lane; v < nv; v += 32) {
-                const uint4 wv = __ldg(w + v);
-                uint4 yv[8];
-#pragma unroll
-                for (int g = 0; g < 8; ++g) yv[g] = g < ng ? __ldg(yr[g] + v) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-                for (int g = 0; g < 8; ++g)
-                    if (g < ng) a[g] += dot8<T>(wv, yv[g]);
-            }
-#pragma unroll
-            for (int g = 0; g < 8; ++g) {
-                if (g < ng) {
-                    const float z = warp_sum(a[g]) + bias;
-                    if (lane == 0) (type == 1 ? Kc : Vc)[((size_t)h * p.tmax + ml[g0 + g]) * p.dh + i] = DT<T>::r(z);
-                }
-            }
+            for (int j = 0; j < kPos; ++j)
+                if (j < np) C[((size_t)h * p.tmax + pos[j]) * dh + i] = DT<T>::r(z[j] + bias);
         }
     }
 }
@@ -461,6 +502,7 @@ struct spffn_attn_ctx {
     spffn_attn_weights w;
     char* ws;
     spffn::ALayout lay;
+    int qkv_blocks;                                     // resident CTAs of the q/k/v kernel
 };
 
 using namespace spffn;
@@ -484,6 +526,7 @@ AParams attn_params(const spffn_attn_ctx& c, const void* y, int32_t* heads, int3
     p.q = reinterpret_cast<float*>(c.ws + c.lay.q);
     p.miss = reinterpret_cast<uint16_t*>(c.ws + c.lay.miss);
     p.nmiss = reinterpret_cast<int32_t*>(c.ws + c.lay.nmiss);
+    p.upref = reinterpret_cast<int32_t*>(c.ws + c.lay.upref);
     p.opart = reinterpret_cast<float*>(c.ws + c.lay.opart);
     p.o = reinterpret_cast<float*>(c.ws + c.lay.o);
     p.ypart = reinterpret_cast<float*>(c.ws + c.lay.ypart);
@@ -503,10 +546,7 @@ cudaError_t step_impl(const spffn_attn_ctx& c, const AParams& p, cudaStream_t st
                                   reinterpret_cast<float*>(c.ws + c.lay.h), G, st);
     if (e != cudaSuccess) return e;
     k_attn_select<T><<<1, 256, 0, st>>>(p);
-    const size_t smem = (size_t)c.cfg.d * 2;
-    e = cudaFuncSetAttribute(k_attn_qkv<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    k_attn_qkv<T><<<2 * G, 256, smem, st>>>(p);      // two CTAs per SM: more loads in flight
+    k_attn_qkv<T><<<c.qkv_blocks, 256, 0, st>>>(p);   // every resident warp takes units
     k_attn_core<T><<<G, 256, 0, st>>>(p);
     k_attn_out<T><<<G, 256, 0, st>>>(p);
     k_attn_reduce<T><<<(c.cfg.d + 255) / 256, 256, 0, st>>>(p, G);
@@ -541,6 +581,15 @@ spffn_status spffn_attn_create(const spffn_attn_config* cfg, const spffn_attn_we
     c->w = *w;
     c->ws = static_cast<char*>(workspace);
     c->lay = lay;
+    int occ = 0;
+    const cudaError_t e = cfg->dtype == SPFFN_BF16
+                              ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_attn_qkv<__nv_bfloat16>, 256, 0)
+                              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_attn_qkv<__half>, 256, 0);
+    if (e != cudaSuccess || occ < 1) {
+        cudaGetLastError();
+        occ = 2;
+    }
+    c->qkv_blocks = lay.S * std::min(occ, 8);
     *out = c;
     return SPFFN_OK;
 }

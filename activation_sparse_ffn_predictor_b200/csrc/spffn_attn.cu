@@ -4,20 +4,19 @@
 // the page's handling of KV-cache misses (a head selected after being skipped
 // computes its missing K/V rows from the stored inputs of the past tokens).
 //
-// One step of one layer, one token, six launches on the caller's stream:
+// One step of one layer, one token, five launches on the caller's stream:
 //   1 SP_A hidden layer h = ReLU(Wa1 y + ba1)                 (the predictor GEMV kernel)
 //   2 head logits, threshold, ascending head list; y stored as Y[t]; for every
-//     selected head the list of positions p < t whose K/V rows are missing
+//     selected head the list of positions p < t whose K/V rows are missing, and
+//     the q/k/v kernel's work units per head
 //   3 q, k, v rows of the selected heads for the new token, and the missing K/V
-//     rows from Y[p] (each weight row streamed once, reused from L1/L2 for the
-//     missing positions)
+//     rows from Y[p], in work units balanced over every resident warp
 //   4 attention per selected head over positions 0..t, split over CTAs with an
 //     online softmax in fixed position order, the splits combined in fixed
 //     order by the last CTA of the head (atomic ticket)
-//   5 output projection: each CTA accumulates o_k[i] WoT[k dh + i] over an equal
-//     share of the selected heads' rows into its own fp32 partial
-//   6 out = bo + the partials in fixed order; t = t + 1 (the position lives on
-//     the device, so a step replays in a CUDA graph)
+//   5 out = bo + sum of o_k[i] WoT[k dh + i] over the selected heads' rows, each
+//     CTA owning a slice of out's columns (sums in a fixed order); t = t + 1 (the
+//     position lives on the device, so a step replays in a CUDA graph)
 // Weight bytes dominate (Wa1, the selected heads' Wq/Wk/Wv/Wo rows, then the
 // cached K/V rows): every kernel streams rows with 16-byte loads.
 #include <algorithm>
@@ -30,7 +29,7 @@
 namespace spffn {
 
 struct ALayout {
-    size_t ctl, h, q, miss, nmiss, upref, opart, o, ypart, tickets, K, V, filled, Y, total;
+    size_t ctl, h, q, miss, nmiss, upref, opart, o, tickets, K, V, filled, Y, total;
     int S, Sa;
 };
 
@@ -48,7 +47,6 @@ inline ALayout attn_layout(const spffn_attn_config& c, int S) {
     L.upref = take((size_t)(c.nh + 1) * sizeof(int32_t));     // work units before each head slot
     L.opart = take((size_t)c.nh * L.Sa * (c.dh + 2) * sizeof(float));
     L.o = take((size_t)c.nh * c.dh * sizeof(float));
-    L.ypart = take((size_t)S * c.d * sizeof(float));
     L.tickets = take((size_t)c.nh * sizeof(uint32_t));
     L.K = take((size_t)c.nh * c.tmax * c.dh * 2);
     L.V = take((size_t)c.nh * c.tmax * c.dh * 2);
@@ -73,7 +71,6 @@ struct AParams {
     int32_t* upref;
     float* opart;
     float* o;
-    float* ypart;
     uint32_t* tickets;
     void* K;
     void* V;
@@ -99,9 +96,12 @@ __device__ __forceinline__ float dot8(const uint4& w, const uint4& x) {
 
 // ---------------------------------------------------------------------------
 // 2: head logits l_k = Wa2[k] . h + ba2_k, selection l_k > 0, ascending list; Y[t] = y;
-// per selected head the positions p < t with no K/V row yet.  One CTA.
+// per selected head the positions p < t with no K/V row yet.  One CTA of 32 warps (a
+// few heads per warp, each row's loads issued together: this kernel is latency-bound).
+constexpr int kSelWarps = 32;
+
 template <typename T>
-__global__ void __launch_bounds__(256) k_attn_select(const AParams p)
+__global__ void __launch_bounds__(kSelWarps * 32) k_attn_select(const AParams p)
 {
     __shared__ unsigned char sel[1024];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -110,19 +110,26 @@ __global__ void __launch_bounds__(256) k_attn_select(const AParams p)
     if (!full) {
         const uint4* src = reinterpret_cast<const uint4*>(p.y);
         uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.Y) + (size_t)t * p.d);
-        for (int v = tid; v < p.d / 8; v += 256) dst[v] = src[v];
+        for (int v = tid; v < p.d / 8; v += kSelWarps * 32) dst[v] = src[v];
     }
     const int hv = p.Ha / 8;
-    for (int k = warp; k < p.nh; k += 8) {
+    for (int k = warp; k < p.nh; k += kSelWarps) {
         const uint4* w = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.Wa2) + (size_t)k * p.Ha);
         float acc = 0.f;
-        for (int v = lane; v < hv; v += 32) {
+        auto fold = [&](const uint4& wv, int v) {
             float wf[8];
-            unpack8<T>(ldg_stream(w + v), wf);
+            unpack8<T>(wv, wf);
             const float4 a = reinterpret_cast<const float4*>(p.h)[2 * v], b = reinterpret_cast<const float4*>(p.h)[2 * v + 1];
             acc = fmaf(wf[0], a.x, acc); acc = fmaf(wf[1], a.y, acc); acc = fmaf(wf[2], a.z, acc); acc = fmaf(wf[3], a.w, acc);
             acc = fmaf(wf[4], b.x, acc); acc = fmaf(wf[5], b.y, acc); acc = fmaf(wf[6], b.z, acc); acc = fmaf(wf[7], b.w, acc);
+        };
+        int v = lane;
+        for (; v + 96 < hv; v += 128) {
+            const uint4 w0 = ldg_stream(w + v), w1 = ldg_stream(w + v + 32);
+            const uint4 w2 = ldg_stream(w + v + 64), w3 = ldg_stream(w + v + 96);
+            fold(w0, v); fold(w1, v + 32); fold(w2, v + 64); fold(w3, v + 96);
         }
+        for (; v < hv; v += 32) fold(ldg_stream(w + v), v);
         acc = warp_sum(acc);
         const float bias = p.ba2 ? DT<T>::f(reinterpret_cast<const T*>(p.ba2)[k]) : 0.f;
         if (lane == 0) sel[k] = !full && (acc + bias) > 0.f;
@@ -145,7 +152,7 @@ __global__ void __launch_bounds__(256) k_attn_select(const AParams p)
     }
     __syncthreads();
     // missing K/V rows of each selected head (one warp per head, ascending positions)
-    for (int s = warp; s < s_count; s += 8) {
+    for (int s = warp; s < s_count; s += kSelWarps) {
         const int h = p.heads[s];
         const uint8_t* f = p.filled + (size_t)h * p.tmax;
         uint16_t* ml = p.miss + (size_t)s * p.tmax;
@@ -181,12 +188,12 @@ __global__ void __launch_bounds__(256) k_attn_select(const AParams p)
 
 // ---------------------------------------------------------------------------
 // 3: q, k, v rows of the selected heads for the new token; missing K/V rows from Y[p].
-// Work units, balanced over every warp of the grid (unit u goes to warp u mod W): per
-// head slot, its dh q rows (the new token), then for each k and each v row one unit per
-// group of kPos positions (the new token first, then the missing positions in order).
-// Consecutive units of one row go to neighbouring warps of one CTA, so the weight row
-// they share is read from HBM once.  The y rows come from the stored inputs Y (the new
-// token was stored by the select kernel).
+// Work units, balanced over every warp of the grid (warp w takes the w-th of W equal
+// contiguous ranges): per head slot, its dh q rows (the new token), then for each k and
+// each v row one unit per group of kPos positions (the new token first, then the missing
+// positions in order).  Contiguous ranges keep a CTA's warps on one head, so the few
+// stored input rows Y[p] they all read stay in L1, and the units of one weight row run
+// back to back on one warp.  The new token was stored in Y by the select kernel.
 
 // NP dot products w . y_j over a d-length row, U rows of 16-byte loads in flight per lane;
 // each position accumulates lane-strided in ascending vector order, then a warp sum.
@@ -230,7 +237,9 @@ __global__ void __launch_bounds__(256) k_attn_qkv(const AParams p)
     const int nv = p.d / 8, dh = p.dh, total = up[count], W = gridDim.x * 8;
     const T* Yh = reinterpret_cast<const T*>(p.Y);
     const uint4* yt = reinterpret_cast<const uint4*>(Yh + (size_t)t * p.d);
-    for (int u = blockIdx.x * 8 + (threadIdx.x >> 5); u < total; u += W) {
+    const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int u0 = (int)((long long)total * gw / W), u1 = (int)((long long)total * (gw + 1) / W);
+    for (int u = u0; u < u1; ++u) {
         int lo = 0, hi = count - 1;                     // the slot: last s with up[s] <= u
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
@@ -288,7 +297,7 @@ __global__ void __launch_bounds__(256) k_attn_qkv(const AParams p)
 // with an online softmax (running max, sum and weighted V); the CTA's warps and then
 // the head's splits are combined in fixed order.  Marks the rows used as filled.
 template <typename T>
-__global__ void __launch_bounds__(256) k_attn_core(const AParams p)
+__global__ void __launch_bounds__(256, 1) k_attn_core(const AParams p)
 {
     __shared__ float qs[256];
     __shared__ float wm[8], wz[8];
@@ -311,48 +320,66 @@ __global__ void __launch_bounds__(256) k_attn_core(const AParams p)
         float m = -INFINITY, z = 0.f, o[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) o[e] = 0.f;
-        // lane's elements c = lane E .. lane E + E - 1 of each K/V row; two positions per step
-        // (independent loads), folded into the running softmax in position order
-        auto kv = [&](const T* row, float* f) {
+        // this warp's share of the split's positions, 32 at a time: lane i scores position
+        // base + i (its whole K row in 16-byte loads, issued together), the chunk's running
+        // max and sum follow, then each lane adds p_i V[base + i] over its E elements of the
+        // output, positions in order (eight rows' loads in flight at a time)
+        const int w0 = p0 + (int)((long long)(p1 - p0) * warp / 8), w1 = p0 + (int)((long long)(p1 - p0) * (warp + 1) / 8);
+        const int nvk = dh / 8;
+        const T* Kh = Kc + (size_t)h * p.tmax * dh;
+        const T* Vh = Vc + (size_t)h * p.tmax * dh;
+        for (int base = w0; base < w1; base += 32) {
+            const int n = min(32, w1 - base);
+            float sc = -INFINITY;
+            if (lane < n) {
+                const uint4* kr = reinterpret_cast<const uint4*>(Kh + (size_t)(base + lane) * dh);
+                float a0 = 0.f, a1 = 0.f;
+                auto qdot = [&](const uint4& kv4, int v) {
+                    float kf[8];
+                    unpack8<T>(kv4, kf);
+                    float a = 0.f;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int c = lane * E + e;
-                f[e] = (e < E && c < dh) ? DT<T>::f(row[c]) : 0.f;
+                    for (int e = 0; e < 8; ++e) a = fmaf(qs[8 * v + e], kf[e], a);
+                    return a;
+                };
+                int v = 0;
+                for (; v + 3 < nvk; v += 4) {
+                    const uint4 k0 = __ldcg(kr + v), k1 = __ldcg(kr + v + 1), k2 = __ldcg(kr + v + 2), k3 = __ldcg(kr + v + 3);
+                    a0 += qdot(k0, v); a1 += qdot(k1, v + 1); a0 += qdot(k2, v + 2); a1 += qdot(k3, v + 3);
+                }
+                for (; v < nvk; ++v) a0 += qdot(__ldcg(kr + v), v);
+                sc = (a0 + a1) * scale;
             }
-        };
-        for (int pos = p0 + warp; pos < p1; pos += 16) {
-            const int pos2 = pos + 8;
-            const bool two = pos2 < p1;
-            float k0[8], v0[8], k1[8], v1[8];
-            kv(Kc + ((size_t)h * p.tmax + pos) * dh, k0);
-            kv(Vc + ((size_t)h * p.tmax + pos) * dh, v0);
-            kv(Kc + ((size_t)h * p.tmax + (two ? pos2 : pos)) * dh, k1);
-            kv(Vc + ((size_t)h * p.tmax + (two ? pos2 : pos)) * dh, v1);
-            float part0 = 0.f, part1 = 0.f;
+            float mc = sc;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int c = lane * E + e;
-                const float qc = (e < E && c < dh) ? qs[c] : 0.f;
-                part0 = fmaf(qc, k0[e], part0);
-                part1 = fmaf(qc, k1[e], part1);
-            }
-            const float sc0 = warp_sum(part0) * scale, sc1 = warp_sum(part1) * scale;
-            {
-                const float mn = fmaxf(m, sc0);
-                const float cf = expf(m - mn), ef = expf(sc0 - mn);
-                z = z * cf + ef;
+            for (int off = 16; off > 0; off >>= 1) mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, off));
+            const float mn = fmaxf(m, mc);
+            const float cf = expf(m - mn);
+            const float ev = lane < n ? expf(sc - mn) : 0.f;
+            z = z * cf + warp_sum(ev);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) o[e] = o[e] * cf + ef * v0[e];
-                m = mn;
-            }
-            if (two) {
-                const float mn = fmaxf(m, sc1);
-                const float cf = expf(m - mn), ef = expf(sc1 - mn);
-                z = z * cf + ef;
+            for (int e = 0; e < 8; ++e) o[e] *= cf;
+            for (int i0 = 0; i0 < n; i0 += 8) {
+                float vv[8][8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) o[e] = o[e] * cf + ef * v1[e];
-                m = mn;
+                for (int j = 0; j < 8; ++j) {
+                    const T* vr = Vh + (size_t)(base + i0 + (i0 + j < n ? j : 0)) * dh;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int c = lane * E + e;
+                        vv[j][e] = (e < E && c < dh) ? DT<T>::f(__ldcg(vr + c)) : 0.f;
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (i0 + j < n) {
+                        const float pj = __shfl_sync(0xffffffffu, ev, i0 + j);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) o[e] = fmaf(pj, vv[j][e], o[e]);
+                    }
+                }
             }
+            m = mn;
         }
         if (lane == 0) { wm[warp] = m; wz[warp] = z; }
 #pragma unroll
@@ -411,61 +438,59 @@ __global__ void __launch_bounds__(256) k_attn_core(const AParams p)
 }
 
 // ---------------------------------------------------------------------------
-// 5: output projection over the selected heads' rows of WoT (head-major, each row
-// contiguous): CTA c accumulates o_k[i] WoT[k dh + i] over rows [c R / G, (c+1) R / G)
-// of the R = count dh rows into its fp32 partial.  Thread tid owns 8-column vectors
-// tid + 256 m (d <= 16384).
-template <typename T>
-__global__ void __launch_bounds__(256) k_attn_out(const AParams p)
-{
-    constexpr int kM = 8;
-    const int tid = threadIdx.x, nv = p.d / 8, G = gridDim.x, c = blockIdx.x;
-    const int t = *p.tcur;
-    const int count = t < p.tmax ? *p.count : 0;
-    const int R = count * p.dh;
-    const int r0 = (int)((long long)R * c / G), r1 = (int)((long long)R * (c + 1) / G);
-    float acc[kM][8];
-#pragma unroll
-    for (int m = 0; m < kM; ++m)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[m][e] = 0.f;
-    for (int r = r0; r < r1; ++r) {
-        const int s = r / p.dh, i = r % p.dh, h = p.heads[s];
-        const float a = p.o[(size_t)s * p.dh + i];
-        const uint4* w = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.WoT) + ((size_t)h * p.dh + i) * p.d);
-#pragma unroll
-        for (int m = 0; m < kM; ++m) {
-            const int v = tid + 256 * m;
-            if (v < nv) {
-                float wf[8];
-                unpack8<T>(ldg_stream(w + v), wf);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[m][e] = fmaf(a, wf[e], acc[m][e]);
-            }
-        }
-    }
-    float* dst = p.ypart + (size_t)c * p.d;
-#pragma unroll
-    for (int m = 0; m < kM; ++m) {
-        const int v = tid + 256 * m;
-        if (v < nv) {
-            __stcg(reinterpret_cast<float4*>(dst + v * 8), make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]));
-            __stcg(reinterpret_cast<float4*>(dst + v * 8) + 1, make_float4(acc[m][4], acc[m][5], acc[m][6], acc[m][7]));
-        }
-    }
-}
+// 5: out = bo + sum over the R = count dh selected rows of o_k[i] WoT[k dh + i]
+// (WoT head-major: each row contiguous).  CTA c owns the 8-column vectors
+// [8c, 8c + 8) of out, so no partials leave the CTA: thread (row lane rl, vector
+// j) walks rows rl, rl + 64, ... eight at a time (eight loads in flight), then the
+// 64 row lanes are added in a fixed order.  The last step: the position advances
+// (no CTA of this kernel reads it; a full cache already gave count = 0).
+constexpr int kOutVec = 8, kOutLanes = 64;
 
-// 6: out = bo + the G partials in fixed order; the position advances
 template <typename T>
-__global__ void __launch_bounds__(256) k_attn_reduce(const AParams p, int G)
+__global__ void __launch_bounds__(kOutVec * kOutLanes) k_attn_out(const AParams p)
 {
-    const int col = blockIdx.x * 256 + threadIdx.x;
-    if (col < p.d) {
-        float v = 0.f;
-        for (int g = 0; g < G; ++g) v += __ldcg(p.ypart + (size_t)g * p.d + col);
-        p.out[col] = v + (p.bo ? DT<T>::f(reinterpret_cast<const T*>(p.bo)[col]) : 0.f);
+    __shared__ float red[kOutLanes][kOutVec][8];
+    const int tid = threadIdx.x, j = tid % kOutVec, rl = tid / kOutVec;
+    const int nv = p.d / 8, v = blockIdx.x * kOutVec + j, dh = p.dh;
+    const int R = *p.count * dh;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    const T* Wo = reinterpret_cast<const T*>(p.WoT);
+    auto row_ptr = [&](int r) {
+        const int s = r / dh;
+        return reinterpret_cast<const uint4*>(Wo + ((size_t)p.heads[s] * dh + (r - s * dh)) * p.d) + v;
+    };
+    auto fold = [&](const uint4& w, float a) {
+        float wf[8];
+        unpack8<T>(w, wf);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = fmaf(a, wf[e], acc[e]);
+    };
+    if (v < nv) {
+        int r = rl;
+        for (; r + 7 * kOutLanes < R; r += 8 * kOutLanes) {
+            uint4 w[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) w[k] = ldg_stream(row_ptr(r + k * kOutLanes));
+#pragma unroll
+            for (int k = 0; k < 8; ++k) fold(w[k], __ldcg(p.o + r + k * kOutLanes));
+        }
+        for (; r < R; r += kOutLanes) fold(ldg_stream(row_ptr(r)), __ldcg(p.o + r));
     }
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[rl][j][e] = acc[e];
+    __syncthreads();
+    if (tid < kOutVec * 8) {
+        const int jj = tid / 8, e = tid % 8, vv = blockIdx.x * kOutVec + jj;
+        if (vv < nv) {
+            float sum = 0.f;
+            for (int q = 0; q < kOutLanes; ++q) sum += red[q][jj][e];
+            const int col = vv * 8 + e;
+            p.out[col] = sum + (p.bo ? DT<T>::f(reinterpret_cast<const T*>(p.bo)[col]) : 0.f);
+        }
+    }
+    if (blockIdx.x == 0 && tid == 0) {
         const int t = *p.tcur;
         if (t < p.tmax) *p.tcur = t + 1;
     }
@@ -529,7 +554,6 @@ AParams attn_params(const spffn_attn_ctx& c, const void* y, int32_t* heads, int3
     p.upref = reinterpret_cast<int32_t*>(c.ws + c.lay.upref);
     p.opart = reinterpret_cast<float*>(c.ws + c.lay.opart);
     p.o = reinterpret_cast<float*>(c.ws + c.lay.o);
-    p.ypart = reinterpret_cast<float*>(c.ws + c.lay.ypart);
     p.tickets = reinterpret_cast<uint32_t*>(c.ws + c.lay.tickets);
     p.K = c.ws + c.lay.K;
     p.V = c.ws + c.lay.V;
@@ -545,11 +569,10 @@ cudaError_t step_impl(const spffn_attn_ctx& c, const AParams& p, cudaStream_t st
     cudaError_t e = launch_hidden(c.cfg.dtype, c.w.Wa1, c.w.ba1, p.y, 1, c.cfg.d, c.cfg.Ha,
                                   reinterpret_cast<float*>(c.ws + c.lay.h), G, st);
     if (e != cudaSuccess) return e;
-    k_attn_select<T><<<1, 256, 0, st>>>(p);
+    k_attn_select<T><<<1, kSelWarps * 32, 0, st>>>(p);
     k_attn_qkv<T><<<c.qkv_blocks, 256, 0, st>>>(p);   // every resident warp takes units
     k_attn_core<T><<<G, 256, 0, st>>>(p);
-    k_attn_out<T><<<G, 256, 0, st>>>(p);
-    k_attn_reduce<T><<<(c.cfg.d + 255) / 256, 256, 0, st>>>(p, G);
+    k_attn_out<T><<<(c.cfg.d / 8 + kOutVec - 1) / kOutVec, kOutVec * kOutLanes, 0, st>>>(p);
     return cudaGetLastError();
 }
 
@@ -630,7 +653,7 @@ spffn_status spffn_attn_cache(spffn_attn_ctx* ctx, spffn_attn_cache_view* view) 
     return SPFFN_OK;
 }
 
-int32_t spffn_attn_step_kernel_launches(void) { return 6; }
+int32_t spffn_attn_step_kernel_launches(void) { return 5; }
 
 spffn_status spffn_attn_last_device_error(spffn_attn_ctx* ctx, uint32_t* code, void* stream) {
     if (!ctx) return SPFFN_ERR_INVALID_ARG;

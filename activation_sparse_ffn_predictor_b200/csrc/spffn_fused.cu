@@ -1358,6 +1358,7 @@ int l2_hot_rows() { return g_hot_rows; }
 unsigned long long wait_test_ns() { return g_wait_ns; }
 uint32_t wait_test_bar_extra() { return g_bar_extra; }
 void* trace_buffer(size_t need) { return (g_trace && g_trace_bytes >= need) ? g_trace : nullptr; }
+size_t trace_bytes() { return g_trace ? g_trace_bytes : 0; }
 
 cudaError_t launch_fused_decode(spffn_ctx* const* layers, int L, const void* x_in, int B, void* x_out, float* y,
                                 int32_t* counts, bool lookahead, cudaStream_t st)

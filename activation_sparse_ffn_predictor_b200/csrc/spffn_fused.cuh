@@ -20,6 +20,7 @@ void set_wait_test(unsigned long long limit_ns, bool unmeetable_barrier);
 unsigned long long wait_test_ns();        // current grid-barrier wait limit of the persistent kernels
 uint32_t wait_test_bar_extra();           // extra arrivals their grid barriers expect (0 or 1)
 void* trace_buffer(size_t need);          // the bound trace buffer if at least `need` bytes, else null
+size_t trace_bytes();                     // bytes of the bound trace buffer (0 if none)
 // hot-neuron L2 residency (process-wide): rows per dealt range copied with evict_last (0 = off)
 void set_l2_hot_rows(int rows);
 int l2_hot_rows();

@@ -81,6 +81,62 @@ __global__ void __launch_bounds__(256) k_hidden(const T* __restrict__ Wp1, const
     }
 }
 
+// The same layer for B <= 8 with each row split over four warps of one CTA (two rows
+// per CTA): four times the warps streaming Wp1, so a 1-8 token GEMV keeps enough
+// loads in flight to cover HBM latency.  The four quarter sums are added in a fixed
+// order.
+template <typename T>
+__global__ void __launch_bounds__(256) k_hidden_split(const T* __restrict__ Wp1, const T* __restrict__ bp1,
+                                                      const T* __restrict__ x, int B, int d, int H,
+                                                      float* __restrict__ h)
+{
+    __shared__ float part[8][8];                        // [warp][token]
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int r = blockIdx.x * 2 + (warp >> 2), q = warp & 3;
+    const int nv = d >> 3, v0 = nv * q / 4, v1 = nv * (q + 1) / 4;
+    float acc[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) acc[t] = 0.f;
+    if (r < H) {
+        const uint4* wrow = reinterpret_cast<const uint4*>(Wp1 + (size_t)r * d);
+        auto fold = [&](const uint4& wv, int v) {
+            float w[8];
+            unpack8<T>(wv, w);
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                if (t < B) {
+                    float xv[8];
+                    unpack8<T>(__ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d) + v), xv);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) acc[t] = fmaf(w[k], xv[k], acc[t]);
+                }
+            }
+        };
+        int v = v0 + lane;
+        for (; v + 96 < v1; v += 128) {
+            const uint4 w0 = ldg_stream(wrow + v), w1 = ldg_stream(wrow + v + 32);
+            const uint4 w2 = ldg_stream(wrow + v + 64), w3 = ldg_stream(wrow + v + 96);
+            fold(w0, v); fold(w1, v + 32); fold(w2, v + 64); fold(w3, v + 96);
+        }
+        for (; v < v1; v += 32) fold(ldg_stream(wrow + v), v);
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+        const float sum = warp_sum(acc[t]);
+        if (lane == 0) part[warp][t] = sum;
+    }
+    __syncthreads();
+    if (threadIdx.x < 2 * B) {
+        const int rr = threadIdx.x / B, t = threadIdx.x - rr * B, row = blockIdx.x * 2 + rr;
+        if (row < H) {
+            const float* pr = &part[rr * 4][0];
+            const float sum = (pr[t] + pr[8 + t]) + (pr[16 + t] + pr[24 + t]);
+            const float bias = bp1 ? DT<T>::f(bp1[row]) : 0.f;
+            h[(size_t)t * H + row] = fmaxf(sum + bias, 0.f);
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // S2  predictor output layer + threshold: neuron i selected iff some token has
 // Wp2[i] . h_t + bp2[i] > 0.  A block of 8 warps owns one 32-neuron word.
@@ -404,8 +460,8 @@ static cudaError_t predict_impl(const spffn_ctx& c, const void* x, int B, int32_
                                 int32_t* count2, cudaStream_t st)
 {
     const auto& g = c.cfg;
-    const int hb = min((g.H + 7) / 8, c.num_sms * 8);
-    k_hidden<T><<<hb, 256, 0, st>>>((const T*)c.w.Wp1, (const T*)c.w.bp1, (const T*)x, B, g.d, g.H, c.h());
+    const cudaError_t e = launch_hidden(g.dtype, c.w.Wp1, c.w.bp1, x, B, g.d, g.H, c.h(), c.num_sms, st);
+    if (e != cudaSuccess) return e;
     const int words = g.n / 32;
     k_logits<T><<<words, 256, 0, st>>>((const T*)c.w.Wp2, (const T*)c.w.bp2, c.h(), B, g.H, g.n, c.mask());
     k_compact<<<1, 1024, 0, st>>>(c.mask(), words, idx, count, count2);
@@ -484,6 +540,16 @@ static cudaError_t profile_impl(const spffn_ctx& c, const void* X, int T_, uint3
 cudaError_t launch_hidden(int dtype, const void* W, const void* b, const void* x, int B, int d, int H, float* h,
                           int num_sms, cudaStream_t st)
 {
+    if (B <= 8) {
+        const int hb2 = (H + 1) / 2;
+        if (dtype == SPFFN_BF16)
+            k_hidden_split<__nv_bfloat16><<<hb2, 256, 0, st>>>((const __nv_bfloat16*)W, (const __nv_bfloat16*)b,
+                                                               (const __nv_bfloat16*)x, B, d, H, h);
+        else
+            k_hidden_split<__half><<<hb2, 256, 0, st>>>((const __half*)W, (const __half*)b, (const __half*)x, B, d,
+                                                        H, h);
+        return cudaGetLastError();
+    }
     const int hb = min((H + 7) / 8, num_sms * 8);
     if (dtype == SPFFN_BF16)
         k_hidden<__nv_bfloat16><<<hb, 256, 0, st>>>((const __nv_bfloat16*)W, (const __nv_bfloat16*)b,

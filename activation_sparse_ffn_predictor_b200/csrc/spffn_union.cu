@@ -17,34 +17,47 @@
 // One persistent CTA per SM:
 // - warp 0 issues TMA loads into a ring of 4..6 stages: 2-D tiles for the
 //   contiguous operands (never multicast);
-// - warps 6..9 gather the table rows of FC1 (K-major, 128-byte pieces) and of
+// - warps 6..13 gather the table rows of FC1 (K-major, 128-byte pieces) and of
 //   FC2 (MN-major, 256-byte pieces) with coalesced 16-byte cp.async into the
 //   128-byte swizzled image a TMA tile would leave.  Each thread fences its
 //   landed copies into the async proxy before it arrives.  For both patterns
 //   this moves rows about 1.7-2x faster than TMA tile::gather4;
 // - warp 1 issues tcgen05.mma into a double-buffered TMEM accumulator;
 // - warps 2..5 read TMEM (tcgen05.ld), 16 columns at a time, and run the epilogue.
-// Split-K partials are summed in fixed split order by the last CTA to finish a
-// tile (atomic ticket, no waiting), so results are deterministic.
+// Split-K partials are summed in fixed split order, so results are deterministic:
+// once all splits of a tile have published (an arrival counter, a bounded wait),
+// each split's CTA reduces its own share of the tile's rows, so no single CTA
+// carries the whole reduction as a tail.
 #include <cuda.h>
 #include <algorithm>
 #include <cstring>
 #include "spffn_internal.cuh"
 #include "spffn_umma.cuh"
 #include "spffn_union.cuh"
+#include "spffn_fused.cuh"
 
 namespace spffn {
 namespace {
 using namespace um;
 
-constexpr int kUThreads = 320;       // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue, 6..9 row gathers
-constexpr int kGatherThreads = 128;
+constexpr int kUThreads = 448;       // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue, 6..13 row gathers
+constexpr int kGatherThreads = 256;  // eight gather warps: the gather rate grows with the warps issuing
 constexpr int kBM = 128;             // D rows per tile
 constexpr int kBK = 64;              // K per stage: one 128-byte swizzle row of 16-bit elements
 constexpr int kMaxStages = 6;       // stage = A tile 16 KB + B tile N x 128 B (N <= 256)
 constexpr int kMaxN = 256;           // MMA N per launch; TMEM holds two accumulators of N columns
 constexpr int kGroup = 128;          // tokens per group of the split-activation modes (1, 3)
+constexpr int kTicketDepart = 1024;  // tickets[kTicketDepart + tile]: split CTAs done with a tile (a tile
+                                     // with splits > 1 has index < the CTA count <= kMaxUnionCtas)
 constexpr unsigned long long kUDrainNs = 20000000ull;   // per stage, abort path only
+// Time stamps of one launch (tracing aid, per CTA): 0 set up, 1 TMA lane past the wait for
+// the previous kernel, 2 first stage consumed by the MMA, 3 last MMA issued, 4 last
+// accumulator read, 5 epilogue done (split reduction included), 6 gathers issued, 7 exit.
+constexpr int kUTraceMarks = 8;
+#define UTRACE(mark)                                                                     \
+    do {                                                                                 \
+        if (p.trace) p.trace[(size_t)blockIdx.x * kUTraceMarks + (mark)] = now_ns();     \
+    } while (0)
 
 struct alignas(64) UParams {
     CUtensorMap tmA;      // modes 0, 1: the weight operand (2-D tiles)
@@ -68,6 +81,7 @@ struct alignas(64) UParams {
     float* out_f32;       // mode 0: h [B][H] (may be null); mode 3: y [B][d]
     uint32_t* mask;       // mode 1
     uint32_t* err;
+    unsigned long long* trace;   // null, or this launch's [CTA][kUTraceMarks] time stamps
 };
 
 // Work decomposition shared by all three roles (same answer in every thread).
@@ -114,14 +128,14 @@ __device__ __forceinline__ float tof(const void* base, int i) {
 // token's hi and lo halves Gt columns apart.  Mode 1 ORs its union decision into *any.
 template <typename T>
 __device__ void finish_chunk(const UParams& p, const Plan& q, int tile, int lane_row, int c0, const float* hi,
-                             const float* lo, bool* any)
+                             const float* lo, bool* any, int nc = 16)
 {
     const int r = tile * kBM + lane_row;
     if (p.mode == 0) {                      // h = ReLU(D + bp1) -> fp32 and its hi/lo pair
         if (r < p.H) {
             const float bias = p.bias ? tof<T>(p.bias, r) : 0.f;
             T* hs = reinterpret_cast<T*>(p.out_split);
-            for (int i = 0; i < 16 && c0 + i < p.B; ++i) {
+            for (int i = 0; i < nc && c0 + i < p.B; ++i) {
                 const int t = c0 + i, g = t / p.Gs, tt = t - g * p.Gs;
                 const float h = fmaxf(hi[i] + bias, 0.f);
                 const T h1 = DT<T>::r(h);
@@ -134,7 +148,7 @@ __device__ void finish_chunk(const UParams& p, const Plan& q, int tile, int lane
     } else if (p.mode == 1) {               // union decision over this group's tokens
         if (r < p.n) {
             const float bias = p.bias ? tof<T>(p.bias, r) : 0.f;
-            for (int i = 0; i < 16 && c0 + i < p.Bt; ++i) *any |= (hi[i] + lo[i] + bias) > 0.f;
+            for (int i = 0; i < nc && c0 + i < p.Bt; ++i) *any |= (hi[i] + lo[i] + bias) > 0.f;
         }
     } else if (p.mode == 2) {               // a = ReLU(D + b1[j]) for table entry r (zeros past U)
         T* as = reinterpret_cast<T*>(p.out_split);
@@ -142,7 +156,7 @@ __device__ void finish_chunk(const UParams& p, const Plan& q, int tile, int lane
             const int j = r < q.M ? p.idx[r] : -1;
             const bool live = (unsigned)j < (unsigned)p.n;     // past U or out of range: zero
             const float bias = live ? tof<T>(p.bias, j) : 0.f;
-            for (int i = 0; i < 16 && c0 + i < p.B; ++i) {
+            for (int i = 0; i < nc && c0 + i < p.B; ++i) {
                 const int t = c0 + i, g = t / p.Gs, tt = t - g * p.Gs;
                 const float a = live ? fmaxf(hi[i] + bias, 0.f) : 0.f;
                 const T a1 = DT<T>::r(a);
@@ -154,7 +168,7 @@ __device__ void finish_chunk(const UParams& p, const Plan& q, int tile, int lane
     } else {                                // y[t][c] = D[c][t] + D[c][Gt+t] + b2[c]
         if (r < p.d) {
             const float bias = p.bias ? tof<T>(p.bias, r) : 0.f;
-            for (int i = 0; i < 16 && c0 + i < p.Bt; ++i)
+            for (int i = 0; i < nc && c0 + i < p.Bt; ++i)
                 p.out_f32[(size_t)(p.t_base + c0 + i) * p.d + r] = hi[i] + lo[i] + bias;
         }
     }
@@ -173,7 +187,7 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
     uint64_t* done = tempty + 2;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(done + 1);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 2);
-    int* s_last = reinterpret_cast<int*>(done + 3);
+    int* s_go = reinterpret_cast<int*>(done + 3);      // split-K: every split of the tile is in
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -194,6 +208,7 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    if (threadIdx.x == 0) UTRACE(0);
     // Programmatic dependent launch: the next kernel may launch now (its CTAs take an SM as
     // this kernel's CTA there retires).  Everything read from the previous kernel's outputs
     // waits for it: the table length and rows (modes 2, 3) from the start; in modes 0 and 1
@@ -219,8 +234,12 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
         // previous kernel; their activation tiles follow it
         bool waited = p.mode >= 2;
         int pend_st[kMaxStages], pend_kb[kMaxStages], npend = 0;
+        if (waited && lane == 0) UTRACE(1);
         auto release = [&]() {
-            if (lane == 0) pdl_wait();
+            if (lane == 0) {
+                pdl_wait();
+                UTRACE(1);
+            }
             __syncwarp();
             waited = true;
             for (int i = 0; i < npend; ++i)
@@ -274,7 +293,7 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
         }
     } else if (warp >= 6) {
         // ------------------------------------------------------------- row gathers (modes 2, 3)
-        // Mode 2: 128 threads copy the stage's 128 table rows of W1 (128 bytes each) with 16-byte
+        // Mode 2: 256 threads copy the stage's 128 table rows of W1 (128 bytes each) with 16-byte
         // cp.async into the same 128-byte swizzled image a TMA tile would leave (16-byte
         // chunk c of row r at r*128 + ((c ^ (r & 7)) << 4)); eight consecutive lanes cover
         // one row.  Each thread commits one group per stage and, kLag - 1 stages later, once
@@ -282,20 +301,20 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
         // full barrier.
         if (p.mode >= 2) {
             constexpr int kLag = 4;                      // stages in flight per thread (kStages >= 4)
-            const int t = threadIdx.x - 6 * 32;          // 0..127
+            const int t = threadIdx.x - 6 * 32;          // 0..255
             const int c = t & 7;
             int st = 0, ph = 0, lag_st[kLag] = {0, 0, 0, 0}, nlag = 0;
             bool okg = true;
             // mode 3 (FC2): K block kb is table rows kb*64..+63 of W2T, each contributing its 128
             // output columns of this tile (two 64-column blocks 8 KB apart, K-row r of a block at
             // r*128 with the same 128-byte swizzle); 16 consecutive lanes cover one row's 256 bytes.
-            // Lane t copies chunk (t & 15) of rows t/16 + 8 i.  Rows past U read row 0 (their
+            // Lane t copies chunk (t & 15) of rows t/16 + 16 i.  Rows past U read row 0 (their
             // activations are zero), entries outside [0, n) too (FC1 latched them).
             const int ch = t & 15, mb = ch >> 3, c3 = ch & 7;
             auto fc2_rows = [&](int kb, const char** rows) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int r = kb * kBK + i * 8 + (t >> 4);
+                for (int i = 0; i < 4; ++i) {
+                    const int r = kb * kBK + i * 16 + (t >> 4);
                     int j = r < q.K ? p.idx[r] : 0;
                     j = (unsigned)j < (unsigned)p.n ? j : 0;
                     rows[i] = reinterpret_cast<const char*>(p.W) + (size_t)j * p.d * 2;
@@ -305,13 +324,13 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
                 const int tile = u / q.splits, sp = u % q.splits;
                 const int kb0 = (int)((long long)sp * q.kblocks / q.splits);
                 const int kb1 = (int)((long long)(sp + 1) * q.kblocks / q.splits);
-                // mode 2: rows 16 i + t / 8 of the tile; a table entry outside [0, n) is latched
+                // mode 2: rows 32 i + t / 8 of the tile; a table entry outside [0, n) is latched
                 // and read as row 0 (its activation is zero)
-                const char* rows[8];
+                const char* rows[4];
                 if (p.mode == 2) {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int r = tile * kBM + i * 16 + (t >> 3);
+                    for (int i = 0; i < 4; ++i) {
+                        const int r = tile * kBM + i * 32 + (t >> 3);
                         int j = p.idx[r < q.M ? r : 0];
                         if ((unsigned)j >= (unsigned)p.n) { atomicOr(p.err, ERR_IDX_RANGE); j = 0; }
                         rows[i] = reinterpret_cast<const char*>(p.W) + (size_t)j * p.d * 2 + c * 16;
@@ -325,14 +344,14 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
                     char* sa = base + st * kStageBytes;
                     if (p.mode == 2) {
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int r = i * 16 + (t >> 3);
+                        for (int i = 0; i < 4; ++i) {
+                            const int r = i * 32 + (t >> 3);
                             cp_async16(sa + r * 128 + ((c ^ (r & 7)) << 4), rows[i] + (size_t)kb * kBK * 2);
                         }
                     } else {
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int r = i * 8 + (t >> 4);
+                        for (int i = 0; i < 4; ++i) {
+                            const int r = i * 16 + (t >> 4);
                             cp_async16(sa + mb * 8192 + r * 128 + ((c3 ^ (r & 7)) << 4), rows[i] + col3);
                         }
                         if (kb + 1 < kb1) fc2_rows(kb + 1, rows);      // next block's rows, off the copy path
@@ -351,6 +370,7 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
                     if (++st == kStages) { st = 0; ph ^= 1; }
                 }
             }
+            if (t == 0) UTRACE(6);
             // land and signal what is still in flight
             cp_async_wait<0>();
             fence_async_smem();
@@ -375,6 +395,7 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
                 bool okm = true;
                 for (int kb = kb0; kb < kb1; ++kb) {
                     if (!ub_wait(&full[st], ph, abort_flag, p.err)) { okm = false; break; }
+                    if (!issued && kb == kb0) UTRACE(2);
                     tc_fence_after();
                     const uint32_t sa = s32(base + st * kStageBytes), sb = sa + 16384u;
 #pragma unroll
@@ -392,6 +413,7 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
                 ucommit(&tfull[ab]);
                 if (++ab == 2) { ab = 0; aph ^= 1; }
             }
+            UTRACE(3);
             // every MMA issued by this thread has completed before TMEM is released
             if (issued) {
                 ucommit(done);
@@ -464,50 +486,75 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
                 __syncwarp();
                 if (lane == 0) ub_arrive(&tempty[ab]);
                 if (++ab == 2) { ab = 0; aph ^= 1; }
+                if (et == 0) UTRACE(4);
             }
             if (q.splits == 1) continue;
-            // the last CTA on the tile reduces the splits in split order
+            // split-K: once every split of the tile has published its partial, the CTA of
+            // split sp sums its share of the tile's rows (rows sp kBM / splits ..) over all
+            // splits, in split order.  All splits' CTAs are resident (one unit per CTA), so
+            // the wait is for work already running; it is bounded all the same.
             __threadfence();
             epi_sync();
             if (et == 0) {
-                const uint32_t old = atomicAdd(&p.tickets[tile], 1u);
-                *s_last = old == (uint32_t)(q.splits - 1);
+                atomicAdd(&p.tickets[tile], 1u);
+                const unsigned long long t0 = now_ns();
+                bool okr = true;
+                while (ld_acquire_u32(&p.tickets[tile]) < (uint32_t)q.splits) {
+                    if (now_ns() - t0 > kUWaitNs) {
+                        atomicOr(p.err, ERR_PIPE_TIMEOUT);
+                        okr = false;
+                        break;
+                    }
+                }
+                *s_go = okr;
             }
             epi_sync();
-            if (*s_last) {
+            if (*s_go) {
                 __threadfence();
-                bool any = false;
-                for (int c0 = 0; c0 < half; c0 += 16) {
-                    float hi[16], lo[16];
+                const int r0 = kBM * sp / q.splits, r1 = kBM * (sp + 1) / q.splits;
+                const int nc4 = half / 4;                       // 4-column groups of one half
+                const size_t sstride = (size_t)kBM * N;
+                auto add4 = [](float* a, const float4& w) { a[0] += w.x; a[1] += w.y; a[2] += w.z; a[3] += w.w; };
+                for (int it = et; it < (r1 - r0) * nc4; it += 128) {
+                    const int row = r0 + it / nc4, c0 = (it % nc4) * 4;
+                    const float* src = p.partial + ((size_t)tile * q.splits * kBM + row) * N + c0;
+                    float hi[4] = {0.f, 0.f, 0.f, 0.f}, lo[4] = {0.f, 0.f, 0.f, 0.f};
+                    // four splits' loads out together, summed in split order
+                    for (int s0 = 0; s0 < q.splits; s0 += 4) {
+                        const int ns = min(4, q.splits - s0);
+                        float4 a[4], b[4];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) hi[i] = lo[i] = 0.f;
-                    for (int s = 0; s < q.splits; ++s) {
-                        const float4* src = reinterpret_cast<const float4*>(
-                            p.partial + ((size_t)(tile * q.splits + s) * kBM + lane_row) * N + c0);
-                        float4 w[8];
-#pragma unroll
-                        for (int c4 = 0; c4 < 4; ++c4) {
-                            w[c4] = __ldcg(src + c4);
-                            w[4 + c4] = pair ? __ldcg(src + half / 4 + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+                        for (int k = 0; k < 4; ++k) {
+                            const float* sk = src + (size_t)(s0 + (k < ns ? k : 0)) * sstride;
+                            a[k] = __ldcg(reinterpret_cast<const float4*>(sk));
+                            b[k] = pair ? __ldcg(reinterpret_cast<const float4*>(sk + half)) : make_float4(0.f, 0.f, 0.f, 0.f);
                         }
 #pragma unroll
-                        for (int c4 = 0; c4 < 4; ++c4) {
-                            hi[4 * c4] += w[c4].x; hi[4 * c4 + 1] += w[c4].y;
-                            hi[4 * c4 + 2] += w[c4].z; hi[4 * c4 + 3] += w[c4].w;
-                            lo[4 * c4] += w[4 + c4].x; lo[4 * c4 + 1] += w[4 + c4].y;
-                            lo[4 * c4 + 2] += w[4 + c4].z; lo[4 * c4 + 3] += w[4 + c4].w;
+                        for (int k = 0; k < 4; ++k) {
+                            if (k < ns) {
+                                add4(hi, a[k]);
+                                add4(lo, b[k]);
+                            }
                         }
                     }
-                    finish_chunk<T>(p, q, tile, lane_row, c0, hi, lo, &any);
+                    bool any = false;
+                    finish_chunk<T>(p, q, tile, row, c0, hi, lo, &any, 4);
                 }
-                if (et == 0) p.tickets[tile] = 0u;     // ready for the next call
+            }
+            // the tile's last CTA through here resets its counters for the next call
+            epi_sync();
+            if (et == 0 && atomicAdd(&p.tickets[kTicketDepart + tile], 1u) == (uint32_t)(q.splits - 1)) {
+                p.tickets[tile] = 0u;
+                p.tickets[kTicketDepart + tile] = 0u;
             }
             epi_sync();
         }
+        if (et == 0) UTRACE(5);
     }
     __syncwarp();
     tc_fence_before();
     __syncthreads();
+    if (threadIdx.x == 0) UTRACE(7);
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(p.tmem_cols));
@@ -523,8 +570,25 @@ void size_launch(UParams& p) {
     p.tmem_cols = cols;
 }
 
+// Trace slots: launch i since the trace buffer was bound writes slot i mod (slots held)
+unsigned g_utrace_seq = 0;
+const void* g_utrace_buf = nullptr;
+
+unsigned long long* trace_slot(int grid) {
+    const size_t per = (size_t)grid * kUTraceMarks * sizeof(unsigned long long);
+    void* buf = trace_buffer(per);
+    if (!buf) return nullptr;
+    if (buf != g_utrace_buf) {
+        g_utrace_buf = buf;
+        g_utrace_seq = 0;
+    }
+    const size_t slots = trace_bytes() / per;
+    return static_cast<unsigned long long*>(buf) + (size_t)(g_utrace_seq++ % slots) * grid * kUTraceMarks;
+}
+
 cudaError_t launch(UParams& p, int grid, cudaStream_t st) {
     size_launch(p);
+    p.trace = trace_slot(grid);
     if (p.N > kMaxN || p.stages < 2) return cudaErrorInvalidValue;
     const size_t smem = (size_t)p.stages * p.stage_bytes + 1024 + 256;
     auto kern = p.dtype == SPFFN_BF16 ? k_umma<__nv_bfloat16> : k_umma<__half>;

@@ -410,6 +410,7 @@ def run_true_mask(args, cfg, world, rank, local):
 
     tabs = [[idx[s_, l] for l in range(L)] for s_ in range(K + W)]
     tcnt = cnt[:, :, 0].contiguous()
+    sp.set_l2_hot_rows(args.l2_hot_rows)
 
     def ffn_step(s_):
         sp.decode_tables(layers, xl[0], tabs[s_], tcnt[s_], xl[L], y, stream=stream)

@@ -227,6 +227,12 @@ spffn_status spffn_permute_vector(const void* src, void* dst, int32_t count, con
  * barrier, 10 reduction and table written, 11 after barrier, 12 first
  * predictor-1 chunk computed, 13/14 later predictor-1 chunk ready/computed.
  * A mark a CTA does not reach in a layer (no rows or no neurons) stays 0.
+ * The union path's per-layer tensor-core launches (batches of 16 or more) write
+ * [launch slot][CTA][8] instead, slot i for the i-th such launch since the buffer
+ * was bound (modulo the slots it holds): 0 set up, 1 past the wait for the
+ * previous kernel, 2 first stage consumed, 3 last MMA issued, 4 last accumulator
+ * read, 5 epilogue done, 6 row gathers issued, 7 exit.  A CUDA graph keeps the
+ * slots of the launches it captured.
  * Buffers smaller than that are ignored.  Process-wide; not thread-safe. */
 spffn_status spffn_set_trace(void* buf, size_t bytes);
 int32_t spffn_trace_marks(void);

@@ -167,7 +167,7 @@ def test_attn_graph_replay_and_reset_are_bitwise_repeatable():
 
 
 def test_attn_launch_count():
-    assert sp.attn_step_kernel_launches() == 6
+    assert sp.attn_step_kernel_launches() == 5
 
 
 def test_attn_opt66b_shape():

@@ -250,12 +250,13 @@ int32_t spffn_decode_kernel_launches(spffn_ctx* const* layers, int32_t L, int32_
     for (int l = 0; l < L; ++l)
         if (!layers[l]) return 0;
     if (fused_decode_supported(layers, L, B) || ustack_supported(layers, L, B)) return 1;
-    // per layer: predictor hidden, logits (per token group), compaction, FC1, FC2 (per group), chaining
+    // per layer: predictor hidden, logits, compaction, FC1 (two launches), chaining; on the
+    // union path the compaction runs inside the last logits launch and logits and FC2 run
+    // once per token group
     int n = 0;
-    for (int l = 0; l < L; ++l) {
-        const int g = union_supported(*layers[l], B) ? union_groups(B).groups : 1;
-        n += 4 + 2 * g;
-    }
+    for (int l = 0; l < L; ++l)
+        n += union_supported(*layers[l], B) ? 3 + 2 * union_groups(B).groups + (union_fused_compaction(*layers[l]) ? 0 : 1)
+                                            : 6;
     return n;
 }
 

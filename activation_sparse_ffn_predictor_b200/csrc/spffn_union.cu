@@ -5,7 +5,8 @@
 // the layer runs on the 5th-generation tensor cores:
 //
 //   mode 0  predictor-1   D[H x B]    = Wp1[H x d]        . X[B x d]^T          split-K
-//   mode 1  predictor-2   D[n x 2Gt]  = Wp2[n x H]        . hsplit_g[2Gt x H]^T -> mask words
+//   mode 1  predictor-2   D[n x 2Gt]  = Wp2[n x H]        . hsplit_g[2Gt x H]^T -> mask words;
+//                         the CTA that finishes last compacts the mask into the table
 //   mode 2  FC1 (union)   D[U x B]    = W1[table][U x d]  . X[B x d]^T          split-K
 //   mode 3  FC2 (union)   D[d x 2Gt]  = W2T[table]^T      . asplit_g[2Gt x U]^T split-K
 //
@@ -47,6 +48,7 @@ constexpr int kBK = 64;              // K per stage: one 128-byte swizzle row of
 constexpr int kMaxStages = 6;       // stage = A tile 16 KB + B tile N x 128 B (N <= 256)
 constexpr int kMaxN = 256;           // MMA N per launch; TMEM holds two accumulators of N columns
 constexpr int kGroup = 128;          // tokens per group of the split-activation modes (1, 3)
+constexpr int kTicketCompact = kUnionTickets - 1;   // mode 1: CTAs done with their mask words
 constexpr int kTicketDepart = 1024;  // tickets[kTicketDepart + tile]: split CTAs done with a tile (a tile
                                      // with splits > 1 has index < the CTA count <= kMaxUnionCtas)
 constexpr unsigned long long kUDrainNs = 20000000ull;   // per stage, abort path only
@@ -80,6 +82,9 @@ struct alignas(64) UParams {
     void* out_split;      // mode 0: hsplit, mode 2: asplit: [groups][2][Gs][H or n] hi/lo pairs
     float* out_f32;       // mode 0: h [B][H] (may be null); mode 3: y [B][d]
     uint32_t* mask;       // mode 1
+    int32_t* cidx;        // mode 1, last token group: the CTA finishing last writes the neuron table
+    int32_t* ccount;      //   here, its length here and (if not null) in ccount2
+    int32_t* ccount2;
     uint32_t* err;
     unsigned long long* trace;   // null, or this launch's [CTA][kUTraceMarks] time stamps
 };
@@ -126,51 +131,109 @@ __device__ __forceinline__ float tof(const void* base, int i) {
 // Final epilogue for one D row (this thread's TMEM lane) and 16 columns c0..c0+15
 // of each half.  Modes 0 and 2 keep one column per token; modes 1 and 3 hold each
 // token's hi and lo halves Gt columns apart.  Mode 1 ORs its union decision into *any.
+// Per output row of a tile: its bias and whether it is written (0 no, 1 as zeros: a
+// mode-2 row past U or with an out-of-range table entry, 2 from the accumulators).
+// Loaded before the accumulators are ready, off the epilogue's critical path.
 template <typename T>
-__device__ void finish_chunk(const UParams& p, const Plan& q, int tile, int lane_row, int c0, const float* hi,
-                             const float* lo, bool* any, int nc = 16)
+__device__ __forceinline__ int row_pre(const UParams& p, const Plan& q, int tile, int lane_row, float& bias) {
+    const int r = tile * kBM + lane_row;
+    bias = 0.f;
+    if (p.mode == 2) {
+        if (r >= p.n) return 0;
+        const int j = r < q.M ? p.idx[r] : -1;
+        if ((unsigned)j >= (unsigned)p.n) return 1;
+        bias = tof<T>(p.bias, j);
+        return 2;
+    }
+    const int lim = p.mode == 0 ? p.H : (p.mode == 1 ? p.n : p.d);
+    if (r >= lim) return 0;
+    if (p.bias) bias = tof<T>(p.bias, r);
+    return 2;
+}
+
+// The epilogue of nc accumulator columns c0.. of one tile row (hi, and in modes 1 and 3
+// the matching lo half): state and bias from row_pre.
+template <typename T>
+__device__ void finish_chunk(const UParams& p, int tile, int lane_row, int c0, const float* hi, const float* lo,
+                             bool* any, int nc, int state, float bias)
 {
+    if (state == 0) return;
     const int r = tile * kBM + lane_row;
     if (p.mode == 0) {                      // h = ReLU(D + bp1) -> fp32 and its hi/lo pair
-        if (r < p.H) {
-            const float bias = p.bias ? tof<T>(p.bias, r) : 0.f;
-            T* hs = reinterpret_cast<T*>(p.out_split);
-            for (int i = 0; i < nc && c0 + i < p.B; ++i) {
-                const int t = c0 + i, g = t / p.Gs, tt = t - g * p.Gs;
-                const float h = fmaxf(hi[i] + bias, 0.f);
-                const T h1 = DT<T>::r(h);
-                const T h2 = DT<T>::r(h - DT<T>::f(h1));
-                hs[(size_t)(2 * g * p.Gs + tt) * p.H + r] = h1;
-                hs[(size_t)(2 * g * p.Gs + p.Gs + tt) * p.H + r] = h2;
-                if (p.out_f32) p.out_f32[(size_t)t * p.H + r] = h;
-            }
+        T* hs = reinterpret_cast<T*>(p.out_split);
+        for (int i = 0; i < nc && c0 + i < p.B; ++i) {
+            const int t = c0 + i, g = t / p.Gs, tt = t - g * p.Gs;
+            const float h = fmaxf(hi[i] + bias, 0.f);
+            const T h1 = DT<T>::r(h);
+            const T h2 = DT<T>::r(h - DT<T>::f(h1));
+            hs[(size_t)(2 * g * p.Gs + tt) * p.H + r] = h1;
+            hs[(size_t)(2 * g * p.Gs + p.Gs + tt) * p.H + r] = h2;
+            if (p.out_f32) p.out_f32[(size_t)t * p.H + r] = h;
         }
     } else if (p.mode == 1) {               // union decision over this group's tokens
-        if (r < p.n) {
-            const float bias = p.bias ? tof<T>(p.bias, r) : 0.f;
-            for (int i = 0; i < nc && c0 + i < p.Bt; ++i) *any |= (hi[i] + lo[i] + bias) > 0.f;
-        }
+        for (int i = 0; i < nc && c0 + i < p.Bt; ++i) *any |= (hi[i] + lo[i] + bias) > 0.f;
     } else if (p.mode == 2) {               // a = ReLU(D + b1[j]) for table entry r (zeros past U)
         T* as = reinterpret_cast<T*>(p.out_split);
-        if (r < p.n) {
-            const int j = r < q.M ? p.idx[r] : -1;
-            const bool live = (unsigned)j < (unsigned)p.n;     // past U or out of range: zero
-            const float bias = live ? tof<T>(p.bias, j) : 0.f;
-            for (int i = 0; i < nc && c0 + i < p.B; ++i) {
-                const int t = c0 + i, g = t / p.Gs, tt = t - g * p.Gs;
-                const float a = live ? fmaxf(hi[i] + bias, 0.f) : 0.f;
-                const T a1 = DT<T>::r(a);
-                const T a2 = DT<T>::r(a - DT<T>::f(a1));
-                as[(size_t)(2 * g * p.Gs + tt) * p.n + r] = a1;
-                as[(size_t)(2 * g * p.Gs + p.Gs + tt) * p.n + r] = a2;
-            }
+        for (int i = 0; i < nc && c0 + i < p.B; ++i) {
+            const int t = c0 + i, g = t / p.Gs, tt = t - g * p.Gs;
+            const float a = state == 2 ? fmaxf(hi[i] + bias, 0.f) : 0.f;
+            const T a1 = DT<T>::r(a);
+            const T a2 = DT<T>::r(a - DT<T>::f(a1));
+            as[(size_t)(2 * g * p.Gs + tt) * p.n + r] = a1;
+            as[(size_t)(2 * g * p.Gs + p.Gs + tt) * p.n + r] = a2;
         }
     } else {                                // y[t][c] = D[c][t] + D[c][Gt+t] + b2[c]
-        if (r < p.d) {
-            const float bias = p.bias ? tof<T>(p.bias, r) : 0.f;
-            for (int i = 0; i < nc && c0 + i < p.Bt; ++i)
-                p.out_f32[(size_t)(p.t_base + c0 + i) * p.d + r] = hi[i] + lo[i] + bias;
+        for (int i = 0; i < nc && c0 + i < p.Bt; ++i)
+            p.out_f32[(size_t)(p.t_base + c0 + i) * p.d + r] = hi[i] + lo[i] + bias;
+    }
+}
+
+// Stream compaction of the union mask by all kUThreads threads of one CTA: each thread
+// loads its run of up to kCompactWords words at once (one round trip), a block scan of
+// the popcounts gives its first slot, and it writes its words' set bits in ascending order.
+constexpr int kCompactWords = 8;   // the fused compaction handles n <= kCompactWords * kUThreads * 32
+
+__device__ void compact_mask_cta(const uint32_t* mask, int words, int32_t* idx, int32_t* count, int32_t* count2,
+                                 uint32_t* wsum)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int kWarps = kUThreads / 32;
+    const int per = (words + kUThreads - 1) / kUThreads;
+    const int w0 = min(words, tid * per), w1 = min(words, w0 + per);
+    uint32_t wv[kCompactWords];
+    uint32_t local = 0;
+#pragma unroll
+    for (int k = 0; k < kCompactWords; ++k) {
+        wv[k] = w0 + k < w1 ? __ldcg(mask + w0 + k) : 0u;
+        local += __popc(wv[k]);
+    }
+    uint32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    uint32_t base = 0, total = 0;
+#pragma unroll
+    for (int k = 0; k < kWarps; ++k) {
+        base += k < warp ? wsum[k] : 0u;
+        total += wsum[k];
+    }
+    uint32_t pos = base + incl - local;
+#pragma unroll
+    for (int k = 0; k < kCompactWords; ++k) {
+        uint32_t bits = wv[k];
+        while (bits) {
+            const int b = __ffs(bits) - 1;
+            bits &= bits - 1;
+            idx[pos++] = (w0 + k) * 32 + b;
         }
+    }
+    if (tid == 0) {
+        *count = (int32_t)total;
+        if (count2) *count2 = (int32_t)total;
     }
 }
 
@@ -188,6 +251,7 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
     volatile int* abort_flag = reinterpret_cast<volatile int*>(done + 1);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 2);
     int* s_go = reinterpret_cast<int*>(done + 3);      // split-K: every split of the tile is in
+    __shared__ uint32_t s_wsum[kUThreads / 32];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -437,6 +501,22 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
             const int kb0 = (int)((long long)sp * q.kblocks / q.splits);
             const int kb1 = (int)((long long)(sp + 1) * q.kblocks / q.splits);
             const bool has = kb1 > kb0;
+            // loaded while the accumulators are still being computed: the row's bias and
+            // state (this thread's row, or its first kPre reduction items under split-K)
+            constexpr int kPre = 4;
+            const int r0 = kBM * sp / q.splits, nrows = kBM * (sp + 1) / q.splits - r0;
+            const int items = nrows * (half / 4);
+            float pre_b[kPre];
+            int pre_s[kPre];
+            if (q.splits == 1) {
+                pre_s[0] = row_pre<T>(p, q, tile, lane_row, pre_b[0]);
+            } else {
+#pragma unroll
+                for (int k = 0; k < kPre; ++k) {
+                    const int it = et + 128 * k;
+                    pre_s[k] = it < items ? row_pre<T>(p, q, tile, r0 + it / (half / 4), pre_b[k]) : 0;
+                }
+            }
             uint32_t taddr = 0;
             if (has) {
                 // time bound only: all four epilogue warps leave this wait the same way
@@ -455,7 +535,7 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
                         if (pair) tmem_ld16(taddr + half + c0, lo);
                         tmem_wait_ld();
                     }
-                    finish_chunk<T>(p, q, tile, lane_row, c0, hi, lo, &any);
+                    finish_chunk<T>(p, tile, lane_row, c0, hi, lo, &any, 16, pre_s[0], pre_b[0]);
                 }
                 if (p.mode == 1) {                   // one mask word per 32 rows
                     const uint32_t bits = __ballot_sync(0xffffffffu, any);
@@ -491,8 +571,10 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
             if (q.splits == 1) continue;
             // split-K: once every split of the tile has published its partial, the CTA of
             // split sp sums its share of the tile's rows (rows sp kBM / splits ..) over all
-            // splits, in split order.  All splits' CTAs are resident (one unit per CTA), so
-            // the wait is for work already running; it is bounded all the same.
+            // splits, in split order.  The tile's counter counts arrivals (all splits' CTAs are
+            // resident, one unit per CTA, so the wait is for work already running; it is
+            // bounded all the same); a second counter counts departures, and the last CTA to
+            // leave resets both for the next call.
             __threadfence();
             epi_sync();
             if (et == 0) {
@@ -511,12 +593,11 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
             epi_sync();
             if (*s_go) {
                 __threadfence();
-                const int r0 = kBM * sp / q.splits, r1 = kBM * (sp + 1) / q.splits;
-                const int nc4 = half / 4;                       // 4-column groups of one half
                 const size_t sstride = (size_t)kBM * N;
                 auto add4 = [](float* a, const float4& w) { a[0] += w.x; a[1] += w.y; a[2] += w.z; a[3] += w.w; };
-                for (int it = et; it < (r1 - r0) * nc4; it += 128) {
-                    const int row = r0 + it / nc4, c0 = (it % nc4) * 4;
+                // thread item it: row it / (half / 4) of the share, columns 4 (it % (half / 4)) ..
+                auto reduce_item = [&](int it, int state, float bias) {
+                    const int row = r0 + it / (half / 4), c0 = (it % (half / 4)) * 4;
                     const float* src = p.partial + ((size_t)tile * q.splits * kBM + row) * N + c0;
                     float hi[4] = {0.f, 0.f, 0.f, 0.f}, lo[4] = {0.f, 0.f, 0.f, 0.f};
                     // four splits' loads out together, summed in split order
@@ -538,27 +619,47 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
                         }
                     }
                     bool any = false;
-                    finish_chunk<T>(p, q, tile, row, c0, hi, lo, &any, 4);
+                    finish_chunk<T>(p, tile, row, c0, hi, lo, &any, 4, state, bias);
+                };
+#pragma unroll
+                for (int k = 0; k < kPre; ++k) {
+                    const int it = et + 128 * k;
+                    if (it < items) reduce_item(it, pre_s[k], pre_b[k]);
+                }
+                for (int it = et + 128 * kPre; it < items; it += 128) {
+                    float bias;
+                    const int state = row_pre<T>(p, q, tile, r0 + it / (half / 4), bias);
+                    reduce_item(it, state, bias);
                 }
             }
-            // the tile's last CTA through here resets its counters for the next call
             epi_sync();
             if (et == 0 && atomicAdd(&p.tickets[kTicketDepart + tile], 1u) == (uint32_t)(q.splits - 1)) {
                 p.tickets[tile] = 0u;
                 p.tickets[kTicketDepart + tile] = 0u;
             }
+        }
+        if (p.mode == 1 && p.cidx) {
+            // the CTA whose mask words land last compacts the union mask into the ascending
+            // neuron table, with all its threads, after the final barrier (no separate launch)
+            __threadfence();
             epi_sync();
+            if (et == 0) *s_go = atomicAdd(&p.tickets[kTicketCompact], 1u) == gridDim.x - 1;
         }
         if (et == 0) UTRACE(5);
     }
     __syncwarp();
     tc_fence_before();
     __syncthreads();
-    if (threadIdx.x == 0) UTRACE(7);
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(p.tmem_cols));
     }
+    if (p.mode == 1 && p.cidx && *s_go) {                 // uniform over the CTA
+        __threadfence();
+        compact_mask_cta(p.mask, p.n >> 5, p.cidx, p.ccount, p.ccount2, s_wsum);
+        if (threadIdx.x == 0) p.tickets[kTicketCompact] = 0u;     // ready for the next call
+    }
+    if (threadIdx.x == 0) UTRACE(7);
 }
 
 // stage ring and TMEM allocation for an MMA of N columns
@@ -633,6 +734,8 @@ UnionGroups union_groups(int B) {
     return u;
 }
 
+bool union_fused_compaction(const spffn_ctx& c) { return c.cfg.n / 32 <= kCompactWords * kUThreads; }
+
 bool union_supported(const spffn_ctx& c, int B) {
     return B >= 16 && B <= kMaxBatch && B <= c.cfg.max_batch && c.cfg.d % 128 == 0 && c.lay.upartial != 0 &&
            c.num_sms <= kMaxUnionCtas && encoder() != nullptr;
@@ -673,12 +776,18 @@ cudaError_t union_predict(const spffn_ctx& c, const void* x, int B, int32_t* idx
         q.mask_or = gi > 0;
         q.bias = c.w.bp2;
         q.mask = c.mask();
+        if (gi == ug.groups - 1 && union_fused_compaction(c)) {
+            q.cidx = idx;
+            q.ccount = count;
+            q.ccount2 = count2;
+        }
         if (!make_map(&q.tmA, c.w.Wp2, g.dtype, g.n, g.H, kBM)) return cudaErrorInvalidValue;
         if (!make_map(&q.tmB, c.hsplit(), g.dtype, 2 * ug.groups * ug.Gt, g.H, q.N)) return cudaErrorInvalidValue;
         e = launch(q, c.num_sms, st);
         if (e != cudaSuccess) return e;
     }
-    return launch_compact(c, idx, count, count2, st);
+    if (!union_fused_compaction(c)) return launch_compact(c, idx, count, count2, st);
+    return cudaSuccess;
 }
 
 cudaError_t union_forward(const spffn_ctx& c, const void* x, int B, const int32_t* idx, const int32_t* count,

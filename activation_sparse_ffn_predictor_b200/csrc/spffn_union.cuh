@@ -8,6 +8,8 @@ struct UnionGroups {
 };
 UnionGroups union_groups(int B);
 bool union_supported(const spffn_ctx& c, int B);
+// the table is compacted inside the last logits launch (else by a launch of its own)
+bool union_fused_compaction(const spffn_ctx& c);
 cudaError_t union_predict(const spffn_ctx& c, const void* x, int B, int32_t* idx, int32_t* count, int32_t* count2,
                           cudaStream_t st);
 cudaError_t union_forward(const spffn_ctx& c, const void* x, int B, const int32_t* idx, const int32_t* count,

@@ -51,7 +51,7 @@ def test_timed_path_matches_oracle(name):
     layers = [sp.Layer.from_device_layer(d, max_batch=B) for d in dls]
     # B < 16: the whole stack is one persistent launch, as in the benchmark
     # (the default dispatch: one launch below 16 tokens, per-layer tensor-core kernels from 16)
-    want_launches = 1 if B < 16 else Lc * (4 + 2 * ((B + 127) // 128))
+    want_launches = 1 if B < 16 else Lc * (3 + 2 * ((B + 127) // 128))
     assert sp.decode_kernel_launches(layers, B) == want_launches
     xb, x64 = x_tokens(cfg, B, aux=4000 + 17 * cid + B)
     dt = torch.bfloat16 if cfg.bf16 else torch.float16

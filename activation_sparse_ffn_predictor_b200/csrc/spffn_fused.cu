@@ -322,7 +322,10 @@ __device__ __forceinline__ bool cwait(const Shared& S, const Params& p, uint64_t
     } while (0)
 
 // ---------------------------------------------------------------------------
-template <typename T, int NB, int HV, bool LA, bool TAB>
+// VPT: 16-byte column vectors per consumer thread held in registers (d <= VPT * 8 * kConsumers);
+// the two-token kernels at d <= 4096 use VPT = 2, which keeps their FFN accumulators out of
+// local memory
+template <typename T, int NB, int HV, bool LA, bool TAB, int VPT = kMaxVPT>
 __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ Params p)
 {
     extern __shared__ __align__(128) char smem[];
@@ -498,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         if (l == 0) {
             const T* xin = reinterpret_cast<const T*>(p.x_in);
 #pragma unroll
-            for (int m = 0; m < kMaxVPT; ++m) {
+            for (int m = 0; m < VPT; ++m) {
                 const int v = tid + m * kConsumers;
 #pragma unroll
                 for (int t = 0; t < NB; ++t)
@@ -508,9 +511,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
             }
             return;
         }
-        float4 uv[kMaxVPT][2][NB];
+        float4 uv[VPT][2][NB];
 #pragma unroll
-        for (int m = 0; m < kMaxVPT; ++m) {
+        for (int m = 0; m < VPT; ++m) {
             const int v = tid + m * kConsumers;
 #pragma unroll
             for (int t = 0; t < NB; ++t) {
@@ -528,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
             for (int t = 0; t < NB; ++t) {
                 sq[t] = 0.f;
 #pragma unroll
-                for (int m = 0; m < kMaxVPT; ++m) {
+                for (int m = 0; m < VPT; ++m) {
                     const int v = tid + m * kConsumers;
                     if (v < nvec) {
                         const float4 a = uv[m][0][t], b = uv[m][1][t];
@@ -553,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         for (int t = 0; t < NB; ++t) {
             const float rs = S.misc[t];
 #pragma unroll
-            for (int m = 0; m < kMaxVPT; ++m) {
+            for (int m = 0; m < VPT; ++m) {
                 const int v = tid + m * kConsumers;
                 if (v < nvec) {
                     const float f[8] = {uv[m][0][t].x, uv[m][0][t].y, uv[m][0][t].z, uv[m][0][t].w,
@@ -568,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         if (l == p.L && c == 0 && p.x_out) {
             T* xo = reinterpret_cast<T*>(p.x_out);
 #pragma unroll
-            for (int m = 0; m < kMaxVPT; ++m) {
+            for (int m = 0; m < VPT; ++m) {
                 const int v = tid + m * kConsumers;
                 for (int t = 0; t < B; ++t)
                     if (v < nvec)
@@ -586,9 +589,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
     auto gemv1 = [&](int q) -> bool {
         float* hq = p.h + (size_t)(q & 1) * NB * H;
         const int seg_lo = split_lo(nvec, kConsumerWarps, warp), seg_hi = split_lo(nvec, kConsumerWarps, warp + 1);
-        u64 xg[kMaxVPT][4][NB];
+        u64 xg[VPT][4][NB];
 #pragma unroll
-        for (int m = 0; m < kMaxVPT; ++m) {
+        for (int m = 0; m < VPT; ++m) {
             const int v = seg_lo + lane + 32 * m;
 #pragma unroll
             for (int t = 0; t < NB; ++t) {
@@ -621,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
     #pragma unroll
                         for (int t = 0; t < NB; ++t) cc[u][t] = 0ull;
     #pragma unroll
-                    for (int m = 0; m < kMaxVPT; ++m) {
+                    for (int m = 0; m < VPT; ++m) {
                         const int v = seg_lo + lane + 32 * m;
                         if (v < seg_hi) {
     #pragma unroll
@@ -655,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
     #pragma unroll
                     for (int t = 0; t < NB; ++t) c0[t] = c1[t] = 0ull;
     #pragma unroll
-                    for (int m = 0; m < kMaxVPT; ++m) {
+                    for (int m = 0; m < VPT; ++m) {
                         const int v = seg_lo + lane + 32 * m;
                         if (v < seg_hi) {
                             const uint4 w0 = w0p[v], w1 = w1p[v];
@@ -822,17 +825,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
     auto ffn = [&](int l, int m) -> bool {
         const int32_t* nl = S.nl + (l & 1) * p.max_rows;
         // FC1 operand: this thread's x column vectors, packed storage pairs
-        uint4 xr[kMaxVPT][NB];
+        uint4 xr[VPT][NB];
 #pragma unroll
-        for (int a = 0; a < kMaxVPT; ++a) {
+        for (int a = 0; a < VPT; ++a) {
             const int v = tid + a * kConsumers;
 #pragma unroll
             for (int t = 0; t < NB; ++t)
                 xr[a][t] = v < nvec ? reinterpret_cast<const uint4*>(xs + (size_t)t * d)[v] : make_uint4(0, 0, 0, 0);
         }
-        u64 acc[kMaxVPT][4][NB];
+        u64 acc[VPT][4][NB];
 #pragma unroll
-        for (int a = 0; a < kMaxVPT; ++a)
+        for (int a = 0; a < VPT; ++a)
 #pragma unroll
             for (int q = 0; q < 4; ++q)
 #pragma unroll
@@ -855,7 +858,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
 #pragma unroll
                     for (int u = 0; u < 4; ++u) part[u][0] = part[u][1] = part[u][2] = part[u][3] = 0.f;
 #pragma unroll
-                    for (int a = 0; a < kMaxVPT; ++a) {
+                    for (int a = 0; a < VPT; ++a) {
                         const int v = tid + a * kConsumers;
                         if (v < nvec) {
 #pragma unroll
@@ -880,7 +883,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
                     }
                     rpar ^= 1;
 #pragma unroll
-                    for (int a = 0; a < kMaxVPT; ++a) {
+                    for (int a = 0; a < VPT; ++a) {
                         const int v = tid + a * kConsumers;
                         if (v < nvec) {
 #pragma unroll
@@ -915,7 +918,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
 #pragma unroll
                 for (int t = 0; t < NB; ++t) part[u][t][0] = part[u][t][1] = part[u][t][2] = part[u][t][3] = 0.f;
 #pragma unroll
-            for (int a = 0; a < kMaxVPT; ++a) {
+            for (int a = 0; a < VPT; ++a) {
                 const int v = tid + a * kConsumers;
                 if (v < nvec) {
                     const uint4 w0 = reinterpret_cast<const uint4*>(sl0)[v];
@@ -953,7 +956,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
             }
             rpar ^= 1;
 #pragma unroll
-            for (int a = 0; a < kMaxVPT; ++a) {
+            for (int a = 0; a < VPT; ++a) {
                 const int v = tid + a * kConsumers;
                 if (v < nvec) {
                     const uint4 w0 = reinterpret_cast<const uint4*>(sl0 + 2 * d)[v];
@@ -984,7 +987,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
             if (!two) fk -= 1;               // only one slot consumed
         }
 #pragma unroll
-        for (int a = 0; a < kMaxVPT; ++a) {
+        for (int a = 0; a < VPT; ++a) {
             const int v = tid + a * kConsumers;
             if (v < nvec) {
 #pragma unroll
@@ -1253,7 +1256,7 @@ Geometry geometry(const spffn_config& c, int G, bool lookahead, bool tables = fa
     return g;
 }
 
-template <typename T, int NB, int HV, bool LA, bool TAB = false>
+template <typename T, int NB, int HV, bool LA, bool TAB = false, int VPT = kMaxVPT>
 cudaError_t launch_t(spffn_ctx* const* layers, int L, const void* x_in, int B, void* x_out, float* y,
                      int32_t* counts, cudaStream_t st, const int32_t* const* tabs = nullptr,
                      const int32_t* const* tab_counts = nullptr)
@@ -1288,7 +1291,7 @@ cudaError_t launch_t(spffn_ctx* const* layers, int L, const void* x_in, int B, v
         p.layer[l] = LayerW{c.w.W1, c.w.b1, c.w.W2T, c.w.b2, c.w.Wp1, c.w.bp1, c.w.Wp2, c.w.bp2, c.idx(),
                             tables ? tabs[l] : nullptr, tables ? tab_counts[l] : nullptr};
     }
-    cudaError_t e = cudaFuncSetAttribute(k_decode<T, NB, HV, LA, TAB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem);
+    cudaError_t e = cudaFuncSetAttribute(k_decode<T, NB, HV, LA, TAB, VPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem);
     if (e != cudaSuccess) return e;
     e = cudaMemsetAsync(&ctl->barrier[0], 0, 2 * sizeof(uint32_t), st);
     if (e != cudaSuccess) return e;
@@ -1302,7 +1305,21 @@ cudaError_t launch_t(spffn_ctx* const* layers, int L, const void* x_in, int B, v
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_decode<T, NB, HV, LA, TAB>, p);
+    return cudaLaunchKernelEx(&cfg, k_decode<T, NB, HV, LA, TAB, VPT>, p);
+}
+
+// the two-token kernels at d <= 4096 keep two column vectors per thread (VPT = 2)
+template <typename T, int NB, int HV>
+cudaError_t launch_vpt(bool lookahead, bool narrow, spffn_ctx* const* layers, int L, const void* x_in, int B,
+                       void* x_out, float* y, int32_t* counts, cudaStream_t st)
+{
+    if constexpr (NB == 2) {
+        if (narrow)
+            return lookahead ? launch_t<T, NB, HV, true, false, 2>(layers, L, x_in, B, x_out, y, counts, st)
+                             : launch_t<T, NB, HV, false, false, 2>(layers, L, x_in, B, x_out, y, counts, st);
+    }
+    return lookahead ? launch_t<T, NB, HV, true>(layers, L, x_in, B, x_out, y, counts, st)
+                     : launch_t<T, NB, HV, false>(layers, L, x_in, B, x_out, y, counts, st);
 }
 
 }  // namespace
@@ -1365,9 +1382,9 @@ cudaError_t launch_fused_decode(spffn_ctx* const* layers, int L, const void* x_i
 {
     const bool bf = layers[0]->cfg.dtype == SPFFN_BF16;
     const int hvn = (layers[0]->cfg.H + 255) / 256;
-#define SPFFN_GO(TT, NBV, HVV)                                                                        \
-    return lookahead ? launch_t<TT, NBV, HVV, true>(layers, L, x_in, B, x_out, y, counts, st)         \
-                     : launch_t<TT, NBV, HVV, false>(layers, L, x_in, B, x_out, y, counts, st)
+    const bool narrow = layers[0]->cfg.d <= 2 * 8 * kConsumers;      // two column vectors per thread
+#define SPFFN_GO(TT, NBV, HVV) \
+    return launch_vpt<TT, NBV, HVV>(lookahead, narrow, layers, L, x_in, B, x_out, y, counts, st)
 #define SPFFN_HV(TT, NBV)                                     \
     if (hvn <= 1) SPFFN_GO(TT, NBV, 1);                       \
     if (hvn <= 2) SPFFN_GO(TT, NBV, 2);                       \
@@ -1392,6 +1409,9 @@ cudaError_t launch_fused_tables(spffn_ctx* const* layers, int L, const void* x_i
         return bf ? launch_t<__nv_bfloat16, 1, 1, false, true>(layers, L, x_in, B, x_out, y, counts, st, tabs, tab_counts)
                   : launch_t<__half, 1, 1, false, true>(layers, L, x_in, B, x_out, y, counts, st, tabs, tab_counts);
     }
+    if (layers[0]->cfg.d <= 2 * 8 * kConsumers)
+        return bf ? launch_t<__nv_bfloat16, 2, 1, false, true, 2>(layers, L, x_in, B, x_out, y, counts, st, tabs, tab_counts)
+                  : launch_t<__half, 2, 1, false, true, 2>(layers, L, x_in, B, x_out, y, counts, st, tabs, tab_counts);
     return bf ? launch_t<__nv_bfloat16, 2, 1, false, true>(layers, L, x_in, B, x_out, y, counts, st, tabs, tab_counts)
               : launch_t<__half, 2, 1, false, true>(layers, L, x_in, B, x_out, y, counts, st, tabs, tab_counts);
 }

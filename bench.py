@@ -156,14 +156,39 @@ DECODE_TRAFFIC = {
 }
 
 
-def decode_sources_sha256() -> str:
+# DRAM traffic of the union path's per-layer launches (predictor modes, FC1, FC2, chaining),
+# from one capture of a 2-layer stack of the OPT-66B-shaped workload at batch 32: per layer
+# a fixed part (predictor weights, chaining) plus a part per table neuron (its W1 and W2T
+# rows), so a run's traffic is scaled by the neurons its layers actually selected.  It holds
+# only for the kernel sources it was captured on: any change to them and the bench reports null.
+UNION_SOURCES = ("spffn_union.cu", "spffn_umma.cuh", "spffn_internal.cuh", "spffn_kernels.cu")
+UNION_TRAFFIC = {
+    "sha256": "e240df62a72353947775f916e542506828a96d4b900f258ada38bee9bd393a39",
+    "workload": "opt66b-d9216-n36864-L64", "batch": 32, "rate": 0.01,
+    "fixed_per_layer": 38.44e6 + 151.90e6 + 1.78e6,
+    "per_neuron": (105.21e6 + 105.36e6) / 5639.17,
+}
+
+
+def decode_sources_sha256(files=DECODE_SOURCES) -> str:
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "activation_sparse_ffn_predictor_b200", "csrc")
-    for f in DECODE_SOURCES:
+    for f in files:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
+
+
+def union_traffic(cfg, batch: int, rate, lookahead: bool, per_layer_counts):
+    """DRAM bytes per step of the union path for this run (mean over the timed steps), or None."""
+    t = UNION_TRAFFIC
+    if lookahead or cfg.name != t["workload"] or batch != t["batch"] or (rate or cfg.rate) != t["rate"]:
+        return None
+    if decode_sources_sha256(UNION_SOURCES) != t["sha256"]:
+        return None
+    steps = [t["fixed_per_layer"] * len(row) + t["per_neuron"] * float(sum(row)) for row in per_layer_counts]
+    return sum(steps) / len(steps)
 
 
 def decode_traffic(cfg, layers: int, batch: int, rate, lookahead: bool):
@@ -355,6 +380,17 @@ def run_ours(args, cfg, world, rank, local):
         f1.record(stream)
     stream.synchronize()
     e2e_ms = max_over_ranks(f0.elapsed_time(f1), world, device)
+    if args.trace and launches_per_step > 1 and B >= 16 and B <= 128 and rank == 0:
+        # one more eager step with per-CTA phase stamps (outside every timed region)
+        nl = 4 * L
+        G = layers[0].num_partials
+        buf = torch.zeros(nl * G * 8, dtype=torch.int64, device=device)
+        sp.set_trace(buf)
+        with torch.cuda.stream(stream):
+            one_step()
+        stream.synchronize()
+        sp.set_trace(None)
+        print(union_phase_table(buf.cpu().numpy(), nl, G), file=sys.stderr, flush=True)
 
     value = world * B * K / (t_max * 1e-3)
     res = {
@@ -367,7 +403,8 @@ def run_ours(args, cfg, world, rank, local):
                            "placement_ranges": layers[0].num_partials},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak,
-                     "traffic": decode_traffic(cfg, L, B, args.rate, args.lookahead) if launches_per_step == 1 else None,
+                     "traffic": (decode_traffic(cfg, L, B, args.rate, args.lookahead) if launches_per_step == 1
+                                 else union_traffic(cfg, B, args.rate, args.lookahead, ks.tolist())),
                      "kernel": "spffn decode step (one graph replay per step, %d launch%s)"
                                % (launches_per_step, "" if launches_per_step == 1 else "es"),
                      "peak_kind": peak_kind},
@@ -378,6 +415,36 @@ def run_ours(args, cfg, world, rank, local):
         "clocks": clk.summary(),
     }
     return res, (rank == 0)
+
+
+def union_phase_table(stamps, launches: int, ctas: int) -> str:
+    """Phase summary of one traced step of the union path's per-layer launches (four
+    tensor-core launches per layer): per mode, the median over layers of the wait for the
+    previous kernel, the streaming span (first stage consumed to last MMA issued) and the
+    tail (last accumulator read to the last CTA's epilogue end), in microseconds."""
+    t = stamps.reshape(launches, ctas, 8).astype(np.float64)
+    rows = {m: [] for m in range(4)}
+    for i in range(launches):
+        m0 = t[i][:, 0]
+        if not (m0 > 0).any():
+            continue
+        start = m0[m0 > 0].min()
+
+        def med(k):
+            v = t[i][:, k]
+            v = v[v > 0]
+            return float(np.median(v)) if v.size else float("nan")
+
+        last5 = t[i][:, 5]
+        tail_end = last5[last5 > 0].max() if (last5 > 0).any() else float("nan")
+        rows[i % 4].append(((med(1) - start) / 1e3, (med(3) - med(2)) / 1e3, (tail_end - med(4)) / 1e3))
+    names = ["mode 0 (predictor hidden)", "mode 1 (logits, compaction)", "mode 2 (FC1)", "mode 3 (FC2)"]
+    out = ["%-30s %12s %12s %12s" % ("launch", "wait us", "stream us", "tail us")]
+    for m in range(4):
+        if rows[m]:
+            a = np.median(np.array(rows[m]), axis=0)
+            out.append("%-30s %12.1f %12.1f %12.1f" % (names[m], a[0], a[1], a[2]))
+    return "\n".join(out)
 
 
 def run_true_mask(args, cfg, world, rank, local):
@@ -847,6 +914,9 @@ def main(argv=None):
     ap.add_argument("--attn", action="store_true",
                     help="head-sparse attention decode with the attention-head predictor (its own metric)")
     ap.add_argument("--attn-config", type=int, default=1)
+    ap.add_argument("--trace", action="store_true",
+                    help="union path (16 <= B <= 128, per-layer launches): after the timed runs, print a "
+                         "phase table of one traced step to stderr")
     ap.add_argument("--dense", action="store_true",
                     help="comparison arm: the dense FFN of every layer with cuBLAS on the same weights")
     args = ap.parse_args(argv)

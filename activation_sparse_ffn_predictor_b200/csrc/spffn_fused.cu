@@ -740,6 +740,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
             unsigned char* sel = S.sel + (pk_ & 1) * 32;
             if (!cwait(S, p, &S.pfull[s], (pk_ / p.pred_slots) & 1)) return -1;
             if (r == b0) TRACE(5);
+            if (r == b0 + 3 * R2) TRACE(12);
+            if (r + R2 >= b1) TRACE(14);
             const uint4* slot = reinterpret_cast<const uint4*>(S.pring + (size_t)s * p.pred_slot_bytes);
             const int rows = min(R2, b1 - r);
             // two rows per warp per step for independent FMA chains
@@ -787,8 +789,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
                 }
             }
             __syncwarp();
+            if (r + R2 >= b1) TRACE(15);
             if (lane == 0) mbar_arrive(&S.pempty[s]);
             consumer_sync();
+            if (r == b0 + 3 * R2) TRACE(13);
             // append this chunk's selected rows in ascending order and publish the count
             if (warp == 0) {
                 for (int q0 = 0; q0 < rows; q0 += 32) {

@@ -380,6 +380,17 @@ def run_ours(args, cfg, world, rank, local):
         f1.record(stream)
     stream.synchronize()
     e2e_ms = max_over_ranks(f0.elapsed_time(f1), world, device)
+    if args.trace and launches_per_step == 1 and B <= 2 and rank == 0:
+        # one more eager step with per-CTA, per-layer phase stamps (outside every timed region)
+        G = layers[0].num_partials
+        M = sp.trace_marks()
+        buf = torch.zeros(G * L * M, dtype=torch.int64, device=device)
+        sp.set_trace(buf)
+        with torch.cuda.stream(stream):
+            one_step()
+        stream.synchronize()
+        sp.set_trace(None)
+        print(fused_phase_table(buf.cpu().numpy(), G, L, M), file=sys.stderr, flush=True)
     if args.trace and launches_per_step > 1 and B >= 16 and B <= 128 and rank == 0:
         # one more eager step with per-CTA phase stamps (outside every timed region)
         nl = 4 * L
@@ -444,6 +455,37 @@ def union_phase_table(stamps, launches: int, ctas: int) -> str:
         if rows[m]:
             a = np.median(np.array(rows[m]), axis=0)
             out.append("%-30s %12.1f %12.1f %12.1f" % (names[m], a[0], a[1], a[2]))
+    return "\n".join(out)
+
+
+FUSED_MARKS = {0: "input formed", 1: "first predictor-1 chunk ready", 2: "hidden layer done",
+               3: "after barrier 1", 4: "h loaded", 5: "first predictor-2 chunk ready",
+               6: "own neuron list final", 7: "first FFN rows ready", 8: "FFN partial written",
+               9: "after barrier 2", 10: "reduction and table written", 11: "after barrier 3",
+               12: "4th predictor-2 chunk ready", 13: "4th chunk computed", 14: "last predictor-2 chunk ready",
+               15: "last chunk computed"}
+
+
+def fused_phase_table(stamps, ctas: int, layers: int, marks: int) -> str:
+    """Phase summary of one traced step of the small-batch whole-stack kernel: per mark,
+    the median over layers of the median (and max) over CTAs of the time since the
+    layer's earliest "input formed" stamp, and the median layer period, in microseconds."""
+    t = stamps.reshape(ctas, layers, marks).astype(np.float64)
+    t0 = np.array([t[:, l, 0][t[:, l, 0] > 0].min() if (t[:, l, 0] > 0).any() else np.nan for l in range(layers)])
+    out = ["%-32s %10s %10s" % ("mark", "median us", "max us")]
+    for m, name in FUSED_MARKS.items():
+        med, mx = [], []
+        for l in range(1, layers):                      # layer 0 includes the launch
+            v = t[:, l, m]
+            v = v[v > 0] - t0[l]
+            if v.size:
+                med.append(np.median(v) / 1e3)
+                mx.append(v.max() / 1e3)
+        if med:
+            out.append("%-32s %10.1f %10.1f" % (name, np.median(med), np.median(mx)))
+    per = np.diff(t0[1:]) / 1e3
+    if per.size:
+        out.append("%-32s %10.1f" % ("layer period", float(np.median(per))))
     return "\n".join(out)
 
 
@@ -915,8 +957,8 @@ def main(argv=None):
                     help="head-sparse attention decode with the attention-head predictor (its own metric)")
     ap.add_argument("--attn-config", type=int, default=1)
     ap.add_argument("--trace", action="store_true",
-                    help="union path (16 <= B <= 128, per-layer launches): after the timed runs, print a "
-                         "phase table of one traced step to stderr")
+                    help="after the timed runs, print a phase table of one traced step to stderr (the "
+                         "small-batch whole-stack kernel, or the union path's per-layer launches)")
     ap.add_argument("--dense", action="store_true",
                     help="comparison arm: the dense FFN of every layer with cuBLAS on the same weights")
     args = ap.parse_args(argv)

@@ -224,8 +224,9 @@ spffn_status spffn_permute_vector(const void* src, void* dst, int32_t count, con
  * 0 input formed, 1 first predictor-1 chunk ready, 2 hidden layer done,
  * 3 after barrier, 4 h loaded, 5 first predictor-2 chunk ready, 6 own
  * neuron list final, 7 first FFN rows ready, 8 FFN partial written, 9 after
- * barrier, 10 reduction and table written, 11 after barrier, 12 first
- * predictor-1 chunk computed, 13/14 later predictor-1 chunk ready/computed.
+ * barrier, 10 reduction and table written, 11 after barrier, 12 fourth
+ * predictor-2 chunk ready, 13 fourth chunk's rows computed by every warp, 14 last
+ * predictor-2 chunk ready, 15 last chunk's rows computed (thread 0).
  * A mark a CTA does not reach in a layer (no rows or no neurons) stays 0.
  * The union path's per-layer tensor-core launches (batches of 16 or more) write
  * [launch slot][CTA][8] instead, slot i for the i-th such launch since the buffer

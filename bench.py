@@ -212,21 +212,32 @@ class Clocks:
         self._stop = threading.Event()
         self._t = None
 
+    def _sample(self):
+        nv = self._nv
+        sm = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+        rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        self.rows.append((sm, self._mx, rs))
+
     def _run(self):
         try:
-            import pynvml as nv
-            nv.nvmlInit()
-            h = nv.nvmlDeviceGetHandleByIndex(self.index)
-            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
-            while not self._stop.is_set():
-                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
-                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-                self.rows.append((sm, mx, rs))
-                self._stop.wait(self.period)
-        except Exception as e:  # NVML missing: leave the record empty and say why
+            while not self._stop.wait(self.period):
+                self._sample()
+        except Exception as e:
             self.error = repr(e)
 
     def __enter__(self):
+        # NVML is opened and sampled once before the timed work starts, so a timed region
+        # shorter than the sampling period still has a record (plus one at its end)
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self._nv = nv
+            self._h = nv.nvmlDeviceGetHandleByIndex(self.index)
+            self._mx = nv.nvmlDeviceGetMaxClockInfo(self._h, nv.NVML_CLOCK_SM)
+            self._sample()
+        except Exception as e:  # NVML missing: leave the record empty and say why
+            self.error = repr(e)
+            return self
         self._t = threading.Thread(target=self._run, daemon=True)
         self._t.start()
         return self
@@ -235,6 +246,10 @@ class Clocks:
         self._stop.set()
         if self._t:
             self._t.join(timeout=10)
+            try:
+                self._sample()
+            except Exception as e:
+                self.error = repr(e)
 
     def summary(self):
         if not self.rows:

@@ -397,8 +397,8 @@ UNION_PER_LAYER, UNION_STACK, UNION_AUTO = 0, 1, 2
 
 def set_union_stack(mode: int):
     """How decode runs 3 <= B <= 128 (spffn_set_union_stack): UNION_STACK (one
-    persistent launch), UNION_PER_LAYER, or UNION_AUTO (the default: the whole
-    stack below 16 tokens, per-layer launches from 16 up)."""
+    persistent launch), UNION_PER_LAYER, or UNION_AUTO (the default: the faster
+    of the two on the measured shapes, per-layer launches at every batch)."""
     _check(library().spffn_set_union_stack(int(mode)), "spffn_set_union_stack")
 
 

@@ -1,4 +1,4 @@
-// Union-mask tensor-core path for batches of 16..256 tokens.
+// Union-mask tensor-core path for batches of 3..256 tokens (below 16 the MMA's N is padded to 16).
 //
 // With B tokens the union of the per-token neuron sets is a dense contraction
 // over the gathered rows (each weight byte feeds B products), so every GEMM of
@@ -737,7 +737,7 @@ UnionGroups union_groups(int B) {
 bool union_fused_compaction(const spffn_ctx& c) { return c.cfg.n / 32 <= kCompactWords * kUThreads; }
 
 bool union_supported(const spffn_ctx& c, int B) {
-    return B >= 16 && B <= kMaxBatch && B <= c.cfg.max_batch && c.cfg.d % 128 == 0 && c.lay.upartial != 0 &&
+    return B >= kUStackMinBatch && B <= kMaxBatch && B <= c.cfg.max_batch && c.cfg.d % 128 == 0 && c.lay.upartial != 0 &&
            c.num_sms <= kMaxUnionCtas && encoder() != nullptr;
 }
 

@@ -805,9 +805,10 @@ void ustack_geometry(int B, int& N1, int& N2, int& stages, int& stage_bytes, int
 }
 
 // spffn_set_union_stack: 0 per-layer launches, 1 whole stack for 3 <= B <= 128, 2 (default)
-// whole stack below 16 tokens only: from 16 up the per-layer tensor-core kernels, chained by
-// programmatic dependent launch, measured faster (OPT-13B shape at B = 16: 3.1 vs 4.0 ms per
-// step; OPT-66B shape at B = 32: 7.7 vs 9.8 ms), and below 16 slower (B = 4: 6.8 vs 3.5 ms)
+// the faster of the two on the measured shapes, which is per-layer at every batch: the
+// per-layer tensor-core kernels, chained by programmatic dependent launch, measured faster at
+// B = 3, 4, 8 (OPT-13B shape: 2.40 / 2.44 / 2.52 vs 3.14 / 3.20 / 3.31 ms per step), B = 16
+// (2.63 vs 3.97 ms) and B = 32 (OPT-66B shape: 6.57 vs 9.83 ms)
 int g_ustack_mode = 2;
 
 }  // namespace
@@ -817,7 +818,7 @@ int ustack_mode() { return g_ustack_mode; }
 
 bool ustack_supported(spffn_ctx* const* layers, int L, int B)
 {
-    if (g_ustack_mode == 0 || (g_ustack_mode == 2 && B >= 16)) return false;
+    if (g_ustack_mode != 1) return false;
     // batches below 16 pad the MMA's N to 16 columns: idle tensor-core lanes, the same bytes
     if (L < 1 || L > kSMaxLayers || B < kUStackMinBatch || B > 128) return false;
     const spffn_ctx& c0 = *layers[0];

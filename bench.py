@@ -961,7 +961,7 @@ def main(argv=None):
                     help="keep this many of the hottest slots of every dealt range in L2 (B <= 2 decode)")
     ap.add_argument("--union-stack", type=int, choices=[0, 1, 2], default=2,
                     help="decode 3 <= B <= 128: 0 per-layer launches, 1 one whole-stack launch, 2 (default) "
-                         "whole stack below 16 tokens")
+                         "the faster on the measured shapes (per-layer)")
     ap.add_argument("--flush-l2", action="store_true",
                     help="write a buffer larger than L2 before every timed step (for workloads that fit in L2)")
     ap.add_argument("--lookahead", action="store_true",

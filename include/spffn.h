@@ -242,11 +242,12 @@ int32_t spffn_trace_marks(void);
  * every layer of one shape, at most 64 layers, no look-ahead):
  *   1  the whole stack as one persistent launch on the union tensor-core path,
  *      with the weights of the next phase streaming across its grid barriers;
- *   0  per-layer launches (the predictor kernels, the compaction, FC1/FC2 and
- *      the chaining for every layer; at B >= 16 the tensor-core kernels of
- *      spffn_predict / spffn_forward, chained by programmatic dependent launch);
- *   2  (the default) 1 below 16 tokens, 0 from 16 up: the faster of the two on
- *      the measured shapes.
+ *   0  per-layer launches (the tensor-core kernels of spffn_predict and
+ *      spffn_forward plus the chaining for every layer, chained by programmatic
+ *      dependent launch; the per-phase kernels where the union path does not
+ *      apply);
+ *   2  (the default) the faster of the two on the measured shapes, which is 0
+ *      at every batch from 3 to 128.
  * Both compute the same function; their fp32 reductions run in different
  * orders, so results agree to rounding.  Process-wide; applies to calls made
  * afterwards; INVALID_ARG outside 0..2.  spffn_union_stack returns the mode. */

@@ -49,9 +49,9 @@ def test_timed_path_matches_oracle(name):
     cfg = wl.CONFIGS[cid]
     dls = [wl.device_layer(cfg, l, rate=rate) for l in range(Lc)]
     layers = [sp.Layer.from_device_layer(d, max_batch=B) for d in dls]
-    # B < 16: the whole stack is one persistent launch, as in the benchmark
-    # (the default dispatch: one launch below 16 tokens, per-layer tensor-core kernels from 16)
-    want_launches = 1 if B < 16 else Lc * (3 + 2 * ((B + 127) // 128))
+    # the default dispatch, as in the benchmark: B <= 2 the whole stack in one persistent
+    # launch, from 3 tokens per-layer tensor-core launches (five per layer and token group)
+    want_launches = 1 if B <= 2 else Lc * (3 + 2 * ((B + 127) // 128))
     assert sp.decode_kernel_launches(layers, B) == want_launches
     xb, x64 = x_tokens(cfg, B, aux=4000 + 17 * cid + B)
     dt = torch.bfloat16 if cfg.bf16 else torch.float16
@@ -72,16 +72,16 @@ def test_timed_path_matches_oracle(name):
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("cid,Lc,B,mode", [(4, 2, 32, 1), (2, 2, 16, 1), (2, 2, 4, 0)])
+@pytest.mark.parametrize("cid,Lc,B,mode", [(4, 2, 32, 1), (2, 2, 16, 1), (2, 2, 4, 1), (2, 2, 4, 0)])
 def test_other_union_dispatch_matches_oracle(cid, Lc, B, mode):
-    """The dispatch the default does not pick at this batch: the whole-stack
-    kernel at B >= 16 (mode 1), per-layer launches below 16 (mode 0)."""
+    """The whole-stack kernel (mode 1, which the default does not pick) and
+    explicit per-layer launches (mode 0)."""
     cfg = wl.CONFIGS[cid]
     dls = [wl.device_layer(cfg, l) for l in range(Lc)]
     layers = [sp.Layer.from_device_layer(d, max_batch=B) for d in dls]
     try:
         sp.set_union_stack(mode)
-        assert sp.decode_kernel_launches(layers, B) == (1 if mode == 1 else Lc * 6)
+        assert sp.decode_kernel_launches(layers, B) == (1 if mode == 1 else Lc * 5)
         xb, x64 = x_tokens(cfg, B, aux=4100 + cid)
         dt = torch.bfloat16 if cfg.bf16 else torch.float16
         x_out = torch.empty(B, cfg.d, dtype=dt, device="cuda")

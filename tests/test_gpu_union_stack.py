@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 @pytest.fixture(autouse=True)
 def whole_stack_mode():
     """These tests run the whole-stack kernel at every batch it serves (the
-    default picks it below 16 tokens only)."""
+    default dispatch uses per-layer launches)."""
     sp.set_union_stack(sp.UNION_STACK)
     yield
     sp.set_union_stack(sp.UNION_AUTO)

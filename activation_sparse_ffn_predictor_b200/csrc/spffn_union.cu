@@ -48,6 +48,7 @@ constexpr int kBK = 64;              // K per stage: one 128-byte swizzle row of
 constexpr int kMaxStages = 6;       // stage = A tile 16 KB + B tile N x 128 B (N <= 256)
 constexpr int kMaxN = 256;           // MMA N per launch; TMEM holds two accumulators of N columns
 constexpr int kGroup = 128;          // tokens per group of the split-activation modes (1, 3)
+constexpr int kMaxCluster = 8;        // portable thread-block cluster size
 constexpr int kTicketCompact = kUnionTickets - 1;   // mode 1: CTAs done with their mask words
 constexpr int kTicketDepart = 1024;  // tickets[kTicketDepart + tile]: split CTAs done with a tile (a tile
                                      // with splits > 1 has index < the CTA count <= kMaxUnionCtas)
@@ -87,6 +88,9 @@ struct alignas(64) UParams {
     int32_t* ccount2;
     uint32_t* err;
     unsigned long long* trace;   // null, or this launch's [CTA][kUTraceMarks] time stamps
+    int cluster;          // > 1: the splits of a tile form one thread-block cluster of this size
+    int red_off, rpo;     //   and reduce through distributed shared memory: the reduction buffer's
+                          //   offset in shared memory, and tile rows owned per CTA of the cluster
 };
 
 // Work decomposition shared by all three roles (same answer in every thread).
@@ -120,6 +124,7 @@ __device__ __forceinline__ Plan make_plan(const UParams& p) {
         q.splits = max(1, min(s, q.kblocks));
     }
     if (q.kblocks > 0 && q.splits > q.kblocks) q.splits = q.kblocks;
+    if (p.cluster > 1) q.splits = p.cluster;   // one CTA per split (an empty K range adds zeros)
     return q;
 }
 
@@ -545,6 +550,24 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
                         else p.mask[word] = bits;
                     }
                 }
+            } else if (p.cluster > 1) {
+                // split-K in a cluster: this row goes to the reduction buffer of the CTA that owns
+                // it (rows rank * rpo ..), slot [sp][row - owner's first row]
+                const uint32_t owner = (uint32_t)(lane_row / p.rpo);
+                const uint32_t slot = s32(base + p.red_off) +
+                                      (uint32_t)(((sp * p.rpo + (lane_row - (int)owner * p.rpo)) * N) * 4);
+                const uint32_t dst = cluster_map(slot, owner);
+                for (int c0 = 0; c0 < N; c0 += 16) {
+                    float v[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = 0.f;
+                    if (has) {
+                        tmem_ld16(taddr + c0, v);
+                        tmem_wait_ld();
+                    }
+#pragma unroll
+                    for (int c = 0; c < 16; c += 4) cluster_st4(dst + (uint32_t)(c0 + c) * 4u, v[c], v[c + 1], v[c + 2], v[c + 3]);
+                }
             } else {
                 // split-K: publish this split's partial
                 float* mine = p.partial + ((size_t)u * kBM + lane_row) * N;
@@ -568,7 +591,7 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
                 if (++ab == 2) { ab = 0; aph ^= 1; }
                 if (et == 0) UTRACE(4);
             }
-            if (q.splits == 1) continue;
+            if (q.splits == 1 || p.cluster > 1) continue;
             // split-K: once every split of the tile has published its partial, the CTA of
             // split sp sums its share of the tile's rows (rows sp kBM / splits ..) over all
             // splits, in split order.  The tile's counter counts arrivals (all splits' CTAs are
@@ -648,6 +671,36 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
         if (et == 0) UTRACE(5);
     }
     __syncwarp();
+    if (p.cluster > 1) {
+        // every split of the tile has written its rows to their owners: reduce this CTA's
+        // rows over the splits in split order, all threads sharing (row, 4-column) items
+        cluster_sync_all();
+        const int S = p.cluster, rank = blockIdx.x % S, tile = blockIdx.x / S;
+        const bool pair = p.mode == 3;
+        const int half = pair ? p.Gt : N;
+        const int r0 = rank * p.rpo, nrows = max(0, min(kBM, r0 + p.rpo) - r0);
+        const int nc4 = half / 4;
+        const float* red = reinterpret_cast<const float*>(base + p.red_off);
+        if (blockIdx.x < q.tiles * S) {
+            for (int it = threadIdx.x; it < nrows * nc4; it += kUThreads) {
+                const int rr = it / nc4, c0 = (it % nc4) * 4;
+                float hi[4] = {0.f, 0.f, 0.f, 0.f}, lo[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int sp = 0; sp < S; ++sp) {
+                    const float* src = red + ((size_t)(sp * p.rpo + rr) * N + c0);
+                    const float4 a = *reinterpret_cast<const float4*>(src);
+                    hi[0] += a.x; hi[1] += a.y; hi[2] += a.z; hi[3] += a.w;
+                    if (pair) {
+                        const float4 b = *reinterpret_cast<const float4*>(src + half);
+                        lo[0] += b.x; lo[1] += b.y; lo[2] += b.z; lo[3] += b.w;
+                    }
+                }
+                float bias;
+                const int state = row_pre<T>(p, q, tile, r0 + rr, bias);
+                bool any = false;
+                finish_chunk<T>(p, tile, r0 + rr, c0, hi, lo, &any, 4, state, bias);
+            }
+        }
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -665,7 +718,9 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
 // stage ring and TMEM allocation for an MMA of N columns
 void size_launch(UParams& p) {
     p.stage_bytes = 16384 + p.N * 128;
-    p.stages = std::min(kMaxStages, (200 * 1024) / p.stage_bytes);
+    const int red_bytes = p.cluster > 1 ? p.cluster * p.rpo * p.N * 4 : 0;
+    p.stages = std::min(kMaxStages, (200 * 1024 - red_bytes - 1024) / p.stage_bytes);
+    p.red_off = p.stages * p.stage_bytes + 1024;
     int cols = 32;
     while (cols < 2 * p.N) cols *= 2;
     p.tmem_cols = cols;
@@ -691,7 +746,11 @@ cudaError_t launch(UParams& p, int grid, cudaStream_t st) {
     size_launch(p);
     p.trace = trace_slot(grid);
     if (p.N > kMaxN || p.stages < 2) return cudaErrorInvalidValue;
-    const size_t smem = (size_t)p.stages * p.stage_bytes + 1024 + 256;
+    // the kernel rounds the dynamic region's start up to 1024 bytes: with a reduction buffer,
+    // its end (red_off + red_bytes past that start) keeps a full 1024 bytes of slack
+    const size_t red_bytes = p.cluster > 1 ? (size_t)p.cluster * p.rpo * p.N * 4 : 0;
+    const size_t smem = red_bytes ? (size_t)p.red_off + red_bytes + 1024
+                                  : (size_t)p.stages * p.stage_bytes + 1024 + 256;
     auto kern = p.dtype == SPFFN_BF16 ? k_umma<__nv_bfloat16> : k_umma<__half>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -701,12 +760,31 @@ cudaError_t launch(UParams& p, int grid, cudaStream_t st) {
     cfg.blockDim = dim3(kUThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (p.cluster > 1) {
+        if (grid % p.cluster) return cudaErrorInvalidValue;
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = (unsigned)p.cluster;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
+    }
     return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+// Split-K through distributed shared memory: the S = splits of each of `tiles` tiles form
+// one cluster (S <= 8, the portable cluster size; N <= 64 keeps the reduction buffer small).
+// Returns the grid (tiles x S), or 0 when the global-memory split reduction is used.
+int use_cluster(UParams& p, int tiles, int splits) {
+    const int S = std::min(splits, kMaxCluster);
+    if (S < 2 || p.N > 64 || tiles * S > p.G) return 0;
+    p.cluster = S;
+    p.rpo = (kBM + S - 1) / S;
+    return tiles * S;
 }
 
 UParams base_params(const spffn_ctx& c, int B) {
@@ -756,12 +834,18 @@ cudaError_t union_predict(const spffn_ctx& c, const void* x, int B, int32_t* idx
     const int tiles = (g.H + kBM - 1) / kBM;
     const int kblocks = g.d / kBK;
     p.splits_fixed = std::max(1, std::min(kblocks, c.num_sms / tiles));
+    // splits of under 8 K blocks reduce through a cluster (their hand-off outweighs their
+    // streaming); longer ones keep all CTAs busy with the global reduction (measured: OPT-13B
+    // shape, 18 splits of ~4 blocks, 2.55 -> 2.39 ms per step at B = 16; OPT-66B shape, 9
+    // splits of 16 blocks, 6.35 -> 6.81 ms with a cluster of 8)
+    const int grid0 = kblocks < 8 * p.splits_fixed ? use_cluster(p, tiles, p.splits_fixed) : 0;
+    if (grid0) p.splits_fixed = p.cluster;
     p.bias = c.w.bp1;
     p.out_split = c.hsplit();
     p.out_f32 = c.h();
     if (!make_map(&p.tmA, c.w.Wp1, g.dtype, g.H, g.d, kBM)) return cudaErrorInvalidValue;
     if (!make_map(&p.tmB, x, g.dtype, B, g.d, p.N)) return cudaErrorInvalidValue;
-    cudaError_t e = launch(p, c.num_sms, st);
+    cudaError_t e = launch(p, grid0 ? grid0 : c.num_sms, st);
     if (e != cudaSuccess) return e;
     // predictor layer 2, one token group at a time: D[n x 2Gt] = Wp2 . hsplit_g^T -> union mask words
     for (int gi = 0; gi < ug.groups; ++gi) {
@@ -824,8 +908,10 @@ cudaError_t union_forward(const spffn_ctx& c, const void* x, int B, const int32_
         q.bias = c.w.b2;
         q.out_f32 = y;
         q.W = c.w.W2T;
+        const int tiles3 = (g.d + kBM - 1) / kBM;
+        const int grid3 = use_cluster(q, tiles3, c.num_sms / tiles3);
         if (!make_map(&q.tmB, c.asplit(), g.dtype, 2 * ug.groups * ug.Gt, g.n, q.N)) return cudaErrorInvalidValue;
-        e = launch(q, c.num_sms, st);
+        e = launch(q, grid3 ? grid3 : c.num_sms, st);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

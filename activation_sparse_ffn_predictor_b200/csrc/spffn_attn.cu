@@ -82,6 +82,7 @@ struct AParams {
 namespace {
 
 constexpr int kPos = 4;                                 // positions per k/v work unit
+constexpr int kRW = 2;                                  // weight rows per q/k/v work unit (dh % 8 == 0)
 
 template <typename T>
 __device__ __forceinline__ float dot8(const uint4& w, const uint4& x) {
@@ -166,13 +167,14 @@ __global__ void __launch_bounds__(kSelWarps * 32) k_attn_select(const AParams p)
         if (lane == 0) p.nmiss[s] = m;
     }
     __syncthreads();
-    // the q/k/v kernel's work units per head slot (dh q rows, then the k and v rows once per
-    // group of kPos positions: the new token and the missing ones) and their exclusive prefix
+    // the q/k/v kernel's work units per head slot (its q rows in pairs, then the k and v row
+    // pairs once per group of kPos positions: the new token and the missing ones) and their
+    // exclusive prefix
     if (warp == 0) {
         int run = 0;
         for (int s0 = 0; s0 < s_count; s0 += 32) {
             const int s = s0 + lane;
-            const int u = s < s_count ? p.dh * (1 + 2 * ((p.nmiss[s] + kPos) / kPos)) : 0;
+            const int u = s < s_count ? (p.dh / kRW) * (1 + 2 * ((p.nmiss[s] + kPos) / kPos)) : 0;
             int x = u;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -189,40 +191,55 @@ __global__ void __launch_bounds__(kSelWarps * 32) k_attn_select(const AParams p)
 // ---------------------------------------------------------------------------
 // 3: q, k, v rows of the selected heads for the new token; missing K/V rows from Y[p].
 // Work units, balanced over every warp of the grid (warp w takes the w-th of W equal
-// contiguous ranges): per head slot, its dh q rows (the new token), then for each k and
-// each v row one unit per group of kPos positions (the new token first, then the missing
-// positions in order).  Contiguous ranges keep a CTA's warps on one head, so the few
-// stored input rows Y[p] they all read stay in L1, and the units of one weight row run
-// back to back on one warp.  The new token was stored in Y by the select kernel.
+// contiguous ranges): per head slot, its q rows in pairs (the new token), then for each pair
+// of k rows and of v rows one unit per group of kPos positions (the new token first, then
+// the missing positions in order).  Contiguous ranges keep a CTA's warps on one head, so the
+// few stored input rows Y[p] they all read stay in L1, and the units of one weight-row pair
+// run back to back on one warp.  The new token was stored in Y by the select kernel.
 
-// NP dot products w . y_j over a d-length row, U rows of 16-byte loads in flight per lane;
 // each position accumulates lane-strided in ascending vector order, then a warp sum.
+// Dot products of two weight rows w0, w1 with NP input rows y_j over a d-length row: each
+// 16-byte input vector is loaded once for both weight rows (the input rows are the traffic
+// that repeats across a head's weight rows).  U vector columns per lane in flight; each sum
+// accumulates lane-strided in ascending vector order, then a warp sum.
 template <typename T, int NP, int U>
-__device__ __forceinline__ void rows_dot(const uint4* w, const uint4* const* y, int nv, int lane, float* z) {
-    float a[NP];
+__device__ __forceinline__ void rows_dot2(const uint4* w0, const uint4* w1, const uint4* const* y, int nv, int lane,
+                                          float* z0, float* z1) {
+    float a[NP], b[NP];
 #pragma unroll
-    for (int j = 0; j < NP; ++j) a[j] = 0.f;
+    for (int j = 0; j < NP; ++j) a[j] = b[j] = 0.f;
     int v = lane;
     for (; v + 32 * (U - 1) < nv; v += 32 * U) {
-        uint4 wv[U], yv[U][NP];
+        uint4 wa[U], wb[U], yv[U][NP];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            wv[u] = __ldg(w + v + 32 * u);
+            wa[u] = __ldg(w0 + v + 32 * u);
+            wb[u] = __ldg(w1 + v + 32 * u);
 #pragma unroll
             for (int j = 0; j < NP; ++j) yv[u][j] = __ldg(y[j] + v + 32 * u);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u)
 #pragma unroll
-            for (int j = 0; j < NP; ++j) a[j] += dot8<T>(wv[u], yv[u][j]);
+            for (int j = 0; j < NP; ++j) {
+                a[j] += dot8<T>(wa[u], yv[u][j]);
+                b[j] += dot8<T>(wb[u], yv[u][j]);
+            }
     }
     for (; v < nv; v += 32) {
-        const uint4 wv = __ldg(w + v);
+        const uint4 wa = __ldg(w0 + v), wb = __ldg(w1 + v);
 #pragma unroll
-        for (int j = 0; j < NP; ++j) a[j] += dot8<T>(wv, __ldg(y[j] + v));
+        for (int j = 0; j < NP; ++j) {
+            const uint4 yv = __ldg(y[j] + v);
+            a[j] += dot8<T>(wa, yv);
+            b[j] += dot8<T>(wb, yv);
+        }
     }
 #pragma unroll
-    for (int j = 0; j < NP; ++j) z[j] = warp_sum(a[j]);
+    for (int j = 0; j < NP; ++j) {
+        z0[j] = warp_sum(a[j]);
+        z1[j] = warp_sum(b[j]);
+    }
 }
 
 template <typename T>
@@ -234,7 +251,7 @@ __global__ void __launch_bounds__(256) k_attn_qkv(const AParams p)
     if (t >= p.tmax || count == 0) return;
     for (int s = threadIdx.x; s <= count; s += 256) up[s] = p.upref[s];
     __syncthreads();
-    const int nv = p.d / 8, dh = p.dh, total = up[count], W = gridDim.x * 8;
+    const int nv = p.d / 8, dh = p.dh, hp = dh / kRW, total = up[count], W = gridDim.x * 8;
     const T* Yh = reinterpret_cast<const T*>(p.Y);
     const uint4* yt = reinterpret_cast<const uint4*>(Yh + (size_t)t * p.d);
     const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -247,24 +264,31 @@ __global__ void __launch_bounds__(256) k_attn_qkv(const AParams p)
         }
         const int s = lo, h = p.heads[s];
         int w = u - up[s];
-        if (w < dh) {
-            const size_t row = (size_t)h * dh + w;
-            const uint4* wr = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.Wq) + row * p.d);
-            const float bias = p.bq ? DT<T>::f(reinterpret_cast<const T*>(p.bq)[row]) : 0.f;
-            float z;
-            rows_dot<T, 1, 4>(wr, &yt, nv, lane, &z);
-            if (lane == 0) p.q[(size_t)s * dh + w] = z + bias;
+        if (w < hp) {                                   // q rows 2w, 2w + 1 for the new token
+            const int i = kRW * w;
+            const size_t row = (size_t)h * dh + i;
+            const T* Wq = reinterpret_cast<const T*>(p.Wq);
+            float z0, z1;
+            rows_dot2<T, 1, 4>(reinterpret_cast<const uint4*>(Wq + row * p.d),
+                               reinterpret_cast<const uint4*>(Wq + (row + 1) * p.d), &yt, nv, lane, &z0, &z1);
+            if (lane == 0) {
+                const T* bq = reinterpret_cast<const T*>(p.bq);
+                p.q[(size_t)s * dh + i] = z0 + (bq ? DT<T>::f(bq[row]) : 0.f);
+                p.q[(size_t)s * dh + i + 1] = z1 + (bq ? DT<T>::f(bq[row + 1]) : 0.f);
+            }
             continue;
         }
-        w -= dh;
+        w -= hp;
         const int nm = p.nmiss[s], ng = (nm + kPos) / kPos;
-        const int type = w / (dh * ng);                 // 0: k row, 1: v row
-        const int rem = w - type * dh * ng, i = rem / ng, g = rem - i * ng;
+        const int type = w / (hp * ng);                 // 0: k rows, 1: v rows
+        const int rem = w - type * hp * ng, ip = rem / ng, g = rem - ip * ng;
+        const int i = kRW * ip;
         const size_t row = (size_t)h * dh + i;
         const T* Wr = reinterpret_cast<const T*>(type == 0 ? p.Wk : p.Wv);
         const T* br = reinterpret_cast<const T*>(type == 0 ? p.bk : p.bv);
-        const float bias = br ? DT<T>::f(br[row]) : 0.f;
-        const uint4* wr = reinterpret_cast<const uint4*>(Wr + row * p.d);
+        const float bias0 = br ? DT<T>::f(br[row]) : 0.f, bias1 = br ? DT<T>::f(br[row + 1]) : 0.f;
+        const uint4* wr0 = reinterpret_cast<const uint4*>(Wr + row * p.d);
+        const uint4* wr1 = reinterpret_cast<const uint4*>(Wr + (row + 1) * p.d);
         const uint16_t* ml = p.miss + (size_t)s * p.tmax;
         const int j0 = g * kPos, np = min(kPos, nm + 1 - j0);
         int pos[kPos];
@@ -275,18 +299,22 @@ __global__ void __launch_bounds__(256) k_attn_qkv(const AParams p)
             pos[j] = jj == 0 ? t : (int)ml[jj - 1];
             yr[j] = reinterpret_cast<const uint4*>(Yh + (size_t)pos[j] * p.d);
         }
-        float z[kPos];
+        float z0[kPos], z1[kPos];
         switch (np) {
-            case 1: rows_dot<T, 1, 4>(wr, yr, nv, lane, z); break;
-            case 2: rows_dot<T, 2, 2>(wr, yr, nv, lane, z); break;
-            case 3: rows_dot<T, 3, 2>(wr, yr, nv, lane, z); break;
-            default: rows_dot<T, 4, 2>(wr, yr, nv, lane, z); break;
+            case 1: rows_dot2<T, 1, 4>(wr0, wr1, yr, nv, lane, z0, z1); break;
+            case 2: rows_dot2<T, 2, 2>(wr0, wr1, yr, nv, lane, z0, z1); break;
+            case 3: rows_dot2<T, 3, 2>(wr0, wr1, yr, nv, lane, z0, z1); break;
+            default: rows_dot2<T, 4, 2>(wr0, wr1, yr, nv, lane, z0, z1); break;
         }
         if (lane == 0) {
             T* C = reinterpret_cast<T*>(type == 0 ? p.K : p.V);
 #pragma unroll
             for (int j = 0; j < kPos; ++j)
-                if (j < np) C[((size_t)h * p.tmax + pos[j]) * dh + i] = DT<T>::r(z[j] + bias);
+                if (j < np) {
+                    T* dst = C + ((size_t)h * p.tmax + pos[j]) * dh + i;
+                    dst[0] = DT<T>::r(z0[j] + bias0);
+                    dst[1] = DT<T>::r(z1[j] + bias1);
+                }
         }
     }
 }

@@ -82,7 +82,7 @@ struct AParams {
 namespace {
 
 constexpr int kPos = 4;                                 // positions per k/v work unit
-constexpr int kRW = 2;                                  // weight rows per q/k/v work unit (dh % 8 == 0)
+constexpr int kRW = 4;                                  // weight rows per q/k/v work unit (dh % 8 == 0)
 
 template <typename T>
 __device__ __forceinline__ float dot8(const uint4& w, const uint4& x) {
@@ -202,44 +202,45 @@ __global__ void __launch_bounds__(kSelWarps * 32) k_attn_select(const AParams p)
 // 16-byte input vector is loaded once for both weight rows (the input rows are the traffic
 // that repeats across a head's weight rows).  U vector columns per lane in flight; each sum
 // accumulates lane-strided in ascending vector order, then a warp sum.
-template <typename T, int NP, int U>
-__device__ __forceinline__ void rows_dot2(const uint4* w0, const uint4* w1, const uint4* const* y, int nv, int lane,
-                                          float* z0, float* z1) {
-    float a[NP], b[NP];
+template <typename T, int R, int NP, int U>
+__device__ __forceinline__ void rows_dotR(const uint4* const* w, const uint4* const* y, int nv, int lane, float (*z)[kPos]) {
+    float a[R][NP];
 #pragma unroll
-    for (int j = 0; j < NP; ++j) a[j] = b[j] = 0.f;
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int j = 0; j < NP; ++j) a[r][j] = 0.f;
     int v = lane;
     for (; v + 32 * (U - 1) < nv; v += 32 * U) {
-        uint4 wa[U], wb[U], yv[U][NP];
+        uint4 wv[U][R], yv[U][NP];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            wa[u] = __ldg(w0 + v + 32 * u);
-            wb[u] = __ldg(w1 + v + 32 * u);
+#pragma unroll
+            for (int r = 0; r < R; ++r) wv[u][r] = __ldg(w[r] + v + 32 * u);
 #pragma unroll
             for (int j = 0; j < NP; ++j) yv[u][j] = __ldg(y[j] + v + 32 * u);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u)
 #pragma unroll
-            for (int j = 0; j < NP; ++j) {
-                a[j] += dot8<T>(wa[u], yv[u][j]);
-                b[j] += dot8<T>(wb[u], yv[u][j]);
-            }
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int j = 0; j < NP; ++j) a[r][j] += dot8<T>(wv[u][r], yv[u][j]);
     }
     for (; v < nv; v += 32) {
-        const uint4 wa = __ldg(w0 + v), wb = __ldg(w1 + v);
+        uint4 wv[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) wv[r] = __ldg(w[r] + v);
 #pragma unroll
         for (int j = 0; j < NP; ++j) {
             const uint4 yv = __ldg(y[j] + v);
-            a[j] += dot8<T>(wa, yv);
-            b[j] += dot8<T>(wb, yv);
+#pragma unroll
+            for (int r = 0; r < R; ++r) a[r][j] += dot8<T>(wv[r], yv);
         }
     }
 #pragma unroll
-    for (int j = 0; j < NP; ++j) {
-        z0[j] = warp_sum(a[j]);
-        z1[j] = warp_sum(b[j]);
-    }
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int j = 0; j < NP; ++j) z[r][j] = warp_sum(a[r][j]);
 }
 
 template <typename T>
@@ -268,13 +269,15 @@ __global__ void __launch_bounds__(256) k_attn_qkv(const AParams p)
             const int i = kRW * w;
             const size_t row = (size_t)h * dh + i;
             const T* Wq = reinterpret_cast<const T*>(p.Wq);
-            float z0, z1;
-            rows_dot2<T, 1, 4>(reinterpret_cast<const uint4*>(Wq + row * p.d),
-                               reinterpret_cast<const uint4*>(Wq + (row + 1) * p.d), &yt, nv, lane, &z0, &z1);
+            const uint4* wr[kRW];
+#pragma unroll
+            for (int r = 0; r < kRW; ++r) wr[r] = reinterpret_cast<const uint4*>(Wq + (row + r) * p.d);
+            float z[kRW][kPos];
+            rows_dotR<T, kRW, 1, 2>(wr, &yt, nv, lane, z);
             if (lane == 0) {
                 const T* bq = reinterpret_cast<const T*>(p.bq);
-                p.q[(size_t)s * dh + i] = z0 + (bq ? DT<T>::f(bq[row]) : 0.f);
-                p.q[(size_t)s * dh + i + 1] = z1 + (bq ? DT<T>::f(bq[row + 1]) : 0.f);
+#pragma unroll
+                for (int r = 0; r < kRW; ++r) p.q[(size_t)s * dh + i + r] = z[r][0] + (bq ? DT<T>::f(bq[row + r]) : 0.f);
             }
             continue;
         }
@@ -286,9 +289,9 @@ __global__ void __launch_bounds__(256) k_attn_qkv(const AParams p)
         const size_t row = (size_t)h * dh + i;
         const T* Wr = reinterpret_cast<const T*>(type == 0 ? p.Wk : p.Wv);
         const T* br = reinterpret_cast<const T*>(type == 0 ? p.bk : p.bv);
-        const float bias0 = br ? DT<T>::f(br[row]) : 0.f, bias1 = br ? DT<T>::f(br[row + 1]) : 0.f;
-        const uint4* wr0 = reinterpret_cast<const uint4*>(Wr + row * p.d);
-        const uint4* wr1 = reinterpret_cast<const uint4*>(Wr + (row + 1) * p.d);
+        const uint4* wr[kRW];
+#pragma unroll
+        for (int r = 0; r < kRW; ++r) wr[r] = reinterpret_cast<const uint4*>(Wr + (row + r) * p.d);
         const uint16_t* ml = p.miss + (size_t)s * p.tmax;
         const int j0 = g * kPos, np = min(kPos, nm + 1 - j0);
         int pos[kPos];
@@ -299,12 +302,12 @@ __global__ void __launch_bounds__(256) k_attn_qkv(const AParams p)
             pos[j] = jj == 0 ? t : (int)ml[jj - 1];
             yr[j] = reinterpret_cast<const uint4*>(Yh + (size_t)pos[j] * p.d);
         }
-        float z0[kPos], z1[kPos];
+        float z[kRW][kPos];
         switch (np) {
-            case 1: rows_dot2<T, 1, 4>(wr0, wr1, yr, nv, lane, z0, z1); break;
-            case 2: rows_dot2<T, 2, 2>(wr0, wr1, yr, nv, lane, z0, z1); break;
-            case 3: rows_dot2<T, 3, 2>(wr0, wr1, yr, nv, lane, z0, z1); break;
-            default: rows_dot2<T, 4, 2>(wr0, wr1, yr, nv, lane, z0, z1); break;
+            case 1: rows_dotR<T, kRW, 1, 2>(wr, yr, nv, lane, z); break;
+            case 2: rows_dotR<T, kRW, 2, 1>(wr, yr, nv, lane, z); break;
+            case 3: rows_dotR<T, kRW, 3, 1>(wr, yr, nv, lane, z); break;
+            default: rows_dotR<T, kRW, 4, 1>(wr, yr, nv, lane, z); break;
         }
         if (lane == 0) {
             T* C = reinterpret_cast<T*>(type == 0 ? p.K : p.V);
@@ -312,8 +315,8 @@ __global__ void __launch_bounds__(256) k_attn_qkv(const AParams p)
             for (int j = 0; j < kPos; ++j)
                 if (j < np) {
                     T* dst = C + ((size_t)h * p.tmax + pos[j]) * dh + i;
-                    dst[0] = DT<T>::r(z0[j] + bias0);
-                    dst[1] = DT<T>::r(z1[j] + bias1);
+#pragma unroll
+                    for (int r = 0; r < kRW; ++r) dst[r] = DT<T>::r(z[r][j] + (br ? DT<T>::f(br[row + r]) : 0.f));
                 }
         }
     }

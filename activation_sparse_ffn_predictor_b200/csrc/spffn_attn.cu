@@ -6,9 +6,9 @@
 //
 // One step of one layer, one token, five launches on the caller's stream:
 //   1 SP_A hidden layer h = ReLU(Wa1 y + ba1)                 (the predictor GEMV kernel)
-//   2 head logits, threshold, ascending head list; y stored as Y[t]; for every
-//     selected head the list of positions p < t whose K/V rows are missing, and
-//     the q/k/v kernel's work units per head
+//   2 one CTA per head: its logit and decision, and for a selected head the list
+//     of positions p < t whose K/V rows are missing; y stored as Y[t]; the CTA
+//     finishing last writes the ascending head list and the q/k/v work units
 //   3 q, k, v rows of the selected heads for the new token, and the missing K/V
 //     rows from Y[p], in work units balanced over every resident warp
 //   4 attention per selected head over positions 0..t, split over CTAs with an
@@ -29,7 +29,7 @@
 namespace spffn {
 
 struct ALayout {
-    size_t ctl, h, q, miss, nmiss, upref, opart, o, tickets, K, V, filled, Y, total;
+    size_t ctl, h, q, miss, nmiss, hsel, upref, opart, o, tickets, K, V, filled, Y, total;
     int S, Sa;
 };
 
@@ -39,11 +39,12 @@ inline ALayout attn_layout(const spffn_attn_config& c, int S) {
     auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
     L.S = S;
     L.Sa = 8;                                                   // position splits per head
-    L.ctl = take(256);                                          // [0] error word, [1] t
+    L.ctl = take(256);                                          // [0] error word, [1] t, [2] select ticket
     L.h = take((size_t)c.Ha * sizeof(float));
     L.q = take((size_t)c.nh * c.dh * sizeof(float));
-    L.miss = take((size_t)c.nh * c.tmax * sizeof(uint16_t));    // per head slot: missing positions
+    L.miss = take((size_t)c.nh * c.tmax * sizeof(uint16_t));    // per head: missing positions
     L.nmiss = take((size_t)c.nh * sizeof(int32_t));
+    L.hsel = take((size_t)c.nh * sizeof(int32_t));             // per head: selected this step
     L.upref = take((size_t)(c.nh + 1) * sizeof(int32_t));     // work units before each head slot
     L.opart = take((size_t)c.nh * L.Sa * (c.dh + 2) * sizeof(float));
     L.o = take((size_t)c.nh * c.dh * sizeof(float));
@@ -68,6 +69,8 @@ struct AParams {
     float* q;
     uint16_t* miss;
     int32_t* nmiss;
+    int32_t* hsel;
+    uint32_t* sticket;
     int32_t* upref;
     float* opart;
     float* o;
@@ -96,95 +99,94 @@ __device__ __forceinline__ float dot8(const uint4& w, const uint4& x) {
 }
 
 // ---------------------------------------------------------------------------
-// 2: head logits l_k = Wa2[k] . h + ba2_k, selection l_k > 0, ascending list; Y[t] = y;
-// per selected head the positions p < t with no K/V row yet.  One CTA of 32 warps (a
-// few heads per warp, each row's loads issued together: this kernel is latency-bound).
-constexpr int kSelWarps = 32;
+// 2: head logits l_k = Wa2[k] . h + ba2_k, selection l_k > 0; Y[t] = y.  One CTA per head:
+// its logit and decision, and for a selected head the positions p < t with no K/V row yet
+// (ascending, by head).  The CTA that finishes last writes the ascending head list, its
+// length and the q/k/v kernel's work-unit prefix (atomic ticket, reset for the next step).
+constexpr int kSelThreads = 128;
 
 template <typename T>
-__global__ void __launch_bounds__(kSelWarps * 32) k_attn_select(const AParams p)
+__global__ void __launch_bounds__(kSelThreads) k_attn_select(const AParams p)
 {
-    __shared__ unsigned char sel[1024];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ float red[kSelThreads / 32];
+    __shared__ int wcnt[kSelThreads / 32];
+    __shared__ int s_last;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, k = blockIdx.x;
     const int t = *p.tcur;
     const bool full = t >= p.tmax;
-    if (!full) {
+    if (k == 0 && !full) {
         const uint4* src = reinterpret_cast<const uint4*>(p.y);
         uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.Y) + (size_t)t * p.d);
-        for (int v = tid; v < p.d / 8; v += kSelWarps * 32) dst[v] = src[v];
+        for (int v = tid; v < p.d / 8; v += kSelThreads) dst[v] = src[v];
     }
     const int hv = p.Ha / 8;
-    for (int k = warp; k < p.nh; k += kSelWarps) {
-        const uint4* w = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.Wa2) + (size_t)k * p.Ha);
-        float acc = 0.f;
-        auto fold = [&](const uint4& wv, int v) {
-            float wf[8];
-            unpack8<T>(wv, wf);
-            const float4 a = reinterpret_cast<const float4*>(p.h)[2 * v], b = reinterpret_cast<const float4*>(p.h)[2 * v + 1];
-            acc = fmaf(wf[0], a.x, acc); acc = fmaf(wf[1], a.y, acc); acc = fmaf(wf[2], a.z, acc); acc = fmaf(wf[3], a.w, acc);
-            acc = fmaf(wf[4], b.x, acc); acc = fmaf(wf[5], b.y, acc); acc = fmaf(wf[6], b.z, acc); acc = fmaf(wf[7], b.w, acc);
-        };
-        int v = lane;
-        for (; v + 96 < hv; v += 128) {
-            const uint4 w0 = ldg_stream(w + v), w1 = ldg_stream(w + v + 32);
-            const uint4 w2 = ldg_stream(w + v + 64), w3 = ldg_stream(w + v + 96);
-            fold(w0, v); fold(w1, v + 32); fold(w2, v + 64); fold(w3, v + 96);
-        }
-        for (; v < hv; v += 32) fold(ldg_stream(w + v), v);
-        acc = warp_sum(acc);
-        const float bias = p.ba2 ? DT<T>::f(reinterpret_cast<const T*>(p.ba2)[k]) : 0.f;
-        if (lane == 0) sel[k] = !full && (acc + bias) > 0.f;
+    const uint4* w = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.Wa2) + (size_t)k * p.Ha);
+    float acc = 0.f;
+    for (int v = tid; v < hv; v += kSelThreads) {
+        float wf[8];
+        unpack8<T>(ldg_stream(w + v), wf);
+        const float4 a = reinterpret_cast<const float4*>(p.h)[2 * v], b = reinterpret_cast<const float4*>(p.h)[2 * v + 1];
+        acc = fmaf(wf[0], a.x, acc); acc = fmaf(wf[1], a.y, acc); acc = fmaf(wf[2], a.z, acc); acc = fmaf(wf[3], a.w, acc);
+        acc = fmaf(wf[4], b.x, acc); acc = fmaf(wf[5], b.y, acc); acc = fmaf(wf[6], b.z, acc); acc = fmaf(wf[7], b.w, acc);
     }
+    acc = warp_sum(acc);
+    if (lane == 0) red[warp] = acc;
     __syncthreads();
-    __shared__ int s_count;
-    if (warp == 0) {
+    const float bias = p.ba2 ? DT<T>::f(reinterpret_cast<const T*>(p.ba2)[k]) : 0.f;
+    const bool on = !full && ((red[0] + red[1]) + (red[2] + red[3])) + bias > 0.f;
+    if (on) {
+        // missing K/V rows of this head, ascending: an ordered block-wide compaction
+        const uint8_t* f = p.filled + (size_t)k * p.tmax;
+        uint16_t* ml = p.miss + (size_t)k * p.tmax;
         int m = 0;
-        for (int k0 = 0; k0 < p.nh; k0 += 32) {
-            const bool on = k0 + lane < p.nh && sel[k0 + lane];
-            const uint32_t bal = __ballot_sync(0xffffffffu, on);
-            if (on) p.heads[m + __popc(bal & ((1u << lane) - 1u))] = k0 + lane;
-            m += __popc(bal);
+        for (int p0 = 0; p0 < t; p0 += kSelThreads) {
+            const bool miss = p0 + tid < t && !f[p0 + tid];
+            const uint32_t bal = __ballot_sync(0xffffffffu, miss);
+            if (lane == 0) wcnt[warp] = __popc(bal);
+            __syncthreads();
+            int base = m;
+            for (int q = 0; q < warp; ++q) base += wcnt[q];
+            if (miss) ml[base + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)(p0 + tid);
+            m += (wcnt[0] + wcnt[1]) + (wcnt[2] + wcnt[3]);
+            __syncthreads();
         }
-        if (lane == 0) {
-            *p.count = m;
-            s_count = m;
-            if (full) latch(p.err, ERR_CACHE_FULL);
-        }
+        if (tid == 0) p.nmiss[k] = m;
     }
+    if (tid == 0) p.hsel[k] = on ? 1 : 0;
+    __threadfence();
     __syncthreads();
-    // missing K/V rows of each selected head (one warp per head, ascending positions)
-    for (int s = warp; s < s_count; s += kSelWarps) {
-        const int h = p.heads[s];
-        const uint8_t* f = p.filled + (size_t)h * p.tmax;
-        uint16_t* ml = p.miss + (size_t)s * p.tmax;
-        int m = 0;
-        for (int p0 = 0; p0 < t; p0 += 32) {
-            const bool on = p0 + lane < t && !f[p0 + lane];
-            const uint32_t bal = __ballot_sync(0xffffffffu, on);
-            if (on) ml[m + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)(p0 + lane);
-            m += __popc(bal);
-        }
-        if (lane == 0) p.nmiss[s] = m;
-    }
+    if (tid == 0) s_last = atomicAdd(p.sticket, 1u) == (uint32_t)(gridDim.x - 1);
     __syncthreads();
-    // the q/k/v kernel's work units per head slot (its q rows in pairs, then the k and v row
-    // pairs once per group of kPos positions: the new token and the missing ones) and their
-    // exclusive prefix
-    if (warp == 0) {
-        int run = 0;
-        for (int s0 = 0; s0 < s_count; s0 += 32) {
-            const int s = s0 + lane;
-            const int u = s < s_count ? (p.dh / kRW) * (1 + 2 * ((p.nmiss[s] + kPos) / kPos)) : 0;
-            int x = u;
+    if (!s_last || warp != 0) return;
+    __threadfence();
+    // ascending head list and the q/k/v work units per head slot (its q rows in groups of kRW,
+    // then the k and v row groups once per group of kPos positions: the new token and the
+    // missing ones), with their exclusive prefix
+    int m = 0, run = 0;
+    for (int k0 = 0; k0 < p.nh; k0 += 32) {
+        const int kk = k0 + lane;
+        const bool o = kk < p.nh && __ldcg(p.hsel + kk) != 0;
+        const uint32_t bal = __ballot_sync(0xffffffffu, o);
+        const int u = o ? (p.dh / kRW) * (1 + 2 * ((__ldcg(p.nmiss + kk) + kPos) / kPos)) : 0;
+        int x = u;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, x, o);
-                if (lane >= o) x += y;
-            }
-            if (s < s_count) p.upref[s] = run + x - u;
-            run += __shfl_sync(0xffffffffu, x, 31);
+        for (int q = 1; q < 32; q <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, q);
+            if (lane >= q) x += y;
         }
-        if (lane == 0) p.upref[s_count] = run;
+        if (o) {
+            const int slot = m + __popc(bal & ((1u << lane) - 1u));
+            p.heads[slot] = kk;
+            p.upref[slot] = run + x - u;
+        }
+        run += __shfl_sync(0xffffffffu, x, 31);
+        m += __popc(bal);
+    }
+    if (lane == 0) {
+        *p.count = m;
+        p.upref[m] = run;
+        *p.sticket = 0u;                                // ready for the next step
+        if (full) latch(p.err, ERR_CACHE_FULL);
     }
 }
 
@@ -282,7 +284,7 @@ __global__ void __launch_bounds__(256) k_attn_qkv(const AParams p)
             continue;
         }
         w -= hp;
-        const int nm = p.nmiss[s], ng = (nm + kPos) / kPos;
+        const int nm = p.nmiss[h], ng = (nm + kPos) / kPos;
         const int type = w / (hp * ng);                 // 0: k rows, 1: v rows
         const int rem = w - type * hp * ng, ip = rem / ng, g = rem - ip * ng;
         const int i = kRW * ip;
@@ -292,7 +294,7 @@ __global__ void __launch_bounds__(256) k_attn_qkv(const AParams p)
         const uint4* wr[kRW];
 #pragma unroll
         for (int r = 0; r < kRW; ++r) wr[r] = reinterpret_cast<const uint4*>(Wr + (row + r) * p.d);
-        const uint16_t* ml = p.miss + (size_t)s * p.tmax;
+        const uint16_t* ml = p.miss + (size_t)h * p.tmax;
         const int j0 = g * kPos, np = min(kPos, nm + 1 - j0);
         int pos[kPos];
         const uint4* yr[kPos];
@@ -582,6 +584,8 @@ AParams attn_params(const spffn_attn_ctx& c, const void* y, int32_t* heads, int3
     p.q = reinterpret_cast<float*>(c.ws + c.lay.q);
     p.miss = reinterpret_cast<uint16_t*>(c.ws + c.lay.miss);
     p.nmiss = reinterpret_cast<int32_t*>(c.ws + c.lay.nmiss);
+    p.hsel = reinterpret_cast<int32_t*>(c.ws + c.lay.hsel);
+    p.sticket = ctl + 2;
     p.upref = reinterpret_cast<int32_t*>(c.ws + c.lay.upref);
     p.opart = reinterpret_cast<float*>(c.ws + c.lay.opart);
     p.o = reinterpret_cast<float*>(c.ws + c.lay.o);
@@ -600,7 +604,7 @@ cudaError_t step_impl(const spffn_attn_ctx& c, const AParams& p, cudaStream_t st
     cudaError_t e = launch_hidden(c.cfg.dtype, c.w.Wa1, c.w.ba1, p.y, 1, c.cfg.d, c.cfg.Ha,
                                   reinterpret_cast<float*>(c.ws + c.lay.h), G, st);
     if (e != cudaSuccess) return e;
-    k_attn_select<T><<<1, kSelWarps * 32, 0, st>>>(p);
+    k_attn_select<T><<<c.cfg.nh, kSelThreads, 0, st>>>(p);
     k_attn_qkv<T><<<c.qkv_blocks, 256, 0, st>>>(p);   // every resident warp takes units
     k_attn_core<T><<<G, 256, 0, st>>>(p);
     k_attn_out<T><<<(c.cfg.d / 8 + kOutVec - 1) / kOutVec, kOutVec * kOutLanes, 0, st>>>(p);

@@ -419,12 +419,44 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
     if (warp == kConsumerWarps + 1) {
         if (lane == 0) {
             const uint64_t pol_last = policy_evict_last(), pol_first = policy_evict_first();
+            // W1[j], W2T[j] and b1[j]'s 16-byte block into FFN slot s
+            auto gather = [&](int s, int j, const char* w1, const char* w2, const char* bb0) {
+                char* dst = S.fring + (size_t)s * fslot_bytes;
+                mbar_expect_tx(&S.ffull[s], (uint32_t)(4 * d + 16));
+                if (p.hot_rows > 0) {
+                    // hot rows ([PI1] §5.2: the most frequently active neurons) stay in L2
+                    const uint64_t pol = range_offset(j, n, G) < p.hot_rows ? pol_last : pol_first;
+                    bulk_g2s_hint(dst, w1 + (size_t)j * 2 * d, (uint32_t)(2 * d), &S.ffull[s], pol);
+                    bulk_g2s_hint(dst + 2 * d, w2 + (size_t)j * 2 * d, (uint32_t)(2 * d), &S.ffull[s], pol);
+                } else {
+                    bulk_g2s(dst, w1 + (size_t)j * 2 * d, (uint32_t)(2 * d), &S.ffull[s]);
+                    bulk_g2s(dst + 2 * d, w2 + (size_t)j * 2 * d, (uint32_t)(2 * d), &S.ffull[s]);
+                }
+                bulk_g2s(dst + 4 * d, bb0 + (size_t)(j & ~7) * 2, 16u, &S.ffull[s]);
+            };
             int k = 0;
             bool stop = false;
             for (int l = 0; l < p.L && !stop; ++l) {
                 const char* w1 = reinterpret_cast<const char*>(p.layer[l].W1);
                 const char* w2 = reinterpret_cast<const char*>(p.layer[l].W2T);
                 const char* bb0 = reinterpret_cast<const char*>(p.layer[l].b1);
+                if constexpr (TAB) {
+                    // caller tables are known at launch: this CTA's slice of every layer's table,
+                    // filtered exactly as the consumers filter it, streams ahead across layers as
+                    // far as the FFN ring allows
+                    int U = __ldcg(p.layer[l].tab_count);
+                    U = U < 0 ? 0 : (U > n ? n : U);
+                    const int lo = split_lo(U, G, c), hi = split_lo(U, G, c + 1);
+                    for (int i = lo; i < hi && !stop; ++i) {
+                        const int j = __ldcg(p.layer[l].tab + i);
+                        if (j < 0 || j >= n) continue;
+                        const int s = k % p.ffn_slots;
+                        if (!wait_bounded(S, p, &S.fempty[s], ((k / p.ffn_slots) & 1) ^ 1, true)) { stop = true; break; }
+                        gather(s, j, w1, w2, bb0);
+                        S.flags[3] = ++k;
+                    }
+                    continue;
+                }
                 int issued = 0;
                 unsigned long long t0 = gtime();
                 while (true) {
@@ -434,19 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
                         __threadfence_block();
                         const int s = k % p.ffn_slots;
                         if (!wait_bounded(S, p, &S.fempty[s], ((k / p.ffn_slots) & 1) ^ 1, true)) { stop = true; break; }
-                        const int j = S.nl[(l & 1) * p.max_rows + issued];
-                        char* dst = S.fring + (size_t)s * fslot_bytes;
-                        mbar_expect_tx(&S.ffull[s], (uint32_t)(4 * d + 16));
-                        if (p.hot_rows > 0) {
-                            // hot rows ([PI1] §5.2: the most frequently active neurons) stay in L2
-                            const uint64_t pol = range_offset(j, n, G) < p.hot_rows ? pol_last : pol_first;
-                            bulk_g2s_hint(dst, w1 + (size_t)j * 2 * d, (uint32_t)(2 * d), &S.ffull[s], pol);
-                            bulk_g2s_hint(dst + 2 * d, w2 + (size_t)j * 2 * d, (uint32_t)(2 * d), &S.ffull[s], pol);
-                        } else {
-                            bulk_g2s(dst, w1 + (size_t)j * 2 * d, (uint32_t)(2 * d), &S.ffull[s]);
-                            bulk_g2s(dst + 2 * d, w2 + (size_t)j * 2 * d, (uint32_t)(2 * d), &S.ffull[s]);
-                        }
-                        bulk_g2s(dst + 4 * d, bb0 + (size_t)(j & ~7) * 2, 16u, &S.ffull[s]);
+                        gather(s, S.nl[(l & 1) * p.max_rows + issued], w1, w2, bb0);
                         S.flags[3] = ++k;
                         ++issued;
                         t0 = gtime();

@@ -726,12 +726,19 @@ void size_launch(UParams& p) {
     p.tmem_cols = cols;
 }
 
-// Trace slots: launch i since the trace buffer was bound writes slot i mod (slots held)
+// Trace slots: launch i since the trace buffer was bound writes slot i mod (slots held).
+// Every slot is as wide as the SM count, whatever the launch's own grid, so that launches of
+// different grids (clustered or not) never overlap.
 unsigned g_utrace_seq = 0;
 const void* g_utrace_buf = nullptr;
 
 unsigned long long* trace_slot(int grid) {
-    const size_t per = (size_t)grid * kUTraceMarks * sizeof(unsigned long long);
+    if (!trace_bytes()) return nullptr;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return nullptr;
+    const size_t per = (size_t)std::max(grid, sms) * kUTraceMarks * sizeof(unsigned long long);
     void* buf = trace_buffer(per);
     if (!buf) return nullptr;
     if (buf != g_utrace_buf) {
@@ -739,7 +746,7 @@ unsigned long long* trace_slot(int grid) {
         g_utrace_seq = 0;
     }
     const size_t slots = trace_bytes() / per;
-    return static_cast<unsigned long long*>(buf) + (size_t)(g_utrace_seq++ % slots) * grid * kUTraceMarks;
+    return static_cast<unsigned long long*>(buf) + (size_t)(g_utrace_seq++ % slots) * (per / sizeof(unsigned long long));
 }
 
 cudaError_t launch(UParams& p, int grid, cudaStream_t st) {

@@ -50,8 +50,11 @@ constexpr int kMaxN = 256;           // MMA N per launch; TMEM holds two accumul
 constexpr int kGroup = 128;          // tokens per group of the split-activation modes (1, 3)
 constexpr int kMaxCluster = 8;        // portable thread-block cluster size
 constexpr int kTicketCompact = kUnionTickets - 1;   // mode 1: CTAs done with their mask words
-constexpr int kTicketDepart = 1024;  // tickets[kTicketDepart + tile]: split CTAs done with a tile (a tile
-                                     // with splits > 1 has index < the CTA count <= kMaxUnionCtas)
+// Split-K hand-off through global memory, per tile (a tile with splits > 1 has index < the
+// CTA count <= kMaxUnionCtas): tickets[kTicketArrive + tile] counts split arrivals and never
+// resets; tickets[kTicketBase + tile] holds its value before the current call's arrivals.
+constexpr int kTicketArrive = 1024;
+constexpr int kTicketBase = 1536;
 constexpr unsigned long long kUDrainNs = 20000000ull;   // per stage, abort path only
 // Time stamps of one launch (tracing aid, per CTA): 0 set up, 1 TMA lane past the wait for
 // the previous kernel, 2 first stage consumed by the MMA, 3 last MMA issued, 4 last
@@ -513,6 +516,8 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
             const int items = nrows * (half / 4);
             float pre_b[kPre];
             int pre_s[kPre];
+            const bool gsplit = q.splits > 1 && p.cluster <= 1;
+            const uint32_t gbase = gsplit && et == 0 ? __ldcg(&p.tickets[kTicketBase + tile]) : 0u;
             if (q.splits == 1) {
                 pre_s[0] = row_pre<T>(p, q, tile, lane_row, pre_b[0]);
             } else {
@@ -594,28 +599,30 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
             if (q.splits == 1 || p.cluster > 1) continue;
             // split-K: once every split of the tile has published its partial, the CTA of
             // split sp sums its share of the tile's rows (rows sp kBM / splits ..) over all
-            // splits, in split order.  The tile's counter counts arrivals (all splits' CTAs are
-            // resident, one unit per CTA, so the wait is for work already running; it is
-            // bounded all the same); a second counter counts departures, and the last CTA to
-            // leave resets both for the next call.
-            __threadfence();
+            // splits, in split order.  The epilogue threads' partial stores are ordered by the
+            // barrier before one release add to the tile's arrival count; the count reaching
+            // base + splits (an acquire, then the barrier) makes every split's partial visible.
+            // All splits' CTAs are resident, one unit per CTA, so the wait is for work already
+            // running; it is bounded all the same.  Split 0 then records the new base for the
+            // next call, after every split has read the old one.
             epi_sync();
             if (et == 0) {
-                atomicAdd(&p.tickets[tile], 1u);
+                const uint32_t target = gbase + (uint32_t)q.splits;
+                red_release_add_u32(&p.tickets[kTicketArrive + tile], 1u);
                 const unsigned long long t0 = now_ns();
                 bool okr = true;
-                while (ld_acquire_u32(&p.tickets[tile]) < (uint32_t)q.splits) {
+                while ((int32_t)(ld_acquire_u32(&p.tickets[kTicketArrive + tile]) - target) < 0) {
                     if (now_ns() - t0 > kUWaitNs) {
                         atomicOr(p.err, ERR_PIPE_TIMEOUT);
                         okr = false;
                         break;
                     }
                 }
+                if (sp == 0) __stcg(&p.tickets[kTicketBase + tile], target);
                 *s_go = okr;
             }
             epi_sync();
             if (*s_go) {
-                __threadfence();
                 const size_t sstride = (size_t)kBM * N;
                 auto add4 = [](float* a, const float4& w) { a[0] += w.x; a[1] += w.y; a[2] += w.z; a[3] += w.w; };
                 // thread item it: row it / (half / 4) of the share, columns 4 (it % (half / 4)) ..
@@ -654,11 +661,6 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
                     const int state = row_pre<T>(p, q, tile, r0 + it / (half / 4), bias);
                     reduce_item(it, state, bias);
                 }
-            }
-            epi_sync();
-            if (et == 0 && atomicAdd(&p.tickets[kTicketDepart + tile], 1u) == (uint32_t)(q.splits - 1)) {
-                p.tickets[tile] = 0u;
-                p.tickets[kTicketDepart + tile] = 0u;
             }
         }
         if (p.mode == 1 && p.cidx) {

@@ -27,6 +27,13 @@ static __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
 static __device__ __forceinline__ void red_release_add_u32(uint32_t* p, uint32_t v) {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+// fetch-add with acquire and release semantics at gpu scope: publishes this thread's prior
+// writes (and those ordered before it by a barrier) and observes those published before it
+static __device__ __forceinline__ uint32_t atom_acq_rel_add_u32(uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
 static __device__ __forceinline__ void ub_init(uint64_t* b, uint32_t c) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(s32(b)), "r"(c) : "memory");
 }

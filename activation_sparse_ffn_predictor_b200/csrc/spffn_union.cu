@@ -665,10 +665,11 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
         }
         if (p.mode == 1 && p.cidx) {
             // the CTA whose mask words land last compacts the union mask into the ascending
-            // neuron table, with all its threads, after the final barrier (no separate launch)
-            __threadfence();
+            // neuron table, with all its threads, after the final barrier (no separate launch).
+            // The barrier orders this CTA's mask words before one acquire-release count: the
+            // last CTA to count sees every CTA's words.
             epi_sync();
-            if (et == 0) *s_go = atomicAdd(&p.tickets[kTicketCompact], 1u) == gridDim.x - 1;
+            if (et == 0) *s_go = atom_acq_rel_add_u32(&p.tickets[kTicketCompact], 1u) == gridDim.x - 1;
         }
         if (et == 0) UTRACE(5);
     }
@@ -710,7 +711,6 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(p.tmem_cols));
     }
     if (p.mode == 1 && p.cidx && *s_go) {                 // uniform over the CTA
-        __threadfence();
         compact_mask_cta(p.mask, p.n >> 5, p.cidx, p.ccount, p.ccount2, s_wsum);
         if (threadIdx.x == 0) p.tickets[kTicketCompact] = 0u;     // ready for the next call
     }

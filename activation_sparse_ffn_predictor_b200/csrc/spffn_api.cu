@@ -172,8 +172,11 @@ spffn_status decode_impl(spffn_ctx* const* layers, int32_t L, const void* x_in, 
     }
     for (int l = 0; l < L; ++l) {
         const spffn_ctx& c = *layers[l];
+        // union path: FC1 derives the table from the mask words (no compaction tail in the
+        // logits launch)
+        const bool tin = !lookahead && union_supported(c, B) && union_fused_compaction(c);
         if (!lookahead) {
-            e = launch_predict(c, xcur, B, c.idx(), c.count(), counts ? counts + l : nullptr, st);
+            e = launch_predict(c, xcur, B, c.idx(), c.count(), counts ? counts + l : nullptr, st, tin);
         } else if (l + 1 < L) {
             // the next layer's set from this layer's input
             const spffn_ctx& cn = *layers[l + 1];
@@ -181,7 +184,8 @@ spffn_status decode_impl(spffn_ctx* const* layers, int32_t L, const void* x_in, 
         }
         if (e != cudaSuccess) return cuda_status(e);
         float* yl = (l == L - 1) ? y : c.ybuf();
-        e = launch_forward(c, xcur, B, c.idx(), c.count(), yl, st);
+        e = launch_forward(c, xcur, B, c.idx(), c.count(), yl, st, tin ? c.idx() : nullptr,
+                           tin && counts ? counts + l : nullptr);
         if (e != cudaSuccess) return cuda_status(e);
         void* xn = (l == L - 1) ? x_out : c.xbuf(l & 1);
         e = launch_chain(c, xcur, yl, B, xn, st);

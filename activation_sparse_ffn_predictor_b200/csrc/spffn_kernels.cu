@@ -567,17 +567,17 @@ cudaError_t launch_compact(const spffn_ctx& c, int32_t* idx, int32_t* count, int
 }
 
 cudaError_t launch_predict(const spffn_ctx& c, const void* x, int B, int32_t* idx, int32_t* count,
-                           int32_t* count2, cudaStream_t st)
+                           int32_t* count2, cudaStream_t st, bool defer_table)
 {
-    if (union_supported(c, B)) return union_predict(c, x, B, idx, count, count2, st);
+    if (union_supported(c, B)) return union_predict(c, x, B, idx, count, count2, st, defer_table);
     return c.cfg.dtype == SPFFN_BF16 ? predict_impl<__nv_bfloat16>(c, x, B, idx, count, count2, st)
                                      : predict_impl<__half>(c, x, B, idx, count, count2, st);
 }
 
 cudaError_t launch_forward(const spffn_ctx& c, const void* x, int B, const int32_t* idx, const int32_t* count,
-                           float* y, cudaStream_t st)
+                           float* y, cudaStream_t st, int32_t* table_out, int32_t* count2)
 {
-    if (union_supported(c, B)) return union_forward(c, x, B, idx, count, y, st);
+    if (union_supported(c, B)) return union_forward(c, x, B, idx, count, y, st, table_out, count2);
     return c.cfg.dtype == SPFFN_BF16 ? forward_impl<__nv_bfloat16>(c, x, B, idx, count, y, st)
                                      : forward_impl<__half>(c, x, B, idx, count, y, st);
 }

@@ -89,6 +89,9 @@ struct alignas(64) UParams {
     int32_t* cidx;        // mode 1, last token group: the CTA finishing last writes the neuron table
     int32_t* ccount;      //   here, its length here and (if not null) in ccount2
     int32_t* ccount2;
+    int32_t* tpriv;       // mode 2, not null: the CTAs rank the mask words themselves, each into its own
+                          //   table copy tpriv[CTA][n], and write the table to cidx and its length to
+                          //   ccount (and ccount2)
     uint32_t* err;
     unsigned long long* trace;   // null, or this launch's [CTA][kUTraceMarks] time stamps
     int cluster;          // > 1: the splits of a tile form one thread-block cluster of this size
@@ -99,11 +102,14 @@ struct alignas(64) UParams {
 // Work decomposition shared by all three roles (same answer in every thread).
 struct Plan {
     int tiles, splits, kblocks, M, K;
+    const int32_t* tab;   // modes 2, 3: the neuron table the rows come from
 };
-__device__ __forceinline__ Plan make_plan(const UParams& p) {
+// Uown >= 0: mode 2's table length as this CTA ranked it from the mask words
+__device__ __forceinline__ Plan make_plan(const UParams& p, int Uown = -1) {
     Plan q;
+    q.tab = p.tpriv ? p.tpriv + (size_t)blockIdx.x * p.n : p.idx;
     if (p.mode == 2) {
-        int U = *reinterpret_cast<const volatile int32_t*>(p.count);
+        int U = Uown >= 0 ? Uown : *reinterpret_cast<const volatile int32_t*>(p.count);
         U = U < 0 ? 0 : (U > p.n ? p.n : U);
         q.M = U;
         q.K = p.K;
@@ -148,7 +154,7 @@ __device__ __forceinline__ int row_pre(const UParams& p, const Plan& q, int tile
     bias = 0.f;
     if (p.mode == 2) {
         if (r >= p.n) return 0;
-        const int j = r < q.M ? p.idx[r] : -1;
+        const int j = r < q.M ? q.tab[r] : -1;
         if ((unsigned)j >= (unsigned)p.n) return 1;
         bias = tof<T>(p.bias, j);
         return 2;
@@ -201,14 +207,17 @@ __device__ void finish_chunk(const UParams& p, int tile, int lane_row, int c0, c
 // the popcounts gives its first slot, and it writes its words' set bits in ascending order.
 constexpr int kCompactWords = 8;   // the fused compaction handles n <= kCompactWords * kUThreads * 32
 
-__device__ void compact_mask_cta(const uint32_t* mask, int words, int32_t* idx, int32_t* count, int32_t* count2,
-                                 uint32_t* wsum)
+// The block scan shared by the compaction and by FC1's own ranking: thread i loads its run
+// of up to kCompactWords mask words (from w0) at once; returns the number of set bits before
+// its run in *first and the total over all words.
+__device__ uint32_t rank_words(const uint32_t* mask, int words, uint32_t (&wv)[kCompactWords], int& w0,
+                               uint32_t* first, uint32_t* wsum)
 {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     constexpr int kWarps = kUThreads / 32;
     const int per = (words + kUThreads - 1) / kUThreads;
-    const int w0 = min(words, tid * per), w1 = min(words, w0 + per);
-    uint32_t wv[kCompactWords];
+    w0 = min(words, tid * per);
+    const int w1 = min(words, w0 + per);
     uint32_t local = 0;
 #pragma unroll
     for (int k = 0; k < kCompactWords; ++k) {
@@ -229,7 +238,17 @@ __device__ void compact_mask_cta(const uint32_t* mask, int words, int32_t* idx, 
         base += k < warp ? wsum[k] : 0u;
         total += wsum[k];
     }
-    uint32_t pos = base + incl - local;
+    *first = base + incl - local;
+    return total;
+}
+
+__device__ void compact_mask_cta(const uint32_t* mask, int words, int32_t* idx, int32_t* count, int32_t* count2,
+                                 uint32_t* wsum)
+{
+    uint32_t wv[kCompactWords];
+    int w0;
+    uint32_t pos;
+    const uint32_t total = rank_words(mask, words, wv, w0, &pos, wsum);
 #pragma unroll
     for (int k = 0; k < kCompactWords; ++k) {
         uint32_t bits = wv[k];
@@ -239,7 +258,7 @@ __device__ void compact_mask_cta(const uint32_t* mask, int words, int32_t* idx, 
             idx[pos++] = (w0 + k) * 32 + b;
         }
     }
-    if (tid == 0) {
+    if (threadIdx.x == 0) {
         *count = (int32_t)total;
         if (count2) *count2 = (int32_t)total;
     }
@@ -287,8 +306,50 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
     // the TMA lane first issues weight tiles, which do not depend on it.
     pdl_trigger();
     if (p.mode >= 2 || (warp != 0 && warp != 1)) pdl_wait();
-    const Plan q = make_plan(p);
-    if (p.mode == 2 && blockIdx.x == 0 && threadIdx.x == 0) {
+    // Mode 2 with its own ranking: every CTA scans the union mask words (left by the logits
+    // launch) and keeps the table entries of its own tiles; the CTA holding split 0 of a tile
+    // also writes that tile's entries to the shared table, and CTA 0 writes the length.
+    uint32_t wv[kCompactWords];
+    int w0 = 0, Uown = -1;
+    uint32_t rank = 0;                       // set bits before this thread's words
+    if (p.mode == 2 && p.tpriv) Uown = (int)rank_words(p.mask, p.n >> 5, wv, w0, &rank, s_wsum);
+    const Plan q = make_plan(p, Uown);
+    if (Uown >= 0) {
+        const int units0 = q.tiles * q.splits, b = blockIdx.x, G = gridDim.x;
+        int32_t* own = p.tpriv + (size_t)b * p.n;
+        // this CTA's units b, b + G, ..: tile u / splits, ranks [tile kBM, tile kBM + kBM); a
+        // thread skips its words outside that window by their popcounts
+        for (int u = b; u < units0; u += G) {
+            const int t = u / q.splits;
+            const bool lead = u % q.splits == 0;
+            const uint32_t lo = (uint32_t)t * kBM, hi = min(lo + kBM, (uint32_t)Uown);
+            uint32_t r = rank;
+#pragma unroll
+            for (int k = 0; k < kCompactWords; ++k) {
+                const uint32_t nb = __popc(wv[k]);
+                if (r + nb <= lo || r >= hi) {
+                    r += nb;
+                    continue;
+                }
+                uint32_t bits = wv[k];
+                while (bits) {
+                    const int j = (w0 + k) * 32 + __ffs(bits) - 1;
+                    bits &= bits - 1;
+                    if (r >= lo && r < hi) {
+                        own[r] = j;
+                        if (lead) p.cidx[r] = j;
+                    }
+                    ++r;
+                }
+            }
+        }
+        if (b == 0 && threadIdx.x == 0) {
+            *p.ccount = Uown;
+            if (p.ccount2) *p.ccount2 = Uown;
+        }
+        __syncthreads();
+    }
+    if (p.mode == 2 && !p.tpriv && blockIdx.x == 0 && threadIdx.x == 0) {
         const int U = *p.count;
         if (U < 0 || U > p.n) atomicOr(p.err, ERR_COUNT_CLAMPED);    // clamped by make_plan
     }
@@ -387,7 +448,7 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int r = kb * kBK + i * 16 + (t >> 4);
-                    int j = r < q.K ? p.idx[r] : 0;
+                    int j = r < q.K ? q.tab[r] : 0;
                     j = (unsigned)j < (unsigned)p.n ? j : 0;
                     rows[i] = reinterpret_cast<const char*>(p.W) + (size_t)j * p.d * 2;
                 }
@@ -403,7 +464,7 @@ __global__ void __launch_bounds__(kUThreads, 1) k_umma(const __grid_constant__ U
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int r = tile * kBM + i * 32 + (t >> 3);
-                        int j = p.idx[r < q.M ? r : 0];
+                        int j = r < q.M ? q.tab[r] : 0;
                         if ((unsigned)j >= (unsigned)p.n) { atomicOr(p.err, ERR_IDX_RANGE); j = 0; }
                         rows[i] = reinterpret_cast<const char*>(p.W) + (size_t)j * p.d * 2 + c * 16;
                     }
@@ -829,8 +890,9 @@ bool union_supported(const spffn_ctx& c, int B) {
 }
 
 cudaError_t union_predict(const spffn_ctx& c, const void* x, int B, int32_t* idx, int32_t* count, int32_t* count2,
-                          cudaStream_t st)
+                          cudaStream_t st, bool defer_table)
 {
+    defer_table = defer_table && union_fused_compaction(c);
     const auto& g = c.cfg;
     const UnionGroups ug = union_groups(B);
     // predictor layer 1: D[H x B] = Wp1 . X^T, split-K, -> h (fp32) and its hi/lo pairs
@@ -869,7 +931,7 @@ cudaError_t union_predict(const spffn_ctx& c, const void* x, int B, int32_t* idx
         q.mask_or = gi > 0;
         q.bias = c.w.bp2;
         q.mask = c.mask();
-        if (gi == ug.groups - 1 && union_fused_compaction(c)) {
+        if (gi == ug.groups - 1 && union_fused_compaction(c) && !defer_table) {
             q.cidx = idx;
             q.ccount = count;
             q.ccount2 = count2;
@@ -884,8 +946,9 @@ cudaError_t union_predict(const spffn_ctx& c, const void* x, int B, int32_t* idx
 }
 
 cudaError_t union_forward(const spffn_ctx& c, const void* x, int B, const int32_t* idx, const int32_t* count,
-                          float* y, cudaStream_t st)
+                          float* y, cudaStream_t st, int32_t* table_out, int32_t* count2)
 {
+    if (table_out && (table_out != idx || !union_fused_compaction(c))) return cudaErrorInvalidValue;
     const auto& g = c.cfg;
     const UnionGroups ug = union_groups(B);
     // FC1 over the table rows: D[U x B] = W1[table] . X^T -> a (hi/lo pairs), zeros past U
@@ -896,6 +959,13 @@ cudaError_t union_forward(const spffn_ctx& c, const void* x, int B, const int32_
     p.Gs = ug.Gt;
     p.count = count;
     p.idx = idx;
+    if (table_out) {
+        p.mask = c.mask();
+        p.tpriv = c.utab();
+        p.cidx = table_out;
+        p.ccount = const_cast<int32_t*>(count);
+        p.ccount2 = count2;
+    }
     p.bias = c.w.b1;
     p.out_split = c.asplit();
     p.W = c.w.W1;

@@ -150,9 +150,9 @@ def dense_bytes_per_layer(cfg) -> int:
 # captured on: any change to them and the bench reports null.
 DECODE_SOURCES = ("spffn_fused.cu", "spffn_fused.cuh", "spffn_internal.cuh")
 DECODE_TRAFFIC = {
-    "sha256": "5b152be61b162ed9f937ae1f502a918d77ee3bb4bdae983212fbe102c4e2ae55",
+    "sha256": "0c61c2bd06d4ce768ff9b8b7c12e6c676bbcb2829f49c481448ec202ddb0ee79",
     "workload": "opt6.7b-d4096-n16384-L32", "batch": 1, "rate": 0.05,
-    "bytes_per_layer": (222.192896e6 + 4.515328e6) / 4,
+    "bytes_per_layer": (222.220544e6 + 4.9152e6) / 4,
 }
 
 
@@ -163,10 +163,10 @@ DECODE_TRAFFIC = {
 # only for the kernel sources it was captured on: any change to them and the bench reports null.
 UNION_SOURCES = ("spffn_union.cu", "spffn_umma.cuh", "spffn_internal.cuh", "spffn_kernels.cu")
 UNION_TRAFFIC = {
-    "sha256": "4046e3abdb096feab4cd092b4cf9d8e4c0097e3d3ef40e7ef43645850049a054",
+    "sha256": "a33d7a16b83a54096f631f2d9ccafedbeb675db8b306cc3998d69452248e8a43",
     "workload": "opt66b-d9216-n36864-L64", "batch": 32, "rate": 0.01,
-    "fixed_per_layer": 38.44e6 + 152.02e6 + 1.78e6,
-    "per_neuron": (105.12e6 + 105.33e6) / 5639.17,
+    "fixed_per_layer": 38.435e6 + 152.19e6 + 1.78e6,
+    "per_neuron": (105.245e6 + 105.32e6) / 5639.17,
 }
 
 

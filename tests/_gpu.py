@@ -33,7 +33,7 @@ def rel_l2(got, want):
 
 
 def check_y(got, want, internal=Y_INTERNAL_BAR):
-    """The benchmark spec's bound on every token (rows of [B, d]) plus the tighter
+    """The 1e-3 relative-L2 bound on every token (rows of [B, d]) plus the tighter
     internal bar on the whole tensor; returns the whole-tensor error."""
     got = np.atleast_2d(np.asarray(got, dtype=np.float64))
     want = np.atleast_2d(np.asarray(want, dtype=np.float64))
